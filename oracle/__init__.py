@@ -1,0 +1,231 @@
+"""Plain CPU oracle for the Ulysses attention layer -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline / reference arm may import this package.  The product path (the CUDA
+library and its binding) never imports, links or executes anything here.
+
+The arithmetic lives in ``ulysses_oracle.c`` (plain loops, fp64, OpenMP over
+independent rows); this module only builds it with gcc and marshals numpy
+arrays.  It shares no code with the CUDA path.  Every function is pinned by
+tests under ``tests/`` against closed forms, brute force, invariants, library
+routines and finite differences.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ulysses_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+MASK_NONE, MASK_CAUSAL, MASK_DOC_CAUSAL = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, OpenMP, -O3)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O3", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
+               "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            i, l, dbl = ctypes.c_int, ctypes.c_long, ctypes.c_double
+            lib.oracle_seq_to_head.argtypes = [i, i, i, i, l, P, P]
+            lib.oracle_head_to_seq.argtypes = [i, i, i, i, l, P, P]
+            attn = [i, i, i, i, i, i, P, i, dbl]
+            lib.oracle_attention_fwd.argtypes = attn + [P, P, P, P, P]
+            lib.oracle_attention_bwd.argtypes = attn + [P, P, P, P, P, P, P]
+            uly = [i, i, i, i, i, i, i, P, i, dbl]
+            lib.oracle_ulysses_fwd.argtypes = uly + [P, P, P, P, P]
+            lib.oracle_ulysses_bwd.argtypes = uly + [P, P, P, P, P, P, P]
+            lib.oracle_head_rows.argtypes = [i, i, i, P, i, dbl, P, P, P, P, P, i, P, P, P]
+            lib.oracle_kv_cols.argtypes = [i, i, i, P, i, dbl, i, P, P, P, P, P, i, P, P]
+            lib.oracle_loss.argtypes = [i, l, i, P, P, i, P, P, P]
+            lib.oracle_loss.restype = l
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else ctypes.c_void_p(0)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _check_ulysses(n, P, H, G):
+    """Divisibility the method needs: n % P (every rank holds n/P positions),
+    H % P and G % P (every rank owns whole heads), H % G (GQA groups)."""
+    if P <= 0 or n % P or H % P or G % P or H % G:
+        raise ValueError(f"need n%P == H%P == G%P == H%G == 0, got n={n} P={P} H={H} G={G}")
+
+
+def _cu(cu_seqlens):
+    if cu_seqlens is None:
+        return None, 0
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    return cu, int(cu.size - 1)
+
+
+# --------------------------------------------------------------------------
+# Steps 1, 3, 5: sharding and the two all-to-alls (byte-exact, any dtype)
+# --------------------------------------------------------------------------
+
+def seq_to_head(x: np.ndarray, B: int, n: int, P: int, heads: int) -> np.ndarray:
+    """[P][B][n/P][heads][d] -> [P][B][heads/P][n][d] (any dtype, byte copy)."""
+    x = np.ascontiguousarray(x)
+    d = x.size // (B * n * heads)
+    out = np.empty(P * B * (heads // P) * n * d, dtype=x.dtype)
+    _load().oracle_seq_to_head(B, n, P, heads, d * x.itemsize, _ptr(x), _ptr(out))
+    return out.reshape(P, B, heads // P, n, d)
+
+
+def head_to_seq(x: np.ndarray, B: int, n: int, P: int, heads: int) -> np.ndarray:
+    """[P][B][heads/P][n][d] -> [P][B][n/P][heads][d] (any dtype, byte copy)."""
+    x = np.ascontiguousarray(x)
+    d = x.size // (B * n * heads)
+    out = np.empty(P * B * (n // P) * heads * d, dtype=x.dtype)
+    _load().oracle_head_to_seq(B, n, P, heads, d * x.itemsize, _ptr(x), _ptr(out))
+    return out.reshape(P, B, n // P, heads, d)
+
+
+# --------------------------------------------------------------------------
+# Step 4: plain full-sequence GQA attention on the natural layout [B][n][H][d]
+# --------------------------------------------------------------------------
+
+def attention_fwd(q, k, v, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+    """O [B][n][H][d] (fp64) and LSE [B][H][n] of plain multi-head GQA attention."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, n, H, d = q.shape
+    G = k.shape[2]
+    cu, nd = _cu(cu_seqlens)
+    o = np.empty((B, n, H, d), np.float64)
+    lse = np.empty((B, H, n), np.float64)
+    _load().oracle_attention_fwd(B, n, H, G, d, mask, _ptr(cu), nd, scale,
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def attention_bwd(q, k, v, dout, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+    """dQ, dK, dV (fp64, natural layout) of sum(O * dO)."""
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, n, H, d = q.shape
+    G = k.shape[2]
+    cu, nd = _cu(cu_seqlens)
+    dq = np.empty((B, n, H, d), np.float64)
+    dk = np.empty((B, n, G, d), np.float64)
+    dv = np.empty((B, n, G, d), np.float64)
+    _load().oracle_attention_bwd(B, n, H, G, d, mask, _ptr(cu), nd, scale,
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                                 _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
+# --------------------------------------------------------------------------
+# The explicit Ulysses procedure (seq layout in and out)
+# --------------------------------------------------------------------------
+
+def ulysses_fwd(q_seq, k_seq, v_seq, P, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+    """q_seq [P][B][s][H][d], k/v_seq [P][B][s][G][d] -> O_seq [P][B][s][H][d]
+    (fp64) and LSE in head layout [P][B][H/P][n]."""
+    q, k, v = _f32(q_seq), _f32(k_seq), _f32(v_seq)
+    _, B, s, H, d = q.shape
+    G = k.shape[3]
+    n = P * s
+    _check_ulysses(n, P, H, G)
+    cu, nd = _cu(cu_seqlens)
+    o = np.empty((P, B, s, H, d), np.float64)
+    lse = np.empty((P, B, H // P, n), np.float64)
+    _load().oracle_ulysses_fwd(B, n, P, H, G, d, mask, _ptr(cu), nd, scale,
+                               _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def ulysses_bwd(q_seq, k_seq, v_seq, do_seq, P, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+    """dQ_seq, dK_seq, dV_seq (fp64, seq layout) of sum(O * dO)."""
+    q, k, v, do = _f32(q_seq), _f32(k_seq), _f32(v_seq), _f32(do_seq)
+    _, B, s, H, d = q.shape
+    G = k.shape[3]
+    n = P * s
+    _check_ulysses(n, P, H, G)
+    cu, nd = _cu(cu_seqlens)
+    dq = np.empty((P, B, s, H, d), np.float64)
+    dk = np.empty((P, B, s, G, d), np.float64)
+    dv = np.empty((P, B, s, G, d), np.float64)
+    _load().oracle_ulysses_bwd(B, n, P, H, G, d, mask, _ptr(cu), nd, scale,
+                               _ptr(q), _ptr(k), _ptr(v), _ptr(do),
+                               _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
+# --------------------------------------------------------------------------
+# Exact values at sampled rows / key columns (large workloads)
+# --------------------------------------------------------------------------
+
+def head_rows(q, k, v, rows, dout=None, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+    """One query head q [n][d] with its KV head k, v [n][d]: exact O, LSE (and
+    dQ if dout is given) at the listed query rows."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    n, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    cu, nd = _cu(cu_seqlens)
+    o = np.empty((rows.size, d), np.float64)
+    lse = np.empty(rows.size, np.float64)
+    dq = np.empty((rows.size, d), np.float64) if dout is not None else None
+    dout = _f32(dout) if dout is not None else None
+    _load().oracle_head_rows(n, d, mask, _ptr(cu), nd, scale, _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(dout), _ptr(rows), rows.size, _ptr(o), _ptr(lse), _ptr(dq))
+    return (o, lse, dq) if dout is not None else (o, lse)
+
+
+def kv_cols(qs, douts, k, v, cols, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+    """One KV head k, v [n][d] and its query heads qs[e], douts[e] [n][d]:
+    exact dK, dV at the listed key columns, summed over the query heads."""
+    qs = [_f32(x) for x in qs]
+    douts = [_f32(x) for x in douts]
+    k, v = _f32(k), _f32(v)
+    n, d = k.shape
+    cols = np.ascontiguousarray(cols, dtype=np.int32)
+    cu, nd = _cu(cu_seqlens)
+    qp = (ctypes.c_void_p * len(qs))(*[x.ctypes.data for x in qs])
+    dp = (ctypes.c_void_p * len(douts))(*[x.ctypes.data for x in douts])
+    dk = np.empty((cols.size, d), np.float64)
+    dv = np.empty((cols.size, d), np.float64)
+    _load().oracle_kv_cols(n, d, mask, _ptr(cu), nd, scale, len(qs),
+                           ctypes.cast(qp, ctypes.c_void_p), ctypes.cast(dp, ctypes.c_void_p),
+                           _ptr(k), _ptr(v), _ptr(cols), cols.size, _ptr(dk), _ptr(dv))
+    return dk, dv
+
+
+# --------------------------------------------------------------------------
+# Token-weighted loss aggregation
+# --------------------------------------------------------------------------
+
+def loss_aggregate(logits, labels, P, ignore_index=-100):
+    """logits [T][V] (shard r = rows [r*T/P, (r+1)*T/P)), labels [T] ->
+    (S [P] fp64, C [P] int64, L fp64, number of bad labels)."""
+    z = _f32(logits)
+    T, V = z.shape
+    y = np.ascontiguousarray(labels, dtype=np.int32)
+    S = np.empty(P, np.float64)
+    C = np.empty(P, np.int64)
+    L = np.empty(1, np.float64)
+    bad = _load().oracle_loss(P, T, V, _ptr(z), _ptr(y), ignore_index, _ptr(S), _ptr(C), _ptr(L))
+    return S, C, float(L[0]), int(bad)
