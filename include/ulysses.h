@@ -1,0 +1,164 @@
+/*
+ * ulysses.h -- C ABI of the single-GPU Ulysses attention layer (sm_100a).
+ *
+ * The method (Ulysses sequence parallelism):
+ *   "Paralelismul de Secvență Ulysses: Antrenarea modelelor AI cu contexte de
+ *    un milion de token-uri", section "Mecanismul de funcționare Ulysses",
+ *    steps 1-6, and "Ulysses 序列平行化：突破百萬標記長上下文的訓練瓶頸",
+ *    section "Ulysses 序列平行化的原理": the sequence is split over P ranks
+ *   (rank r holds positions [r*n/P, (r+1)*n/P)); a first all-to-all gives
+ *   every rank all n positions of H/P heads; each rank runs ordinary attention
+ *   on its heads; a second all-to-all restores the sequence split.  The loss
+ *   is aggregated over ranks weighted by each rank's count of valid tokens
+ *   (same page, section "Integrarea cu Accelerate").
+ *
+ * Here the P ranks are logical: all of them live in one GPU's memory and the
+ * two all-to-alls are layout permutations inside HBM.
+ *
+ * Layouts (row = head_dim contiguous elements):
+ *   seq layout   X[P][B][n/P][heads][head_dim]   (rank-major stack of the
+ *                per-rank [B][n/P][heads][d] buffers; for B = 1 this is the
+ *                natural [n][heads][d] order)
+ *   head layout  X[P][B][heads/P][n][head_dim]   (rank r holds heads
+ *                [r*heads/P, (r+1)*heads/P) for all n positions)
+ *   LSE          float[P][B][H/P][n] (natural log of the softmax denominator)
+ * GQA: query head q uses KV head floor(q / (H/G)); rank r holds query heads
+ * [r*H/P, (r+1)*H/P) and KV heads [r*G/P, (r+1)*G/P), so every rank's query
+ * heads find their KV heads locally (needs H % P == G % P == H % G == 0).
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees device memory.  `stream` is a cudaStream_t (or
+ *    NULL for the legacy default stream) passed as void*.
+ *  - Every call is asynchronous on `stream`; nothing synchronises the host.
+ *  - Errors detectable from the arguments are returned before any launch and
+ *    then nothing is launched.  Data-dependent errors (a bad label, a bounded
+ *    wait that ran out) are OR-ed as (1 << status) into a device error word,
+ *    read with ulysses_read_error(); kernels never trap.
+ *  - Pointers must be 16-byte aligned and rows (head_dim * element bytes) a
+ *    multiple of 16 bytes.  Inputs and outputs must not overlap.
+ */
+#ifndef ULYSSES_H
+#define ULYSSES_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ULY_OK = 0,
+  ULY_ERR_NULL = 1,        /* a required pointer is NULL                          */
+  ULY_ERR_SHAPE = 2,       /* n % P, H % P, G % P, H % G, non-positive sizes     */
+  ULY_ERR_DTYPE = 3,       /* unknown dtype / element size                        */
+  ULY_ERR_ALIGN = 4,       /* pointer or row not 16-byte aligned                  */
+  ULY_ERR_ALIAS = 5,       /* input and output ranges overlap                     */
+  ULY_ERR_UNSUPPORTED = 6, /* valid but not implemented (e.g. bf16 head_dim!=128)*/
+  ULY_ERR_CUDA = 7,        /* a CUDA runtime call failed                          */
+  ULY_ERR_LABEL = 8,       /* async: a label outside [0, V) and != ignore_index   */
+  ULY_ERR_TIMEOUT = 9,     /* async: a bounded wait inside a kernel ran out       */
+  ULY_ERR_WORKSPACE = 10   /* workspace missing or smaller than required          */
+} uly_status;
+
+typedef enum { ULY_F32 = 0, ULY_BF16 = 1 } uly_dtype;
+
+typedef enum {
+  ULY_MASK_NONE = 0,       /* every key visible                                   */
+  ULY_MASK_CAUSAL = 1,     /* key j visible to query i iff j <= i                 */
+  ULY_MASK_DOC_CAUSAL = 2  /* causal and same document (packed sequences)         */
+} uly_mask;
+
+/* Shape of one Ulysses attention layer (all P logical ranks at once). */
+typedef struct {
+  int32_t batch;           /* B                                                   */
+  int32_t seq_len;         /* n (global, all ranks); n % world == 0               */
+  int32_t world;           /* P logical ranks                                     */
+  int32_t n_q_heads;       /* H                                                   */
+  int32_t n_kv_heads;      /* G (GQA); H % G == 0                                 */
+  int32_t head_dim;        /* d: f32 supports 64 and 128, bf16 supports 128       */
+  int32_t dtype;           /* uly_dtype of q, k, v, o, dout, dq, dk, dv           */
+  int32_t mask;            /* uly_mask                                            */
+  const int32_t *cu_seqlens; /* DEVICE int32[num_docs+1], doc-causal only: document
+                              * e covers positions [cu[e], cu[e+1]); cu[0] = 0 and
+                              * cu[num_docs] = n; shared by all batch rows        */
+  int32_t num_docs;
+  float softmax_scale;     /* 0 => 1/sqrt(head_dim)                               */
+} uly_attn_desc;
+
+/*
+ * First all-to-all (step 3): seq layout -> head layout.
+ * src: [P][B][n/P][heads][head_dim], dst: [P][B][heads/P][n][head_dim]; the
+ * element type is opaque (elem_bytes in {1,2,4,8}); the copy is bit-exact.
+ * Requires n % P == 0, heads % P == 0, head_dim * elem_bytes % 16 == 0.
+ */
+uly_status ulysses_seq_to_head(int32_t batch, int32_t seq_len, int32_t world, int32_t heads,
+                               int32_t head_dim, int32_t elem_bytes, const void *src,
+                               void *dst, void *stream);
+
+/* Second all-to-all (step 5): head layout -> seq layout; exact inverse of
+ * ulysses_seq_to_head, same arguments and rules. */
+uly_status ulysses_head_to_seq(int32_t batch, int32_t seq_len, int32_t world, int32_t heads,
+                               int32_t head_dim, int32_t elem_bytes, const void *src,
+                               void *dst, void *stream);
+
+/*
+ * Local attention (step 4) of every logical rank, head layout in and out:
+ * q, o [P][B][H/P][n][d]; k, v [P][B][G/P][n][d]; lse [P][B][H/P][n] (fp32).
+ * O = softmax(scale * Q K^T + mask) V per query head, LSE its log-sum-exp.
+ * bf16: tensor-core path (fp32 accumulation), needs head_dim == 128 and an
+ * even number of query heads per KV head.  f32: exact-fp32 SIMT path.
+ */
+uly_status ulysses_attn_fwd(const uly_attn_desc *desc, const void *q, const void *k,
+                            const void *v, void *o, float *lse, void *stream);
+
+/* Bytes of device workspace ulysses_attn_bwd needs for this shape. */
+uly_status ulysses_attn_bwd_workspace_size(const uly_attn_desc *desc, size_t *bytes);
+
+/*
+ * Backward of the local attention (gradients of sum(O * dO)), head layout:
+ * dout, dq like q; dk, dv like k (summed over the query heads of each KV
+ * head); o and lse are the forward's outputs.  `workspace` must hold
+ * ulysses_attn_bwd_workspace_size() bytes (caller owned, 256-byte aligned).
+ */
+uly_status ulysses_attn_bwd(const uly_attn_desc *desc, const void *q, const void *k,
+                            const void *v, const void *o, const float *lse, const void *dout,
+                            void *dq, void *dk, void *dv, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace ulysses_loss_aggregate needs. */
+uly_status ulysses_loss_workspace_size(int32_t world, int64_t tokens, int32_t vocab,
+                                       size_t *bytes);
+
+/*
+ * Token-weighted cross-entropy over the P shards ("Integrarea cu Accelerate":
+ * weight every rank's loss by its count of valid tokens):
+ *   l_t = logsumexp(z_t) - z_t[y_t] for every token with y_t != ignore_index,
+ *   shard_sum[r] = sum of l_t over shard r, shard_count[r] = its valid count,
+ *   *loss = sum_r shard_sum[r] / sum_r shard_count[r]  (NaN if no valid token).
+ * logits: [P][tokens/P][vocab] (ULY_BF16 or ULY_F32), labels int32 [P][tokens/P].
+ * Needs tokens % P == 0.  A label outside [0, vocab) that is not ignore_index
+ * sets ULY_ERR_LABEL in the error word and is not counted.  The reduction order
+ * is fixed, so repeated calls give bitwise-equal results.
+ */
+uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab,
+                                  int32_t logit_dtype, const void *logits,
+                                  const int32_t *labels, int32_t ignore_index,
+                                  float *shard_sum, int64_t *shard_count, float *loss,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* Asynchronous error word of the current device: reads it (synchronising the
+ * device) into *word (bit s set <=> status s was raised) and clears it. */
+uly_status ulysses_read_error(int32_t *word);
+
+/* Human-readable name of a status. */
+const char *ulysses_status_string(uly_status status);
+
+/* Number of kernels launched by this process through the library so far. */
+uint64_t ulysses_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ULYSSES_H */

@@ -1,0 +1,255 @@
+// C ABI of the Ulysses attention layer: argument validation and dispatch to
+// the kernels.  Declarations and the contract of every entry point are in
+// include/ulysses.h.  Nothing here allocates device memory.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace uly {
+
+// Device error word, one per device context (module globals are per context).
+__device__ int g_error_word_storage = 0;
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_err_mu;
+int *g_err_ptr[64] = {nullptr};
+}  // namespace
+
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int *error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word_storage) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+// launchers implemented in the kernel translation units
+uly_status permute_validate(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *,
+                            const void *);
+uly_status permute_launch(bool, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *,
+                          void *, cudaStream_t);
+uly_status attn_f32_fwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
+                               const void *, const void *, const void *, void *, float *,
+                               cudaStream_t);
+uly_status attn_f32_bwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
+                               const void *, const void *, const void *, const void *,
+                               const float *, const void *, void *, void *, void *, float *,
+                               cudaStream_t);
+uly_status attn_bf16_fwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
+                                const void *, const void *, const void *, void *, float *,
+                                cudaStream_t);
+uly_status attn_bf16_bwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
+                                const void *, const void *, const void *, const void *,
+                                const float *, const void *, void *, void *, void *, float *,
+                                cudaStream_t);
+size_t loss_workspace_bytes(int P, long long per_shard);
+uly_status loss_validate(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *,
+                         const float *, const int64_t *, const float *);
+uly_status loss_launch(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *, int32_t,
+                       float *, int64_t *, float *, void *, cudaStream_t);
+
+namespace {
+
+uly_status check_desc(const uly_attn_desc *d, HeadGeom &g, MaskInfo &mk) {
+  if (!d) return ULY_ERR_NULL;
+  if (d->batch <= 0 || d->seq_len <= 0 || d->world <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 ||
+      d->head_dim <= 0)
+    return ULY_ERR_SHAPE;
+  if (d->seq_len % d->world || d->n_q_heads % d->world || d->n_kv_heads % d->world ||
+      d->n_q_heads % d->n_kv_heads)
+    return ULY_ERR_SHAPE;
+  if (d->dtype != ULY_F32 && d->dtype != ULY_BF16) return ULY_ERR_DTYPE;
+  if (d->mask < ULY_MASK_NONE || d->mask > ULY_MASK_DOC_CAUSAL) return ULY_ERR_UNSUPPORTED;
+  if (d->mask == ULY_MASK_DOC_CAUSAL && (!d->cu_seqlens || d->num_docs < 1)) return ULY_ERR_NULL;
+  if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return ULY_ERR_SHAPE;
+  const long long heads_q = (long long)d->batch * d->n_q_heads;
+  if (heads_q > 65535 || (d->seq_len + 63) / 64 > 65535) return ULY_ERR_SHAPE;  // grid limits
+  if (d->dtype == ULY_F32 && d->head_dim != 64 && d->head_dim != 128) return ULY_ERR_UNSUPPORTED;
+  if (d->dtype == ULY_BF16 && (d->head_dim != 128 || (d->n_q_heads / d->n_kv_heads) % 2 != 0))
+    return ULY_ERR_UNSUPPORTED;
+  g.B = d->batch;
+  g.n = d->seq_len;
+  g.P = d->world;
+  g.hl = d->n_q_heads / d->world;
+  g.gl = d->n_kv_heads / d->world;
+  g.group = d->n_q_heads / d->n_kv_heads;
+  g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)d->head_dim);
+  mk.mask = d->mask;
+  mk.n = d->seq_len;
+  mk.cu = d->cu_seqlens;
+  mk.num_docs = d->num_docs;
+  return ULY_OK;
+}
+
+size_t elem_bytes(int dtype) { return dtype == ULY_BF16 ? 2 : 4; }
+size_t q_bytes(const uly_attn_desc *d) {
+  return (size_t)d->batch * d->seq_len * d->n_q_heads * d->head_dim * elem_bytes(d->dtype);
+}
+size_t kv_bytes(const uly_attn_desc *d) {
+  return (size_t)d->batch * d->seq_len * d->n_kv_heads * d->head_dim * elem_bytes(d->dtype);
+}
+size_t lse_bytes(const uly_attn_desc *d) {
+  return (size_t)d->batch * d->seq_len * d->n_q_heads * sizeof(float);
+}
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool all_aligned(std::initializer_list<const void *> ps) {
+  for (const void *p : ps)
+    if (!aligned16(p)) return false;
+  return true;
+}
+
+}  // namespace
+}  // namespace uly
+
+using namespace uly;
+
+extern "C" {
+
+uly_status ulysses_seq_to_head(int32_t batch, int32_t seq_len, int32_t world, int32_t heads,
+                               int32_t head_dim, int32_t eb, const void *src, void *dst,
+                               void *stream) {
+  uly_status st = permute_validate(batch, seq_len, world, heads, head_dim, eb, src, dst);
+  if (st != ULY_OK) return st;
+  return permute_launch(true, batch, seq_len, world, heads, head_dim, eb, src, dst,
+                        static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_head_to_seq(int32_t batch, int32_t seq_len, int32_t world, int32_t heads,
+                               int32_t head_dim, int32_t eb, const void *src, void *dst,
+                               void *stream) {
+  uly_status st = permute_validate(batch, seq_len, world, heads, head_dim, eb, src, dst);
+  if (st != ULY_OK) return st;
+  return permute_launch(false, batch, seq_len, world, heads, head_dim, eb, src, dst,
+                        static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_attn_fwd(const uly_attn_desc *d, const void *q, const void *k, const void *v,
+                            void *o, float *lse, void *stream) {
+  HeadGeom g;
+  MaskInfo mk;
+  uly_status st = check_desc(d, g, mk);
+  if (st != ULY_OK) return st;
+  if (!q || !k || !v || !o || !lse) return ULY_ERR_NULL;
+  if (!all_aligned({q, k, v, o, lse})) return ULY_ERR_ALIGN;
+  const size_t qb = q_bytes(d), kb = kv_bytes(d), lb = lse_bytes(d);
+  for (const void *in : {q, k, v}) {
+    const size_t ib = (in == q) ? qb : kb;
+    if (overlap(in, ib, o, qb) || overlap(in, ib, lse, lb)) return ULY_ERR_ALIAS;
+  }
+  if (overlap(o, qb, lse, lb)) return ULY_ERR_ALIAS;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->dtype == ULY_F32) return attn_f32_fwd_launch(d, g, mk, q, k, v, o, lse, s);
+  return attn_bf16_fwd_launch(d, g, mk, q, k, v, o, lse, s);
+}
+
+uly_status ulysses_attn_bwd_workspace_size(const uly_attn_desc *d, size_t *bytes) {
+  HeadGeom g;
+  MaskInfo mk;
+  if (!bytes) return ULY_ERR_NULL;
+  uly_status st = check_desc(d, g, mk);
+  if (st != ULY_OK) return st;
+  *bytes = align256(lse_bytes(d));  // D_i = <dO_i, O_i> for every query row
+  return ULY_OK;
+}
+
+uly_status ulysses_attn_bwd(const uly_attn_desc *d, const void *q, const void *k, const void *v,
+                            const void *o, const float *lse, const void *dout, void *dq, void *dk,
+                            void *dv, void *workspace, size_t workspace_bytes, void *stream) {
+  HeadGeom g;
+  MaskInfo mk;
+  uly_status st = check_desc(d, g, mk);
+  if (st != ULY_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ULY_ERR_NULL;
+  size_t need = 0;
+  ulysses_attn_bwd_workspace_size(d, &need);
+  if (!workspace || workspace_bytes < need) return ULY_ERR_WORKSPACE;
+  if (!all_aligned({q, k, v, o, lse, dout, dq, dk, dv, workspace})) return ULY_ERR_ALIGN;
+  const size_t qb = q_bytes(d), kb = kv_bytes(d), lb = lse_bytes(d);
+  const void *ins[6] = {q, k, v, o, lse, dout};
+  const size_t inb[6] = {qb, kb, kb, qb, lb, qb};
+  void *outs[4] = {dq, dk, dv, workspace};
+  const size_t outb[4] = {qb, kb, kb, need};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlap(outs[a], outb[a], ins[b], inb[b])) return ULY_ERR_ALIAS;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlap(outs[a], outb[a], outs[b], outb[b])) return ULY_ERR_ALIAS;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *Dv = static_cast<float *>(workspace);
+  if (d->dtype == ULY_F32)
+    return attn_f32_bwd_launch(d, g, mk, q, k, v, o, lse, dout, dq, dk, dv, Dv, s);
+  return attn_bf16_bwd_launch(d, g, mk, q, k, v, o, lse, dout, dq, dk, dv, Dv, s);
+}
+
+uly_status ulysses_loss_workspace_size(int32_t world, int64_t tokens, int32_t vocab, size_t *bytes) {
+  if (!bytes) return ULY_ERR_NULL;
+  if (world <= 0 || tokens < 0 || vocab <= 0 || tokens % world) return ULY_ERR_SHAPE;
+  *bytes = align256(loss_workspace_bytes(world, tokens / world));
+  return ULY_OK;
+}
+
+uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab, int32_t logit_dtype,
+                                  const void *logits, const int32_t *labels, int32_t ignore_index,
+                                  float *shard_sum, int64_t *shard_count, float *loss,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+  uly_status st = loss_validate(world, tokens, vocab, logit_dtype, logits, labels, shard_sum,
+                                shard_count, loss);
+  if (st != ULY_OK) return st;
+  size_t need = 0;
+  ulysses_loss_workspace_size(world, tokens, vocab, &need);
+  if (!workspace || workspace_bytes < need) return ULY_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ULY_ERR_ALIGN;
+  const size_t zb = (size_t)tokens * vocab * (logit_dtype == ULY_BF16 ? 2 : 4);
+  const size_t yb = (size_t)tokens * 4;
+  const void *outs[4] = {shard_sum, shard_count, loss, workspace};
+  const size_t outb[4] = {(size_t)world * 4, (size_t)world * 8, 4, need};
+  for (int a = 0; a < 4; ++a)
+    if (overlap(outs[a], outb[a], logits, zb) || overlap(outs[a], outb[a], labels, yb))
+      return ULY_ERR_ALIAS;
+  return loss_launch(world, tokens, vocab, logit_dtype, logits, labels, ignore_index, shard_sum,
+                     shard_count, loss, workspace, static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_read_error(int32_t *word) {
+  if (!word) return ULY_ERR_NULL;
+  int *p = error_word();
+  if (!p) return ULY_ERR_CUDA;
+  int host = 0, zero = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ULY_ERR_CUDA;
+  if (cudaMemcpy(&host, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ULY_ERR_CUDA;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ULY_ERR_CUDA;
+  *word = host;
+  return ULY_OK;
+}
+
+const char *ulysses_status_string(uly_status s) {
+  switch (s) {
+    case ULY_OK: return "ok";
+    case ULY_ERR_NULL: return "null pointer";
+    case ULY_ERR_SHAPE: return "invalid shape";
+    case ULY_ERR_DTYPE: return "invalid dtype";
+    case ULY_ERR_ALIGN: return "misaligned pointer or row";
+    case ULY_ERR_ALIAS: return "input and output overlap";
+    case ULY_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ULY_ERR_CUDA: return "CUDA runtime error";
+    case ULY_ERR_LABEL: return "label out of range";
+    case ULY_ERR_TIMEOUT: return "bounded wait timed out";
+    case ULY_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+uint64_t ulysses_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

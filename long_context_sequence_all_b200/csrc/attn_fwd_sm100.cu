@@ -1,0 +1,390 @@
+// Local attention forward of every logical rank on the 5th-generation tensor
+// cores (Ulysses step 4: "Paralelismul de Secvență Ulysses", section
+// "Mecanismul de funcționare Ulysses"; each rank runs ordinary attention on
+// its heads over all n positions).  bf16 inputs, fp32 accumulation, head_dim
+// 128, causal / doc-causal / no mask, GQA.
+//
+// One CTA = two 128-row query tiles at the same positions m0..m0+127 of two
+// query heads of one GQA group, so both tiles read the same K/V tiles and see
+// the same mask: K/V are loaded once for 256 query rows.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tiles once, then K_j, V_j into a 3-slot ring
+//   warp 1      TMEM allocator and MMA issuer (one thread):
+//                 S_t = Q_t K_j^T          (M=128 N=128 K=128, SS, into TMEM)
+//                 O_t += P_t V_j           (M=128 N=128 K=128, SS, into TMEM)
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread
+//               per query row reads its S row from TMEM, keeps the running
+//               max / sum, writes P (bf16) to shared memory in the MMA's
+//               swizzled layout, rescales O in TMEM when the max moved by more
+//               than 2^8, and finally normalises O and writes O and LSE.
+// TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512) columns.
+//
+// Ordering: s_full[t] is committed after S_j(t), which is issued after
+// O_t += P_{j-1} V_{j-1}; a commit tracks every earlier MMA of the thread, so
+// when softmax sees S_j it also knows the previous PV finished (O may be
+// rescaled, P may be overwritten).  p_full[t] hands P_j back to the MMA warp.
+// Every wait is bounded (ULY_ERR_TIMEOUT), no wait can spin forever.
+#include "sm100.cuh"
+
+namespace uly {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kBM = 128, kBN = 128, kHD = 128;
+constexpr int kThreads = 384;
+constexpr int kSlots = 3;
+constexpr uint32_t kTileBytes = 128 * 128 * 2;       // one 128 x 128 bf16 tile
+constexpr uint32_t kOffQ = 0;                        // 2 tiles
+constexpr uint32_t kOffP = 2 * kTileBytes;           // 2 tiles
+constexpr uint32_t kOffKV = 4 * kTileBytes;          // kSlots tiles
+constexpr uint32_t kOffBar = kOffKV + kSlots * kTileBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;            // log2 units
+
+constexpr uint32_t kIdescS = sm100::idesc_bf16_f32(128, 128, false, false);   // Q K^T
+constexpr uint32_t kIdescPV = sm100::idesc_bf16_f32(128, 128, false, true);   // P V (V MN-major)
+
+struct FwdParams {
+  __nv_bfloat16 *o;
+  float *lse;
+  HeadGeom g;
+  MaskInfo mk;
+  float scale_log2;  // softmax scale * log2(e)
+  int *err;          // device error word
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                          const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const FwdParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  // barrier indices
+  enum { B_Q = 0, B_KVF = 1, B_KVE = 1 + kSlots, B_SF = 1 + 2 * kSlots, B_PF = B_SF + 2,
+         B_OF = B_PF + 2, B_DRAIN = B_OF + 2, B_N = B_DRAIN + 1 };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const HeadGeom &g = prm.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = g.hl >> 1;
+  const int pair = blockIdx.x;                   // (r*B + b) * (hl/2) + pp
+  const int rb = pair / half, pp = pair - rb * half;
+  const int qhead0 = rb * g.hl + 2 * pp;         // tiles: qhead0, qhead0 + 1
+  const int kvhead = rb * g.gl + (2 * pp) / g.group;
+  const int mt = gridDim.y - 1 - blockIdx.y;     // heaviest (latest) query tiles first
+  const int m0 = mt * kBM;
+
+  // KV tiles this query tile touches, and which of them need element masks.
+  int lo_first, hi_first, lo_last, hi_last;
+  prm.mk.row_range(m0, lo_first, hi_first);
+  prm.mk.row_range(min(m0 + kBM - 1, g.n - 1), lo_last, hi_last);
+  const int jt0 = lo_first / kBN;
+  const int NT = (hi_last >= lo_first) ? hi_last / kBN - jt0 + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_N; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_PF || i == B_PF + 1) cnt = 128;
+      mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0 && NT > 0) {
+      mbar_arrive_expect_tx(bar(B_Q), 2 * kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(sb + kOffQ + t * kTileBytes + c * 16384, &tmQ, bar(B_Q), c * 64, m0, qhead0 + t);
+      int issued = 0;
+      for (int idx = 0; idx < 2 * NT; ++idx) {
+        const int slot = idx % kSlots, use = idx / kSlots;
+        if (use > 0 && !mbar_wait(bar(B_KVE + slot), (use - 1) & 1, abort_flag, prm.err)) break;
+        mbar_arrive_expect_tx(bar(B_KVF + slot), kTileBytes);
+        const CUtensorMap *map = (idx & 1) ? &tmV : &tmK;
+        const int row0 = (jt0 + idx / 2) * kBN;
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(sb + kOffKV + slot * kTileBytes + c * 16384, map, bar(B_KVF + slot), c * 64, row0, kvhead);
+        issued = idx + 1;
+      }
+      if (*abort_flag, prm.err) {
+        // let the copies already in flight land before the CTA exits
+        for (int idx = (issued > kSlots ? issued - kSlots : 0); idx < issued; ++idx) {
+          mbar_wait(bar(B_KVF + idx % kSlots), (idx / kSlots) & 1, nullptr, prm.err);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0 && NT > 0) {
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err);
+      tc_fence_after();
+      for (int it = 0; ok && it < NT; ++it) {
+        const int idxK = 2 * it, slotK = idxK % kSlots;
+        ok = mbar_wait(bar(B_KVF + slotK), (idxK / kSlots) & 1, abort_flag, prm.err);
+        if (!ok) break;
+        const int idxV = 2 * (it - 1) + 1, slotV = (idxV + kSlots) % kSlots;
+        if (it > 0) {
+          ok = mbar_wait(bar(B_KVF + slotV), (idxV / kSlots) & 1, abort_flag, prm.err);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const uint32_t k_base = sb + kOffKV + slotK * kTileBytes;
+        const uint32_t v_base = sb + kOffKV + slotV * kTileBytes;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (it > 0) {
+            ok = mbar_wait(bar(B_PF + t), (it - 1) & 1, abort_flag, prm.err);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t p_base = sb + kOffP + t * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(v_base + kk * 2048, 16384, 1024);
+              mma_bf16_ss(tmem + 256 + t * 128, ad, bd, kIdescPV, (it > 1 || kk > 0) ? 1u : 0u);
+            }
+          }
+          const uint32_t q_base = sb + kOffQ + t * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ss(tmem + t * 128, sdesc_sw128(q_base + koff, 16, 1024),
+                        sdesc_sw128(k_base + koff, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(B_SF + t));
+        }
+        if (!ok) break;
+        tc_commit(bar(B_KVE + slotK));
+        if (it > 0) tc_commit(bar(B_KVE + slotV));
+      }
+      if (ok) {
+        const int idxV = 2 * (NT - 1) + 1, slotV = idxV % kSlots;
+        ok = mbar_wait(bar(B_KVF + slotV), (idxV / kSlots) & 1, abort_flag, prm.err);
+        tc_fence_after();
+        const uint32_t v_base = sb + kOffKV + slotV * kTileBytes;
+        for (int t = 0; t < 2 && ok; ++t) {
+          ok = mbar_wait(bar(B_PF + t), (NT - 1) & 1, abort_flag, prm.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t p_base = sb + kOffP + t * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(v_base + kk * 2048, 16384, 1024);
+            mma_bf16_ss(tmem + 256 + t * 128, ad, bd, kIdescPV, (NT > 1 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar(B_OF + t));
+        }
+        if (ok) tc_commit(bar(B_KVE + slotV));
+      }
+      if (!ok) {
+        // drain: wait for every MMA issued so far before TMEM is released
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int wg = (warp - 4) >> 2;        // query tile 0 or 1
+    const int wq = warp & 3;               // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;
+    const int i = m0 + row;
+    const bool valid = i < g.n;
+    int lo_i = 1, hi_i = 0;
+    if (valid) prm.mk.row_range(i, lo_i, hi_i);
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + wg * 128;
+    const uint32_t tO = tmem + lane_off + 256 + wg * 128;
+    const uint32_t p_base = sb + kOffP + wg * kTileBytes;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int it = 0; it < NT; ++it) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + wg), it & 1, abort_flag, prm.err));
+      if (!ok) break;
+      tc_fence_after();
+      const int n0 = (jt0 + it) * kBN;
+      // the tile needs no element mask when every row of the CTA sees all of it
+      const bool full = (n0 >= lo_last) && (n0 + kBN - 1 <= hi_first) && (n0 + kBN <= g.n);
+      uint32_t r[32];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tS + c * 32, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          float sv = __uint_as_float(r[x]) * prm.scale_log2;
+          if (!full) {
+            const int j = n0 + c * 32 + x;
+            if (j < lo_i || j > hi_i) sv = -INFINITY;
+          }
+          mx = fmaxf(mx, sv);
+        }
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const bool had = m_run != -INFINITY;
+      const bool rescale = had && (m_new > m_run + kRescaleThreshold);
+      if (!had) {
+        m_run = m_new;
+      } else if (rescale) {
+        l_run *= exp2f(m_run - m_new);
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        const float a = rescale ? exp2f(m_run - m_new) : 1.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tO + c * 32, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * a);
+          tmem_st32(tO + c * 32, r);
+        }
+      }
+      if (rescale) m_run = m_new;
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tS + c * 32, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          float s0 = __uint_as_float(r[x]) * prm.scale_log2;
+          float s1 = __uint_as_float(r[x + 1]) * prm.scale_log2;
+          if (!full) {
+            const int j = n0 + c * 32 + x;
+            if (j < lo_i || j > hi_i) s0 = -INFINITY;
+            if (j + 1 < lo_i || j + 1 > hi_i) s1 = -INFINITY;
+          }
+          const float p0 = exp2f(s0 - m_use), p1 = exp2f(s1 - m_use);
+          l_run += p0 + p1;
+          pk[x >> 1] = pack_bf16x2(p0, p1);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_shared_v4(p_base + sw128_offset(row, c * 4 + u), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
+                       pk[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_PF + wg));
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + wg), 0, abort_flag, prm.err));
+    tc_fence_after();
+    const long long orow = (long long)(qhead0 + wg) * g.n + i;
+    const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    if (ok && NT > 0) {
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tO + c * 32, r);
+        if (valid) {
+          uint4 *dst = reinterpret_cast<uint4 *>(prm.o + orow * kHD + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * inv, __uint_as_float(r[8 * u + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv);
+            dst[u] = w;
+          }
+        }
+      }
+    } else if (valid && NT == 0) {
+      uint4 *dst = reinterpret_cast<uint4 *>(prm.o + orow * kHD);
+      for (int u = 0; u < kHD / 8; ++u) dst[u] = make_uint4(0, 0, 0, 0);
+    }
+    if (valid && (ok || NT == 0))
+      prm.lse[orow] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag, prm.err) raise_error(prm.err, ULY_ERR_TIMEOUT);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 3-D bf16 map over [heads][n][d] (d = 128) with 64 x 128 x 1 boxes, 128-byte
+// swizzle; rows past n read as zero.
+bool make_tmap_heads_bf16(CUtensorMap *map, const void *base, int d, int n, int heads, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const MaskInfo &mk,
+                                const void *q, const void *k, const void *v, void *o, float *lse,
+                                cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  const int qheads = g.P * g.B * g.hl, kvheads = g.P * g.B * g.gl;
+  if (!make_tmap_heads_bf16(&tq, q, kHD, g.n, qheads, 128) ||
+      !make_tmap_heads_bf16(&tk, k, kHD, g.n, kvheads, 128) ||
+      !make_tmap_heads_bf16(&tv, v, kHD, g.n, kvheads, 128))
+    return ULY_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return ULY_ERR_CUDA;
+    attr_set = true;
+  }
+  FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16 *>(o);
+  prm.lse = lse;
+  prm.g = g;
+  prm.mk = mk;
+  prm.scale_log2 = g.scale * kLog2e;
+  prm.err = error_word();
+  dim3 grid(g.P * g.B * (g.hl / 2), (g.n + kBM - 1) / kBM);
+  attn_fwd_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);
+  note_launches(1);
+  return last_launch_status();
+}
+
+}  // namespace uly

@@ -1,0 +1,80 @@
+// Internal helpers shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/ulysses.h"
+
+namespace uly {
+
+// Data-dependent failures are OR-ed as (1 << status) into the device error
+// word of the current device (see error_word()); kernels never trap.
+__device__ __forceinline__ void raise_error(int *err, uly_status s) {
+  if (err) atomicOr(err, 1 << (int)s);
+}
+
+// Device address of the error word of the current device (nullptr on failure).
+int *error_word();
+
+// Host-side launch bookkeeping (counts every kernel launched by the library).
+void note_launches(int n);
+
+inline uly_status last_launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+  uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Position ranges of the three masks.  Row i may see keys [lo, hi].
+// doc-causal: the document containing i, found by binary search in cu_seqlens.
+__device__ __forceinline__ int doc_start_of(const int32_t *__restrict__ cu, int num_docs, int i) {
+  int lo = 0, hi = num_docs - 1;  // find the largest e with cu[e] <= i
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
+  }
+  return __ldg(cu + lo);
+}
+__device__ __forceinline__ int doc_end_of(const int32_t *__restrict__ cu, int num_docs, int i) {
+  int lo = 0, hi = num_docs - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
+  }
+  return __ldg(cu + lo + 1);
+}
+
+struct MaskInfo {
+  int mask;            // uly_mask
+  int n;
+  const int32_t *cu;
+  int num_docs;
+  // visible keys of query row i (i < n): [lo, hi]
+  __device__ __forceinline__ void row_range(int i, int &lo, int &hi) const {
+    if (mask == ULY_MASK_NONE) { lo = 0; hi = n - 1; return; }
+    hi = i;
+    lo = (mask == ULY_MASK_DOC_CAUSAL) ? doc_start_of(cu, num_docs, i) : 0;
+  }
+  // query rows that see key j (j < n): [lo, hi]
+  __device__ __forceinline__ void col_range(int j, int &lo, int &hi) const {
+    if (mask == ULY_MASK_NONE) { lo = 0; hi = n - 1; return; }
+    lo = j;
+    hi = (mask == ULY_MASK_DOC_CAUSAL) ? doc_end_of(cu, num_docs, j) - 1 : n - 1;
+  }
+};
+
+// Per-launch geometry of the head layout shared by the attention kernels.
+struct HeadGeom {
+  int B, n, P, hl, gl, group;  // hl = H/P, gl = G/P, group = H/G
+  float scale;                 // softmax scale
+};
+
+}  // namespace uly

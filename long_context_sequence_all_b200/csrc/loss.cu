@@ -1,0 +1,210 @@
+// Token-weighted cross-entropy aggregated over the P logical ranks
+// ("Paralelismul de Secvență Ulysses", section "Integrarea cu Accelerate":
+// each rank's loss is weighted by its number of valid tokens, so padding and
+// masked prompt tokens do not bias the mean).
+//
+//   l_t = logsumexp(z_t) - z_t[y_t]          (tokens with y_t != ignore_index)
+//   S_r = sum_{t in shard r} l_t,  C_r = #valid tokens of shard r
+//   L   = sum_r S_r / sum_r C_r
+//
+// Pass 1: one warp per token streams the token's logits row once (16-byte
+// loads, eight in flight per lane), keeping a running (max, sum) per lane;
+// lanes merge with shuffles.  Every CTA writes one (sum, count) partial for
+// its shard into the workspace.  Pass 2: one CTA per launch folds the
+// partials in a fixed order (deterministic) into S_r, C_r and L.
+// HBM-bound: each logits byte is read once.
+#include "common.cuh"
+
+namespace uly {
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kLoadsInFlight = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void merge(float &m, float &s, float m2, float s2) {
+  // (m, s) represents sum exp(x - m) = s; combine two such pairs.
+  const float mm = fmaxf(m, m2);
+  if (mm == -INFINITY) return;
+  s = s * exp2f((m - mm) * kLog2e) + s2 * exp2f((m2 - mm) * kLog2e);
+  m = mm;
+}
+
+template <typename T>
+__device__ __forceinline__ void load_vals(const uint4 &u, float (&x)[8]);
+
+template <>
+__device__ __forceinline__ void load_vals<__nv_bfloat16>(const uint4 &u, float (&x)[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 f = __bfloat1622float2(h[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+
+// fp32 logits: one uint4 holds 4 values; pad the rest with -inf.
+template <>
+__device__ __forceinline__ void load_vals<float>(const uint4 &u, float (&x)[8]) {
+  x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
+  x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
+  x[4] = x[5] = x[6] = x[7] = -INFINITY;
+}
+
+// grid = (blocks_per_shard, P).  Partials: part_sum[r * nb + blockIdx.x], part_cnt[...].
+template <typename T>
+__global__ void __launch_bounds__(kThreads) ce_partial_kernel(
+    const T *__restrict__ logits, const int32_t *__restrict__ labels, long long per_shard,
+    int vocab, int ignore_index, double *__restrict__ part_sum, long long *__restrict__ part_cnt,
+    int *err) {
+  constexpr int kPerVec = 16 / sizeof(T);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y, nb = gridDim.x;
+  const int vecs = vocab / kPerVec;  // vocab * sizeof(T) % 16 == 0 checked on the host
+  double acc = 0.0;
+  long long cnt = 0;
+  for (long long tt = (long long)blockIdx.x * kWarps + warp; tt < per_shard;
+       tt += (long long)nb * kWarps) {
+    const long long t = (long long)r * per_shard + tt;
+    const int y = __ldg(labels + t);
+    if (y == ignore_index) continue;
+    if (y < 0 || y >= vocab) {
+      if (lane == 0) raise_error(err, ULY_ERR_LABEL);
+      continue;
+    }
+    const uint4 *row = reinterpret_cast<const uint4 *>(logits + t * (long long)vocab);
+    float m = -INFINITY, s = 0.f;
+    for (int v0 = lane; v0 < vecs; v0 += 32 * kLoadsInFlight) {
+      uint4 u[kLoadsInFlight];
+#pragma unroll
+      for (int k = 0; k < kLoadsInFlight; ++k) {
+        const int v = v0 + k * 32;
+        if (v < vecs) u[k] = __ldcs(row + v);
+      }
+#pragma unroll
+      for (int k = 0; k < kLoadsInFlight; ++k) {
+        const int v = v0 + k * 32;
+        if (v < vecs) {
+          float x[8];
+          load_vals<T>(u[k], x);
+          float mx = x[0];
+#pragma unroll
+          for (int e = 1; e < 8; ++e) mx = fmaxf(mx, x[e]);
+          if (mx > m) {
+            s = (m == -INFINITY) ? 0.f : s * exp2f((m - mx) * kLog2e);
+            m = mx;
+          }
+          const float ml = m * kLog2e;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s += exp2f(fmaf(x[e], kLog2e, -ml));
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+      merge(m, s, m2, s2);
+    }
+    if (lane == 0) {
+      const float zy = static_cast<float>(logits[t * (long long)vocab + y]);
+      const float lse = m + logf(s);
+      acc += (double)lse - (double)zy;
+      cnt += 1;
+    }
+  }
+  __shared__ double sh_sum[kWarps];
+  __shared__ long long sh_cnt[kWarps];
+  if (lane == 0) { sh_sum[warp] = acc; sh_cnt[warp] = cnt; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0;
+    long long c = 0;
+    for (int w = 0; w < kWarps; ++w) { a += sh_sum[w]; c += sh_cnt[w]; }  // fixed order
+    part_sum[(long long)r * nb + blockIdx.x] = a;
+    part_cnt[(long long)r * nb + blockIdx.x] = c;
+  }
+}
+
+// One CTA: shard r's partials are folded by thread r in index order; then
+// thread 0 folds the shards in rank order.
+__global__ void __launch_bounds__(256) ce_finalize_kernel(
+    const double *__restrict__ part_sum, const long long *__restrict__ part_cnt, int P, int nb,
+    float *__restrict__ shard_sum, int64_t *__restrict__ shard_count, float *__restrict__ loss) {
+  __shared__ double sh_s[256];
+  __shared__ long long sh_c[256];
+  for (int r = threadIdx.x; r < P; r += blockDim.x) {
+    double a = 0.0;
+    long long c = 0;
+    for (int i = 0; i < nb; ++i) { a += part_sum[(long long)r * nb + i]; c += part_cnt[(long long)r * nb + i]; }
+    shard_sum[r] = (float)a;
+    shard_count[r] = c;
+    if (r < 256) { sh_s[r] = a; sh_c[r] = c; }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0;
+    long long c = 0;
+    for (int r = 0; r < P; ++r) {
+      if (r < 256) { a += sh_s[r]; c += sh_c[r]; }
+      else { a += (double)shard_sum[r]; c += shard_count[r]; }
+    }
+    *loss = (float)(a / (double)c);  // 0/0 -> NaN when no token is valid
+  }
+}
+
+}  // namespace
+
+int loss_blocks_per_shard(int P, long long per_shard) {
+  // about four CTAs per SM in total, at most one warp per token
+  long long nb = (4LL * 148 + P - 1) / P;
+  long long need = (per_shard + kWarps - 1) / kWarps;
+  if (nb > need) nb = need;
+  if (nb < 1) nb = 1;
+  return (int)nb;
+}
+
+size_t loss_workspace_bytes(int P, long long per_shard) {
+  const size_t nb = (size_t)loss_blocks_per_shard(P, per_shard);
+  return nb * (size_t)P * (sizeof(double) + sizeof(long long));
+}
+
+uly_status loss_validate(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, const void *logits,
+                         const int32_t *labels, const float *shard_sum, const int64_t *shard_count,
+                         const float *loss) {
+  if (!logits || !labels || !shard_sum || !shard_count || !loss) return ULY_ERR_NULL;
+  if (dtype != ULY_BF16 && dtype != ULY_F32) return ULY_ERR_DTYPE;
+  if (P <= 0 || P > 65535 || tokens < 0 || vocab <= 0) return ULY_ERR_SHAPE;
+  if (tokens % P) return ULY_ERR_SHAPE;
+  const int eb = dtype == ULY_BF16 ? 2 : 4;
+  if (((long long)vocab * eb) % 16) return ULY_ERR_ALIGN;
+  if (!aligned16(logits) || !aligned16(labels)) return ULY_ERR_ALIGN;
+  return ULY_OK;
+}
+
+// `ws` holds nb*P doubles followed by nb*P long longs.
+uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, const void *logits,
+                       const int32_t *labels, int32_t ignore_index, float *shard_sum,
+                       int64_t *shard_count, float *loss, void *ws, cudaStream_t stream) {
+  const long long per = tokens / P;
+  const int nb = loss_blocks_per_shard(P, per);
+  double *psum = static_cast<double *>(ws);
+  long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb * P);
+  dim3 grid(nb, P);
+  if (dtype == ULY_BF16)
+    ce_partial_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(logits), labels, per, vocab, ignore_index, psum, pcnt,
+        error_word());
+  else
+    ce_partial_kernel<float><<<grid, kThreads, 0, stream>>>(
+        static_cast<const float *>(logits), labels, per, vocab, ignore_index, psum, pcnt,
+        error_word());
+  ce_finalize_kernel<<<1, 256, 0, stream>>>(psum, pcnt, P, nb, shard_sum, shard_count, loss);
+  note_launches(2);
+  return last_launch_status();
+}
+
+}  // namespace uly

@@ -1,0 +1,222 @@
+"""ctypes binding of ``libulysses.so`` -- argument marshalling only.
+
+Every entry point of the C ABI (``include/ulysses.h``) is exposed under the
+same name.  The functions take CUDA torch tensors (torch is used for device
+memory and streams only), pass raw device pointers and the current CUDA
+stream to the library, and raise :class:`UlyssesError` on a non-OK status.
+All arithmetic happens in the library's kernels; there is no fallback: if the
+library is missing or cannot be loaded, every call fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libulysses.so")
+
+ULY_F32, ULY_BF16 = 0, 1
+MASK_NONE, MASK_CAUSAL, MASK_DOC_CAUSAL = 0, 1, 2
+STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE",
+          4: "ULY_ERR_ALIGN", 5: "ULY_ERR_ALIAS", 6: "ULY_ERR_UNSUPPORTED", 7: "ULY_ERR_CUDA",
+          8: "ULY_ERR_LABEL", 9: "ULY_ERR_TIMEOUT", 10: "ULY_ERR_WORKSPACE"}
+EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd",
+           "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
+           "ulysses_loss_aggregate", "ulysses_read_error", "ulysses_status_string",
+           "ulysses_launch_count"]
+
+
+class UlyssesError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("world", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int32), ("mask", ctypes.c_int32),
+                ("cu_seqlens", ctypes.c_void_p), ("num_docs", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once).  Raises if it is missing: there is no fallback."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                                   "`python -m long_context_sequence_all_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+            for name in ("ulysses_seq_to_head", "ulysses_head_to_seq"):
+                getattr(L, name).argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
+                getattr(L, name).restype = ctypes.c_int
+            D = ctypes.POINTER(AttnDesc)
+            L.ulysses_attn_fwd.argtypes = [D, vp, vp, vp, vp, vp, vp]
+            L.ulysses_attn_bwd_workspace_size.argtypes = [D, ctypes.POINTER(sz)]
+            L.ulysses_attn_bwd.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.ulysses_loss_workspace_size.argtypes = [i32, i64, i32, ctypes.POINTER(sz)]
+            L.ulysses_loss_aggregate.argtypes = [i32, i64, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+            L.ulysses_read_error.argtypes = [ctypes.POINTER(i32)]
+            L.ulysses_status_string.argtypes = [ctypes.c_int]
+            L.ulysses_status_string.restype = ctypes.c_char_p
+            L.ulysses_launch_count.restype = ctypes.c_uint64
+            for name in ("ulysses_attn_fwd", "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd",
+                         "ulysses_loss_workspace_size", "ulysses_loss_aggregate", "ulysses_read_error"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise UlyssesError(st, where)
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ULY_BF16
+    if t.dtype == torch.float32:
+        return ULY_F32
+    raise UlyssesError(3, f"dtype {t.dtype}")
+
+
+def make_desc(B, n, P, H, G, d, dtype_code, mask, cu_seqlens=None, scale=0.0) -> AttnDesc:
+    nd = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    return AttnDesc(B, n, P, H, G, d, dtype_code, mask,
+                    ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None,
+                    nd, float(scale))
+
+
+# --------------------------------------------------------------- all-to-alls
+
+def ulysses_seq_to_head(x: torch.Tensor, P: int, out: torch.Tensor | None = None, stream=None):
+    """[P][B][n/P][heads][d] -> [P][B][heads/P][n][d] (bit-exact copy)."""
+    P_, B, s, heads, d = x.shape
+    assert P_ == P
+    n = P * s
+    if out is None:
+        out = torch.empty((P, B, heads // P, n, d), dtype=x.dtype, device=x.device)
+    _check(lib().ulysses_seq_to_head(B, n, P, heads, d, x.element_size(), _p(x), _p(out),
+                                     _stream(stream)), "ulysses_seq_to_head")
+    return out
+
+
+def ulysses_head_to_seq(x: torch.Tensor, P: int, out: torch.Tensor | None = None, stream=None):
+    """[P][B][heads/P][n][d] -> [P][B][n/P][heads][d] (bit-exact copy)."""
+    P_, B, hl, n, d = x.shape
+    assert P_ == P
+    heads = hl * P
+    if out is None:
+        out = torch.empty((P, B, n // P, heads, d), dtype=x.dtype, device=x.device)
+    _check(lib().ulysses_head_to_seq(B, n, P, heads, d, x.element_size(), _p(x), _p(out),
+                                     _stream(stream)), "ulysses_head_to_seq")
+    return out
+
+
+# ----------------------------------------------------------------- attention
+
+def _desc_from(q, k, mask, cu_seqlens, scale):
+    P, B, hl, n, d = q.shape
+    gl = k.shape[2]
+    return make_desc(B, n, P, hl * P, gl * P, d, _dtype_code(q), mask, cu_seqlens, scale)
+
+
+def ulysses_attn_fwd(q, k, v, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0, o=None, lse=None,
+                     stream=None):
+    """Head layout in/out: q [P][B][H/P][n][d], k, v [P][B][G/P][n][d] ->
+    o like q, lse float32 [P][B][H/P][n]."""
+    desc = _desc_from(q, k, mask, cu_seqlens, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:4], dtype=torch.float32, device=q.device)
+    _check(lib().ulysses_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse),
+                                  _stream(stream)), "ulysses_attn_fwd")
+    return o, lse
+
+
+def ulysses_attn_bwd_workspace_size(desc: AttnDesc) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ulysses_attn_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(n)),
+           "ulysses_attn_bwd_workspace_size")
+    return n.value
+
+
+def ulysses_attn_bwd(q, k, v, o, lse, dout, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0,
+                     dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of sum(O * dO) in head layout: dq like q, dk/dv like k."""
+    desc = _desc_from(q, k, mask, cu_seqlens, scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = ulysses_attn_bwd_workspace_size(desc)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().ulysses_attn_bwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout),
+                                  _p(dq), _p(dk), _p(dv), _p(workspace), workspace.numel(),
+                                  _stream(stream)), "ulysses_attn_bwd")
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------- loss
+
+def ulysses_loss_workspace_size(P: int, tokens: int, vocab: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ulysses_loss_workspace_size(P, tokens, vocab, ctypes.byref(n)),
+           "ulysses_loss_workspace_size")
+    return n.value
+
+
+def ulysses_loss_aggregate(logits, labels, P, ignore_index=-100, shard_sum=None, shard_count=None,
+                           loss=None, workspace=None, stream=None):
+    """logits [T][V] (bf16/fp32; shard r = rows [r*T/P, (r+1)*T/P)), labels int32 [T] ->
+    (shard_sum float32 [P], shard_count int64 [P], loss float32 [1]) on the device."""
+    T, V = logits.shape
+    dev = logits.device
+    shard_sum = torch.empty(P, dtype=torch.float32, device=dev) if shard_sum is None else shard_sum
+    shard_count = torch.empty(P, dtype=torch.int64, device=dev) if shard_count is None else shard_count
+    loss = torch.empty(1, dtype=torch.float32, device=dev) if loss is None else loss
+    need = ulysses_loss_workspace_size(P, T, V)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib().ulysses_loss_aggregate(P, T, V, _dtype_code(logits), _p(logits), _p(labels),
+                                        ignore_index, _p(shard_sum), _p(shard_count), _p(loss),
+                                        _p(workspace), workspace.numel(), _stream(stream)),
+           "ulysses_loss_aggregate")
+    return shard_sum, shard_count, loss
+
+
+# -------------------------------------------------------------------- misc
+
+def ulysses_read_error() -> int:
+    """Read and clear the device error word (synchronises the device)."""
+    w = ctypes.c_int32(0)
+    _check(lib().ulysses_read_error(ctypes.byref(w)), "ulysses_read_error")
+    return w.value
+
+
+def ulysses_status_string(status: int) -> str:
+    return lib().ulysses_status_string(status).decode()
+
+
+def ulysses_launch_count() -> int:
+    return int(lib().ulysses_launch_count())

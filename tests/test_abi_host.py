@@ -1,0 +1,101 @@
+"""CPU-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments before launching anything (these
+calls validate on the host and never reach a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ulysses.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_sequence_all_b200 import build, ulysses
+    build.build()
+    return ulysses.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ulysses_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_path_entry_points():
+    names = declared_functions()
+    for n in ["ulysses_seq_to_head", "ulysses_attn_fwd", "ulysses_attn_bwd", "ulysses_head_to_seq",
+              "ulysses_loss_aggregate"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    from long_context_sequence_all_b200 import ulysses
+    assert set(ulysses.EXPORTS) <= set(declared_functions())
+
+
+def test_status_strings(L):
+    from long_context_sequence_all_b200 import ulysses
+    for code, name in ulysses.STATUS.items():
+        assert ulysses.ulysses_status_string(code)
+    assert ulysses.ulysses_status_string(0) == "ok"
+
+
+def test_permute_validation(L):
+    vp = ctypes.c_void_p
+    a, b = vp(1 << 20), vp(1 << 30)   # never dereferenced: validation fails first
+    assert L.ulysses_seq_to_head(1, 1024, 4, 8, 64, 4, None, b, None) == 1        # NULL
+    assert L.ulysses_seq_to_head(1, 1022, 4, 8, 64, 4, a, b, None) == 2           # n % P
+    assert L.ulysses_seq_to_head(1, 1024, 4, 6, 64, 4, a, b, None) == 2           # heads % P
+    assert L.ulysses_seq_to_head(1, 1024, 4, 8, 64, 3, a, b, None) == 3           # elem bytes
+    assert L.ulysses_seq_to_head(1, 1024, 4, 8, 6, 2, a, b, None) == 4            # row not 16 B
+    assert L.ulysses_seq_to_head(1, 1024, 4, 8, 64, 4, vp((1 << 20) + 4), b, None) == 4  # misaligned
+    assert L.ulysses_head_to_seq(1, 1024, 4, 8, 64, 4, a, vp((1 << 20) + 4096), None) == 5  # overlap
+    assert L.ulysses_seq_to_head(0, 1024, 4, 8, 64, 4, a, b, None) == 2
+
+
+def test_attn_desc_validation(L):
+    from long_context_sequence_all_b200 import ulysses as U
+    n = ctypes.c_size_t(0)
+    ok = U.make_desc(1, 8192, 4, 32, 8, 128, U.ULY_BF16, U.MASK_CAUSAL)
+    assert L.ulysses_attn_bwd_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == 0
+    assert n.value >= 8192 * 32 * 4
+    bad = [U.make_desc(1, 8190, 4, 32, 8, 128, U.ULY_BF16, 1),   # n % P
+           U.make_desc(1, 8192, 4, 30, 8, 128, U.ULY_BF16, 1),   # H % P
+           U.make_desc(1, 8192, 4, 32, 6, 128, U.ULY_BF16, 1),   # G % P, H % G
+           U.make_desc(1, 8192, 4, 32, 8, 128, 7, 1)]            # dtype
+    codes = [L.ulysses_attn_bwd_workspace_size(ctypes.byref(d), ctypes.byref(n)) for d in bad]
+    assert codes == [2, 2, 2, 3]
+    assert L.ulysses_attn_bwd_workspace_size(
+        ctypes.byref(U.make_desc(1, 8192, 4, 32, 8, 64, U.ULY_BF16, 1)), ctypes.byref(n)) == 6
+    assert L.ulysses_attn_bwd_workspace_size(
+        ctypes.byref(U.make_desc(1, 8192, 4, 32, 8, 128, U.ULY_BF16, 2)), ctypes.byref(n)) == 1  # no cu
+    d = U.make_desc(1, 8192, 4, 32, 8, 128, U.ULY_BF16, 1)
+    vp = ctypes.c_void_p
+    assert L.ulysses_attn_fwd(ctypes.byref(d), None, vp(1 << 20), vp(1 << 21), vp(1 << 22),
+                              vp(1 << 23), None) == 1
+    # bwd without workspace
+    assert L.ulysses_attn_bwd(ctypes.byref(d), *[vp(1 << (20 + i)) for i in range(9)], None, 0, None) == 10
+
+
+def test_loss_validation(L):
+    vp = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    assert L.ulysses_loss_workspace_size(4, 65536, 8192, ctypes.byref(n)) == 0 and n.value > 0
+    assert L.ulysses_loss_workspace_size(4, 65535, 8192, ctypes.byref(n)) == 2
+    args = [vp(1 << 30), vp(1 << 20), -100, vp(1 << 21), vp(1 << 22), vp(1 << 23), vp(1 << 24), 1 << 20, None]
+    assert L.ulysses_loss_aggregate(4, 1023, 8192, 1, *args) == 2
+    assert L.ulysses_loss_aggregate(4, 1024, 8191, 1, *args) == 4           # row not 16 B
+    assert L.ulysses_loss_aggregate(4, 1024, 8192, 9, *args) == 3
+    small = args[:-3] + [vp(1 << 24), 8, None]
+    assert L.ulysses_loss_aggregate(4, 1024, 8192, 1, *small) == 10
+
+
+def test_library_has_no_cpu_fallback_symbols():
+    """The product binding never imports the oracle."""
+    src = open(os.path.join(ROOT, "long_context_sequence_all_b200", "ulysses.py")).read()
+    assert "oracle" not in src.replace("no fallback", "")
