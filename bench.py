@@ -1,0 +1,547 @@
+#!/usr/bin/env python
+"""Benchmark of the single-GPU Ulysses attention layer (sm_100a).
+
+One step = the whole hot path over one batch of the workload:
+  seq->head(Q, K, V) -> attention forward -> head->seq(O)
+  seq->head(dO) -> attention backward -> head->seq(dQ, dK, dV)
+  token-weighted cross-entropy aggregated over the P shards.
+Default workload: the Qwen3-4B-shaped layer at n = 65536 (B=1, P=4 logical
+ranks, 32 query / 8 KV heads, head_dim 128, bf16, causal, vocab 8192).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is whole-job tokens/s with inputs
+resident in HBM (CUDA events on the launch stream, max over ranks); `e2e`
+repeats the step through the same C ABI with pinned host buffers, the
+host->device copies of the step's inputs and the device->host copies of its
+outputs inside the timed region.  Every GPU runs an independent replica
+(different seed): the path has no data-path collective, so scaling is weak.
+`--impl reference` times the CPU oracle (the plain fp64 reference
+implementation) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from long_context_sequence_all_b200.workloads import WORKLOADS, make_inputs, to_natural  # noqa: E402
+
+METRIC = "Ulysses attn layer tokens/s + TFLOP/s (frac BF16 peak); permute GB/s (frac HBM)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CLOCK_FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------- workload
+
+def causal_pairs(inp) -> float:
+    """Unmasked (query, key) pairs of one head: n(n+1)/2 causal, n^2 full,
+    sum over documents of L(L+1)/2 for the doc-causal mask."""
+    n = inp["n"]
+    if inp["mask"] == 0:
+        return float(n) * n
+    if inp["mask"] == 1:
+        return n * (n + 1) / 2.0
+    cu = inp["cu_seqlens"].tolist()
+    return float(sum((b - a) * (b - a + 1) / 2.0 for a, b in zip(cu[:-1], cu[1:])))
+
+
+def algorithmic_work(inp):
+    """Algorithmic flops / bytes of each kernel per launch (see the design notes)."""
+    B, H, G, d, n = inp["B"], inp["H"], inp["G"], inp["d"], inp["n"]
+    pairs = causal_pairs(inp)
+    qb = B * n * H * d * 2
+    kvb = B * n * G * d * 2
+    w = {
+        "attn_fwd_sm100": ("flops", 4.0 * B * H * d * pairs),
+        "attn_dkdv_sm100": ("flops", 8.0 * B * H * d * pairs),   # S, dP, dV, dK
+        "attn_dq_sm100": ("flops", 2.0 * B * H * d * pairs),     # dQ (S, dP recomputed)
+        "attn_bwd_dot": ("bytes", 2.0 * qb + B * n * H * 4),
+    }
+    if "logits" in inp:
+        valid = int((inp["labels"] != -100).sum())
+        w["loss_partial"] = ("bytes", valid * inp["vocab"] * 2.0 + inp["labels"].numel() * 4)
+    # permutations: one read + one write of every element, per step
+    w["seq_to_head"] = ("bytes_step", 2.0 * (qb + 2 * kvb + qb))    # Q, K, V, dO
+    w["head_to_seq"] = ("bytes_step", 2.0 * (qb + qb + 2 * kvb))    # O, dQ, dK, dV
+    return w, pairs
+
+
+# ------------------------------------------------------------- GPU ("ours")
+
+class Layer:
+    """Device buffers and one step of the layer through the C ABI."""
+
+    def __init__(self, inp, dev):
+        from long_context_sequence_all_b200 import ulysses as U
+        self.U = U
+        self.inp = inp
+        self.P = inp["P"]
+        self.mask = inp["mask"]
+        f = lambda x: x.to(dev, non_blocking=False)
+        self.q, self.k, self.v, self.do = (f(inp[x]) for x in ("q", "k", "v", "do"))
+        self.cu = None if inp["cu_seqlens"] is None else f(inp["cu_seqlens"])
+        self.logits = f(inp["logits"]) if "logits" in inp else None
+        self.labels = f(inp["labels"]) if "labels" in inp else None
+        P = self.P
+        self.qh = U.ulysses_seq_to_head(self.q, P)
+        self.kh = U.ulysses_seq_to_head(self.k, P)
+        self.vh = U.ulysses_seq_to_head(self.v, P)
+        self.doh = U.ulysses_seq_to_head(self.do, P)
+        self.oh, self.lse = U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu)
+        self.o = U.ulysses_head_to_seq(self.oh, P)
+        self.dqh, self.dkh, self.dvh = (torch.empty_like(x) for x in (self.qh, self.kh, self.vh))
+        desc = U._desc_from(self.qh, self.kh, self.mask, self.cu, 0.0)
+        self.ws = torch.empty(max(256, U.ulysses_attn_bwd_workspace_size(desc)), dtype=torch.uint8, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(x) for x in (self.q, self.k, self.v))
+        if self.logits is not None:
+            T, V = self.logits.shape
+            self.S = torch.empty(P, dtype=torch.float32, device=dev)
+            self.C = torch.empty(P, dtype=torch.int64, device=dev)
+            self.L = torch.empty(1, dtype=torch.float32, device=dev)
+            self.lws = torch.empty(max(256, U.ulysses_loss_workspace_size(P, T, V)), dtype=torch.uint8, device=dev)
+
+    def step(self):
+        U, P = self.U, self.P
+        U.ulysses_seq_to_head(self.q, P, out=self.qh)
+        U.ulysses_seq_to_head(self.k, P, out=self.kh)
+        U.ulysses_seq_to_head(self.v, P, out=self.vh)
+        U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.oh, lse=self.lse)
+        U.ulysses_head_to_seq(self.oh, P, out=self.o)
+        U.ulysses_seq_to_head(self.do, P, out=self.doh)
+        U.ulysses_attn_bwd(self.qh, self.kh, self.vh, self.oh, self.lse, self.doh, mask=self.mask,
+                           cu_seqlens=self.cu, dq=self.dqh, dk=self.dkh, dv=self.dvh, workspace=self.ws)
+        U.ulysses_head_to_seq(self.dqh, P, out=self.dq)
+        U.ulysses_head_to_seq(self.dkh, P, out=self.dk)
+        U.ulysses_head_to_seq(self.dvh, P, out=self.dv)
+        if self.logits is not None:
+            U.ulysses_loss_aggregate(self.logits, self.labels, P, shard_sum=self.S, shard_count=self.C,
+                                     loss=self.L, workspace=self.lws)
+
+
+class HostIO:
+    """Pinned host copies of one step's inputs and outputs (end-to-end arm)."""
+
+    def __init__(self, layer: Layer):
+        self.layer = layer
+        L = layer
+        self.ins = [(L.q, L.inp["q"].pin_memory()), (L.k, L.inp["k"].pin_memory()),
+                    (L.v, L.inp["v"].pin_memory()), (L.do, L.inp["do"].pin_memory())]
+        if L.logits is not None:
+            self.ins += [(L.logits, L.inp["logits"].pin_memory()), (L.labels, L.inp["labels"].pin_memory())]
+        outs = [L.o, L.dq, L.dk, L.dv] + ([L.L, L.S, L.C] if L.logits is not None else [])
+        self.outs = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in outs]
+        self.h2d = sum(h.numel() * h.element_size() for _, h in self.ins)
+        self.d2h = sum(h.numel() * h.element_size() for _, h in self.outs)
+
+    def step(self):
+        for d, h in self.ins:
+            d.copy_(h, non_blocking=True)
+        self.layer.step()
+        for d, h in self.outs:
+            h.copy_(d, non_blocking=True)
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of the SM clock and throttle reasons."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(CLOCK_FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < len(CLOCK_FIELDS):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(kernel: str) -> str:
+    files = {"attn_fwd_sm100": "attn_fwd_sm100.cu", "attn_dkdv_sm100": "attn_bwd_sm100.cu",
+             "attn_dq_sm100": "attn_bwd_sm100.cu", "seq_to_head": "permute.cu", "head_to_seq": "permute.cu",
+             "loss_partial": "loss.cu", "attn_bwd_dot": "attn_f32.cu"}
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_sequence_all_b200", "csrc")
+    for f in [files.get(kernel, ""), "sm100.cuh", "common.cuh"]:
+        p = os.path.join(csrc, f)
+        if f and os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
+    when there is none or the kernel's source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[workload][kernel]
+        if e.get("source_hash") != kernel_source_hash(kernel):
+            return None
+        return float(e["bytes_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
+        return None
+
+
+def run_ours(args, rank, world, dev):
+    from long_context_sequence_all_b200 import build, ulysses as U
+    build.build()
+    U.lib()
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, seed=1000 + w.index + 7919 * rank)
+    work, pairs = algorithmic_work(inp)
+    layer = Layer(inp, dev)
+    U.ulysses_read_error()
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    err = U.ulysses_read_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x} after warm-up")
+
+    stream = torch.cuda.current_stream()
+    gpu_index = _gpu_index(dev)
+    n0 = U.ulysses_launch_count()
+    U.ulysses_profile_enable(True)
+    with ClockSampler(gpu_index) as clk:
+        _barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            layer.step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        _barrier(world)
+    prof = U.ulysses_profile_read()
+    U.ulysses_profile_enable(False)
+    launches = U.ulysses_launch_count() - n0
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = _max_over_ranks(ms, world, dev)
+    err = U.ulysses_read_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x} in the timed region")
+
+    # end to end through the same C ABI with pinned host buffers
+    io = HostIO(layer)
+    io.step()
+    torch.cuda.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        io.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+
+    tokens = inp["B"] * inp["n"]
+    value = world * tokens / (ms_max / 1e3)
+    peaks, peak_src = load_peaks()
+    kernels = {}
+    for name, (tot_ms, cnt) in prof.items():
+        per_launch = tot_ms / cnt
+        k = {"launches_per_step": cnt / args.steps, "ms_per_launch": per_launch,
+             "ms_per_step": tot_ms / args.steps}
+        if name in work:
+            kind, amount = work[name]
+            if kind == "flops":
+                k["tflops"] = amount / (per_launch / 1e3) / 1e12
+                k["frac_bf16_sustained"] = k["tflops"] / peaks["bf16_tflops_sustained"]
+            elif kind == "bytes":
+                k["gbs"] = amount / (per_launch / 1e3) / 1e9
+                k["frac_hbm"] = k["gbs"] / peaks["hbm_gbs"]
+            else:  # bytes per step over all launches of the kernel
+                k["gbs"] = amount / (tot_ms / args.steps / 1e3) / 1e9
+                k["frac_hbm"] = k["gbs"] / peaks["hbm_gbs"]
+        kernels[name] = k
+    dominant = max(kernels, key=lambda n: kernels[n]["ms_per_step"])
+    dk = kernels[dominant]
+    kind, amount = work.get(dominant, ("flops", float("nan")))
+    if kind == "flops":
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": dk["tflops"],
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": dk["tflops"] / peaks["bf16_tflops_sustained"]}
+    else:
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dk["gbs"] / peaks["hbm_gbs"]}
+    roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if kind == 'flops' else 'hbm_gbs'})"
+    roof["traffic"] = dram_traffic(dominant, args.workload)
+    attn_ms = sum(kernels[k]["ms_per_step"] for k in kernels if k.startswith("attn_"))
+    fwd_fl = 4.0 * inp["B"] * inp["H"] * inp["d"] * pairs
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(128) Q/K/V, N(0,1) dO and logits, uniform labels)",
+        "config": {"workload": f"{w.name}: Qwen3-4B-shaped Ulysses attention layer, B={w.B} n={inp['n']} "
+                               f"P={w.P} H={w.H} G={w.G} d={w.d} bf16 causal fwd+bwd + CE loss V={w.vocab}",
+                   "global_batch": inp["B"] * world, "seq_len": inp["n"],
+                   "parallelism": f"P={w.P} logical Ulysses ranks per GPU; {world} independent replica(s)",
+                   "l2": "no flush: every input tensor (Q 512 MiB, logits 1 GiB) exceeds the 126 MB L2"},
+        "attn_tflops": (fwd_fl * 3.5) / (attn_ms / 1e3) / 1e12,
+        "attn_fwd_tflops": kernels.get("attn_fwd_sm100", {}).get("tflops"),
+        "attn_bwd_tflops": (10.0 * inp["B"] * inp["H"] * inp["d"] * pairs) /
+                           (sum(kernels[k]["ms_per_step"] for k in ("attn_dkdv_sm100", "attn_dq_sm100",
+                                                                   "attn_bwd_dot") if k in kernels) / 1e3) / 1e12,
+        "permute_gbs": {k: kernels[k]["gbs"] for k in ("seq_to_head", "head_to_seq") if k in kernels},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "e2e": {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": io.h2d, "d2h_bytes_per_step": io.d2h},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp, budget_s=args.cpu_budget)
+    return line
+
+
+def _gpu_index(dev):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    idx = dev.index or 0
+    if vis:
+        parts = [p for p in vis.split(",") if p.strip()]
+        if idx < len(parts) and parts[idx].strip().isdigit():
+            return int(parts[idx])
+    return idx
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------ CPU oracle timings
+
+def cpu_step_sample(inp, rows_per_head: int, token_frac: float):
+    """Time the oracle on a bounded sample of one step and extrapolate to the
+    whole step: `rows_per_head` uniformly spaced query rows of every head
+    (forward, dQ and their dK/dV terms: all the attention work of those rows)
+    and a `token_frac` fraction of the tokens for the two all-to-alls and the
+    loss.  Returns (extrapolated seconds for the full step, seconds the
+    sample took, description)."""
+    import oracle
+    P, B, n, H, G, d = inp["P"], inp["B"], inp["n"], inp["H"], inp["G"], inp["d"]
+    group = H // G
+    f32 = lambda t: t.to(torch.float32).numpy()
+    spent = 0.0
+    # all-to-alls on a token subset (same P and heads), both directions
+    s_sub = max(1, int(round(n // P * token_frac)))
+    frac_perm = s_sub / (n // P)
+    t_perm = 0.0
+    for x, heads in ((inp["q"], H), (inp["k"], G), (inp["v"], G), (inp["do"], H)):
+        sub = np.ascontiguousarray(x[:, :, :s_sub].contiguous().view(torch.int16).numpy())
+        t0 = time.perf_counter()
+        h = oracle.seq_to_head(sub, B, s_sub * P, P, heads)
+        oracle.head_to_seq(h, B, s_sub * P, P, heads)           # O, dQ, dK, dV come back
+        t_perm += time.perf_counter() - t0
+    spent += t_perm
+    t_perm /= frac_perm
+    # loss on a token subset
+    t_loss = 0.0
+    if "logits" in inp:
+        T = inp["logits"].shape[0]
+        tsub = max(P, int(round(T * token_frac)) // P * P)
+        z = f32(inp["logits"][:tsub])
+        y = inp["labels"][:tsub].numpy()
+        t0 = time.perf_counter()
+        oracle.loss_aggregate(z, y, P)
+        dt = time.perf_counter() - t0
+        spent += dt
+        t_loss = dt * T / tsub
+    # attention: uniformly spaced rows of every head
+    qn, kn, vn, don = (to_natural(inp[x])[0] for x in ("q", "k", "v", "do"))
+    rows = np.unique(np.linspace(0, n - 1, rows_per_head).astype(np.int32))
+    cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy()
+    t_attn = 0.0
+    for g in range(G):
+        kg, vg = f32(kn[:, g].contiguous()), f32(vn[:, g].contiguous())
+        dk = np.zeros((n, d)); dv = np.zeros((n, d))
+        for h in range(g * group, (g + 1) * group):
+            qg, dg = f32(qn[:, h].contiguous()), f32(don[:, h].contiguous())
+            t0 = time.perf_counter()
+            oracle.head_rows_step(qg, kg, vg, dg, rows, mask=inp["mask"], cu_seqlens=cu, dk=dk, dv=dv)
+            t_attn += time.perf_counter() - t0
+    spent += t_attn
+    desc = (f"{rows.size} uniformly spaced query rows of each of the {H} heads (forward, dQ and their "
+            f"dK/dV terms: {rows.size}/{n} of the attention work) and {token_frac:.4g} of the tokens for "
+            f"the all-to-alls and the loss, each extrapolated linearly to the full step; "
+            f"the sample took {spent:.1f} s")
+    return t_perm + t_loss + t_attn * n / rows.size, spent, desc
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def _rows_for(inp, budget_s, token_frac):
+    """Rows per head so that one sample takes about budget_s seconds."""
+    _, spent, _ = cpu_step_sample(inp, rows_per_head=2, token_frac=token_frac)
+    return int(max(2, min(1024, 2 * budget_s / max(1e-6, spent))))
+
+
+def cpu_baseline(inp, budget_s: float = 20.0):
+    rows = _rows_for(inp, budget_s, token_frac=1 / 64)
+    t_full, spent, desc = cpu_step_sample(inp, rows_per_head=rows, token_frac=1 / 64)
+    tokens = inp["B"] * inp["n"]
+    return {"value": tokens / t_full, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+            "sample": desc, "step_s_extrapolated": t_full}
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle, as it stands, on this machine's host cores: every step is a
+    bounded sample of the workload, extrapolated to the whole step."""
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = _rows_for(inp, per_step, token_frac=1 / 256)
+    for _ in range(args.warmup):
+        cpu_step_sample(inp, rows_per_head=rows, token_frac=1 / 256)
+    ts, desc = [], ""
+    for _ in range(args.steps):
+        t, _, desc = cpu_step_sample(inp, rows_per_head=rows, token_frac=1 / 256)
+        ts.append(t)
+    step_s = statistics.median(ts)
+    tokens = inp["B"] * inp["n"]
+    value = tokens / step_s
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": f"{w.name}: Qwen3-4B-shaped Ulysses attention layer, B={w.B} n={inp['n']} "
+                               f"P={w.P} H={w.H} G={w.G} d={w.d} causal fwd+bwd + CE loss V={w.vocab}",
+                   "global_batch": inp["B"], "seq_len": inp["n"], "parallelism": "CPU oracle (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen64k", choices=sorted(k for k in WORKLOADS if k != "tiny_f32"))
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=dev)
+    try:
+        line = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

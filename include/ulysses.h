@@ -152,11 +152,29 @@ uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab,
  * device) into *word (bit s set <=> status s was raised) and clears it. */
 uly_status ulysses_read_error(int32_t *word);
 
+/* Like ulysses_read_error, but copies up to n words of the error record:
+ * info[0] = the error word; if a bounded wait ran out, info[1] = 1 and
+ * info[2..8] = CTA x, CTA y, thread, shared-memory barrier address, phase
+ * parity, cycles waited >> 20, and polls of the first wait that gave up.
+ * The record is cleared. */
+uly_status ulysses_read_error_info(int32_t *info, int32_t n);
+
 /* Human-readable name of a status. */
 const char *ulysses_status_string(uly_status status);
 
 /* Number of kernels launched by this process through the library so far. */
 uint64_t ulysses_launch_count(void);
+
+/* Per-kernel device timing.  ulysses_profile_enable(1) clears the totals and
+ * makes every later launch record two CUDA events on its own stream (a few
+ * microseconds of host time per launch); ulysses_profile_enable(0) stops.
+ * ulysses_profile_read() waits for the recorded events and returns, for
+ * kernel id `kernel` (0 <= kernel < ulysses_kernel_count()), the summed
+ * device milliseconds and the number of timed launches. */
+uly_status ulysses_profile_enable(int32_t on);
+uly_status ulysses_profile_read(int32_t kernel, double *total_ms, int64_t *launches);
+int32_t ulysses_kernel_count(void);
+const char *ulysses_kernel_name(int32_t kernel);
 
 #ifdef __cplusplus
 }

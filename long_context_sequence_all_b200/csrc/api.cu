@@ -10,7 +10,7 @@
 namespace uly {
 
 // Device error word, one per device context (module globals are per context).
-__device__ int g_error_word_storage = 0;
+__device__ int g_error_word_storage[kErrInfoWords] = {0};
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
@@ -221,16 +221,22 @@ uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab, 
                      shard_count, loss, workspace, static_cast<cudaStream_t>(stream));
 }
 
-uly_status ulysses_read_error(int32_t *word) {
-  if (!word) return ULY_ERR_NULL;
+uly_status ulysses_read_error_info(int32_t *info, int32_t n) {
+  if (!info) return ULY_ERR_NULL;
+  if (n < 1) return ULY_ERR_SHAPE;
   int *p = error_word();
   if (!p) return ULY_ERR_CUDA;
-  int host = 0, zero = 0;
+  int host[kErrInfoWords] = {0}, zero[kErrInfoWords] = {0};
   if (cudaDeviceSynchronize() != cudaSuccess) return ULY_ERR_CUDA;
-  if (cudaMemcpy(&host, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ULY_ERR_CUDA;
-  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ULY_ERR_CUDA;
-  *word = host;
+  if (cudaMemcpy(host, p, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return ULY_ERR_CUDA;
+  if (cudaMemcpy(p, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return ULY_ERR_CUDA;
+  for (int i = 0; i < n; ++i) info[i] = i < kErrInfoWords ? host[i] : 0;
   return ULY_OK;
+}
+
+uly_status ulysses_read_error(int32_t *word) {
+  if (!word) return ULY_ERR_NULL;
+  return ulysses_read_error_info(word, 1);
 }
 
 const char *ulysses_status_string(uly_status s) {

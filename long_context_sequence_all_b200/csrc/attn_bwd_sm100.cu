@@ -1,13 +1,579 @@
-// Local attention backward on the tensor cores (bf16): see the kernels below.
+// Local attention backward of every logical rank on the 5th-generation tensor
+// cores (the adjoint of Ulysses step 4; the gradients of sum(O * dO)):
+//
+//   P_ij  = exp(scale * q_i.k_j - LSE_i)          (recomputed, never stored)
+//   dP_ij = dO_i . v_j,   D_i = dO_i . O_i,   dS_ij = P_ij (dP_ij - D_i)
+//   dV_j  = sum_i P_ij dO_i          dK_j = scale * sum_i dS_ij q_i
+//   dQ_i  = scale * sum_j dS_ij k_j
+// with dK, dV summed over the query heads that share a KV head (GQA).
+//
+// Three launches, all deterministic (no atomics):
+//  1. D_i = <dO_i, O_i>   (one warp per row, HBM-bound)
+//  2. dK/dV kernel, KV-stationary: a CTA owns 128 keys of one KV head and
+//     visits every 64-row query tile (of every query head of the group) that
+//     sees them.  Two compute warpgroups take alternate query tiles (ping-
+//     pong) so one group's exp/dS work overlaps the other group's MMAs:
+//       S^T  = K Q^T,  dP^T = V dO^T          (M=128 keys, N=64 queries, K=128)
+//       dV  += P^T dO, dK  += dS^T Q           (M=128 keys, N=128,      K=64)
+//     P^T and dS^T go through shared memory (bf16, swizzled); dK and dV stay
+//     in TMEM until the end.
+//  3. dQ kernel, query-stationary (like the forward: two query heads of one
+//     group at the same positions share K/V tiles of 64 keys):
+//       S = Q K^T, dP = dO V^T (M=128, N=64, K=128);  dQ += dS K (N=128, K=64)
+//
+// TMA loads with 128-byte swizzle feed shared memory; one thread issues all
+// MMAs; every wait is bounded (ULY_ERR_TIMEOUT).
+#include "prof.cuh"
 #include "sm100.cuh"
 
 namespace uly {
 
-uly_status attn_bf16_bwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
-                                const void *, const void *, const void *, const void *,
-                                const float *, const void *, void *, void *, void *, float *,
-                                cudaStream_t) {
-  return ULY_ERR_UNSUPPORTED;
+using namespace sm100;
+
+bool make_tmap_heads_bf16(CUtensorMap *map, const void *base, int d, int n, int heads, int box_rows);
+uly_status attn_bwd_dot_launch(int dtype, int head_dim, const void *o, const void *dout, float *Dv,
+                               long long rows, cudaStream_t stream);
+
+namespace {
+
+constexpr int kHD = 128;
+constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr uint32_t kIdescN64 = idesc_bf16_f32(128, 64, false, false);    // K-major A and B, N = 64
+constexpr uint32_t kIdescN128MN = idesc_bf16_f32(128, 128, false, true); // B MN-major, N = 128
+
+struct BwdParams {
+  const float *lse;   // [qheads][n]
+  const float *Dv;    // [qheads][n]
+  __nv_bfloat16 *out0;  // dkdv: dV, dq: dQ
+  __nv_bfloat16 *out1;  // dkdv: dK
+  HeadGeom g;
+  MaskInfo mk;
+  float scale_log2;
+  int *err;
+};
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a [rows][64]
+// bf16 operand stored as one 128-byte-swizzled span per row.
+__device__ __forceinline__ uint32_t sw128_row64(int row, int chunk) {
+  return (uint32_t)(row * 128 + (((chunk ^ (row & 7))) << 4));
+}
+
+// ============================================================== dK / dV
+namespace kv {
+constexpr int kBN = 128;   // keys per CTA
+constexpr int kBQ = 64;    // query rows per tile
+constexpr int kStages = 3;
+constexpr uint32_t kKVBytes = 128 * 128 * 2;       // K or V tile
+constexpr uint32_t kQBytes = 64 * 128 * 2;         // Q or dO tile
+constexpr uint32_t kOffK = 0, kOffV = kKVBytes;
+constexpr uint32_t kOffStage = 2 * kKVBytes;       // stage s: Q at +s*2*kQBytes, dO after it
+constexpr uint32_t kOffPT = kOffStage + kStages * 2 * kQBytes;   // per WG: P^T then dS^T (16 KB each)
+constexpr uint32_t kOffLD = kOffPT + 2 * 2 * (128 * 64 * 2);     // per WG: 64 lse2 + 64 D floats
+constexpr uint32_t kOffBar = kOffLD + 2 * 512;
+constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
+}  // namespace kv
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                           const BwdParams prm) {
+  using namespace kv;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  enum { B_KV = 0, B_SF_ = 1, B_SE = 1 + kStages, B_S = 1 + 2 * kStages, B_P = B_S + 2, B_DONE = B_P + 2,
+         B_DRAIN = B_DONE + 1, B_N = B_DRAIN + 1 };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const HeadGeom &g = prm.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kvh = blockIdx.x;                    // (r*B + b)*gl + gg
+  const int rb = kvh / g.gl, gg = kvh - rb * g.gl;
+  const int qh_base = rb * g.hl + gg * g.group;  // first query head of the group
+  const int n0 = blockIdx.y * kBN;               // earliest keys (heaviest) first
+
+  // query rows that see any of the keys [n0, n0+127]
+  int lo_a, hi_a, lo_b, hi_b;
+  prm.mk.col_range(n0, lo_a, hi_a);
+  prm.mk.col_range(min(n0 + kBN - 1, g.n - 1), lo_b, hi_b);
+  const int qt0 = lo_a / kBQ;
+  const int nqt = (hi_b >= lo_a) ? hi_b / kBQ - qt0 + 1 : 0;
+  const int T = nqt * g.group;                   // tiles: head-major
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: dV [0,128) dK [128,256); WG w: S^T [256+128w, +64), dP^T [+64, +64)
+
+  if (warp == 0) {
+    if (lane == 0 && T > 0) {
+      mbar_arrive_expect_tx(bar(B_KV), 2 * kKVBytes);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_3d(sb + kOffK + c * 16384, &tmK, bar(B_KV), c * 64, n0, kvh);
+        tma_load_3d(sb + kOffV + c * 16384, &tmV, bar(B_KV), c * 64, n0, kvh);
+      }
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % kStages, use = t / kStages;
+        if (use > 0 && !mbar_wait(bar(B_SE + s), (use - 1) & 1, abort_flag, prm.err)) break;
+        const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
+        const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
+        mbar_arrive_expect_tx(bar(B_SF_ + s), 2 * kQBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(st + c * 8192, &tmQ, bar(B_SF_ + s), c * 64, i0, qh_base + e);
+          tma_load_3d(st + kQBytes + c * 8192, &tmO, bar(B_SF_ + s), c * 64, i0, qh_base + e);
+        }
+        issued = t + 1;
+      }
+      if (*abort_flag)
+        for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
+          mbar_wait(bar(B_SF_ + t % kStages), (t / kStages) & 1, nullptr, prm.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && T > 0) {
+      bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
+      tc_fence_after();
+      auto issue_sdp = [&](int t) -> bool {
+        const int w = t & 1, s = t % kStages;
+        if (!mbar_wait(bar(B_SF_ + s), (t / kStages) & 1, abort_flag, prm.err)) return false;
+        tc_fence_after();
+        const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
+        const uint32_t tS = tmem + 256 + 128 * w;
+#pragma unroll
+        for (int kk = 0; kk < kHD / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32, qo = (kk >> 2) * 8192 + (kk & 3) * 32;
+          mma_bf16_ss(tS, sdesc_sw128(sb + kOffK + ko, 16, 1024), sdesc_sw128(st + qo, 16, 1024),
+                      kIdescN64, kk > 0);
+          mma_bf16_ss(tS + 64, sdesc_sw128(sb + kOffV + ko, 16, 1024),
+                      sdesc_sw128(st + kQBytes + qo, 16, 1024), kIdescN64, kk > 0);
+        }
+        tc_commit(bar(B_S + w));
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      if (ok && T > 1) ok = issue_sdp(1);
+      for (int t = 0; ok && t < T; ++t) {
+        const int w = t & 1, s = t % kStages;
+        ok = mbar_wait(bar(B_P + w), (t >> 1) & 1, abort_flag, prm.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
+        const uint32_t pt = sb + kOffPT + w * 32768, dst = pt + 16384;
+#pragma unroll
+        for (int kk = 0; kk < kBQ / 16; ++kk) {
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16_ss(tmem + 0, sdesc_sw128(pt + kk * 32, 16, 1024),
+                      sdesc_sw128(st + kQBytes + kk * 2048, 8192, 1024), kIdescN128MN, acc);
+          mma_bf16_ss(tmem + 128, sdesc_sw128(dst + kk * 32, 16, 1024),
+                      sdesc_sw128(st + kk * 2048, 8192, 1024), kIdescN128MN, acc);
+        }
+        tc_commit(bar(B_SE + s));
+        if (t + 2 < T) ok = issue_sdp(t + 2);
+      }
+      if (ok) tc_commit(bar(B_DONE));
+      if (!ok) {
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
+      }
+    }
+  } else if (warp >= 4) {
+    const int w = (warp - 4) >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane;            // key row within the tile
+    const int j = n0 + row;
+    const int tid = threadIdx.x - 128 * (w + 1);  // 0..127 within the warpgroup
+    int lo_j = 1, hi_j = 0;
+    if (j < g.n) prm.mk.col_range(j, lo_j, hi_j);
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 256 + 128 * w;
+    const uint32_t pt = sb + kOffPT + w * 32768, dst = pt + 16384;
+    float *lsm = reinterpret_cast<float *>(smem + kOffLD + w * 512);  // [0,64) lse*log2e, [64,128) D
+    bool ok = true;
+    for (int t = w; t < T; t += 2) {
+      const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
+      const int qh = qh_base + e;
+      named_bar_sync(1 + w, 128);              // previous tile's LSE/D reads are done
+      {
+        const int c = tid & 63, i = i0 + c;
+        if (tid < 64) lsm[c] = (i < g.n) ? prm.lse[(long long)qh * g.n + i] * kLog2e : INFINITY;
+        else lsm[64 + c] = (i < g.n) ? prm.Dv[(long long)qh * g.n + i] : 0.f;
+      }
+      named_bar_sync(1 + w, 128);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + w), (t >> 1) & 1, abort_flag, prm.err));
+      if (!ok) break;
+      tc_fence_after();
+      const bool full = (i0 >= n0 + kBN - 1) && (i0 + kBQ - 1 <= hi_a) && (i0 + kBQ <= g.n) &&
+                        (n0 + kBN <= g.n) && (prm.mk.mask != ULY_MASK_DOC_CAUSAL || i0 + kBQ - 1 <= hi_a);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(tS + ch * 32, rs);
+        tmem_ld32(tS + 64 + ch * 32, rd);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          float p[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = ch * 32 + x + u;
+            float pv = exp2f(fmaf(__uint_as_float(rs[x + u]), prm.scale_log2, -lsm[c]));
+            if (!full) {
+              const int i = i0 + c;
+              if (i < lo_j || i > hi_j) pv = 0.f;
+            }
+            p[u] = pv;
+            ds[u] = pv * (__uint_as_float(rd[x + u]) - lsm[64 + c]);
+          }
+          pp[x >> 1] = pack_bf16x2(p[0], p[1]);
+          dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t off = sw128_row64(row, ch * 4 + u);
+          st_shared_v4(pt + off, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
+          st_shared_v4(dst + off, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_P + w));
+    }
+    // epilogue: WG0 writes dV, WG1 writes dK (scaled)
+    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err));
+    tc_fence_after();
+    __nv_bfloat16 *outp = (w == 0) ? prm.out0 : prm.out1;
+    const float mul = (w == 0) ? 1.f : g.scale;
+    const long long orow = (long long)kvh * g.n + j;
+    if (ok && T > 0) {
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tmem + lane_off + 128 * w + c * 32, r);
+        if (j < g.n) {
+          uint4 *dptr = reinterpret_cast<uint4 *>(outp + orow * kHD + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * mul, __uint_as_float(r[8 * u + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * mul, __uint_as_float(r[8 * u + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * mul, __uint_as_float(r[8 * u + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * mul, __uint_as_float(r[8 * u + 7]) * mul);
+            dptr[u] = v;
+          }
+        }
+      }
+    } else if (T == 0 && j < g.n) {
+      uint4 *dptr = reinterpret_cast<uint4 *>(outp + orow * kHD);
+      for (int u = 0; u < kHD / 8; ++u) dptr[u] = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ================================================================== dQ
+namespace qk {
+constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
+constexpr int kBK = 64;    // keys per K/V tile
+constexpr int kStages = 2;
+constexpr uint32_t kQBytes = 128 * 128 * 2;
+constexpr uint32_t kKBytes = 64 * 128 * 2;
+constexpr uint32_t kOffQ = 0;                      // Q_0, Q_1
+constexpr uint32_t kOffO = 2 * kQBytes;            // dO_0, dO_1
+constexpr uint32_t kOffKV = 4 * kQBytes;           // stage s: K at +s*2*kKBytes, V after it
+constexpr uint32_t kOffDS = kOffKV + kStages * 2 * kKBytes;   // dS_0, dS_1 (128 x 64 bf16)
+constexpr uint32_t kOffBar = kOffDS + 2 * (128 * 64 * 2);
+constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
+}  // namespace qk
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                         const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const BwdParams prm) {
+  using namespace qk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  enum { B_Q = 0, B_KF = 1, B_KE = 1 + kStages, B_S = 1 + 2 * kStages, B_P = B_S + 2, B_DQ = B_P + 2,
+         B_DRAIN = B_DQ + 2, B_N = B_DRAIN + 1 };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const HeadGeom &g = prm.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = g.hl >> 1;
+  const int pair = blockIdx.x;
+  const int rb = pair / half, pp = pair - rb * half;
+  const int qhead0 = rb * g.hl + 2 * pp;
+  const int kvhead = rb * g.gl + (2 * pp) / g.group;
+  const int mt = gridDim.y - 1 - blockIdx.y;
+  const int m0 = mt * kBM;
+
+  int lo_first, hi_first, lo_last, hi_last;
+  prm.mk.row_range(m0, lo_first, hi_first);
+  prm.mk.row_range(min(m0 + kBM - 1, g.n - 1), lo_last, hi_last);
+  const int jt0 = lo_first / kBK;
+  const int NT = (hi_last >= lo_first) ? hi_last / kBK - jt0 + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns, tile t: S [256t, +64), dP [256t+64, +64), dQ [256t+128, +128)
+
+  if (warp == 0) {
+    if (lane == 0 && NT > 0) {
+      mbar_arrive_expect_tx(bar(B_Q), 4 * kQBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sb + kOffQ + t * kQBytes + c * 16384, &tmQ, bar(B_Q), c * 64, m0, qhead0 + t);
+          tma_load_3d(sb + kOffO + t * kQBytes + c * 16384, &tmO, bar(B_Q), c * 64, m0, qhead0 + t);
+        }
+      int issued = 0;
+      for (int j = 0; j < NT; ++j) {
+        const int s = j % kStages, use = j / kStages;
+        if (use > 0 && !mbar_wait(bar(B_KE + s), (use - 1) & 1, abort_flag, prm.err)) break;
+        const uint32_t st = sb + kOffKV + s * 2 * kKBytes;
+        const int row0 = (jt0 + j) * kBK;
+        mbar_arrive_expect_tx(bar(B_KF + s), 2 * kKBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(st + c * 8192, &tmK, bar(B_KF + s), c * 64, row0, kvhead);
+          tma_load_3d(st + kKBytes + c * 8192, &tmV, bar(B_KF + s), c * 64, row0, kvhead);
+        }
+        issued = j + 1;
+      }
+      if (*abort_flag)
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(bar(B_KF + j % kStages), (j / kStages) & 1, nullptr, prm.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && NT > 0) {
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err);
+      tc_fence_after();
+      auto issue_dq = [&](int t, int j) {
+        // dQ_t += dS_t K_j   (A = dS K-major, B = K tile MN-major over d)
+        const uint32_t kst = sb + kOffKV + (j % kStages) * 2 * kKBytes;
+        const uint32_t ds = sb + kOffDS + t * 16384;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          mma_bf16_ss(tmem + 256 * t + 128, sdesc_sw128(ds + kk * 32, 16, 1024),
+                      sdesc_sw128(kst + kk * 2048, 8192, 1024), kIdescN128MN, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      for (int j = 0; ok && j < NT; ++j) {
+        const int s = j % kStages;
+        ok = mbar_wait(bar(B_KF + s), (j / kStages) & 1, abort_flag, prm.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kst = sb + kOffKV + s * 2 * kKBytes;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j > 0) {
+            ok = mbar_wait(bar(B_P + t), (j - 1) & 1, abort_flag, prm.err);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dq(t, j - 1);
+          }
+          const uint32_t q = sb + kOffQ + t * kQBytes, o = sb + kOffO + t * kQBytes;
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t qo = (kk >> 2) * 16384 + (kk & 3) * 32, ko = (kk >> 2) * 8192 + (kk & 3) * 32;
+            mma_bf16_ss(tmem + 256 * t, sdesc_sw128(q + qo, 16, 1024), sdesc_sw128(kst + ko, 16, 1024),
+                        kIdescN64, kk > 0);
+            mma_bf16_ss(tmem + 256 * t + 64, sdesc_sw128(o + qo, 16, 1024),
+                        sdesc_sw128(kst + kKBytes + ko, 16, 1024), kIdescN64, kk > 0);
+          }
+          tc_commit(bar(B_S + t));
+        }
+        if (!ok) break;
+        if (j > 0) tc_commit(bar(B_KE + (j - 1) % kStages));
+      }
+      for (int t = 0; t < 2 && ok; ++t) {
+        ok = mbar_wait(bar(B_P + t), (NT - 1) & 1, abort_flag, prm.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dq(t, NT - 1);
+        tc_commit(bar(B_DQ + t));
+      }
+      if (ok) tc_commit(bar(B_KE + (NT - 1) % kStages));
+      if (!ok) {
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
+      }
+    }
+  } else if (warp >= 4) {
+    const int t = (warp - 4) >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int i = m0 + row;
+    const bool valid = i < g.n;
+    int lo_i = 1, hi_i = 0;
+    if (valid) prm.mk.row_range(i, lo_i, hi_i);
+    const long long qrow = (long long)(qhead0 + t) * g.n + i;
+    const float lse2 = valid ? prm.lse[qrow] * kLog2e : INFINITY;
+    const float Di = valid ? prm.Dv[qrow] : 0.f;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 256 * t;
+    const uint32_t ds_base = sb + kOffDS + t * 16384;
+    bool ok = true;
+    for (int j = 0; j < NT; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + t), j & 1, abort_flag, prm.err));
+      if (!ok) break;
+      tc_fence_after();
+      const int n0 = (jt0 + j) * kBK;
+      const bool full = (n0 >= lo_last) && (n0 + kBK - 1 <= hi_first) && (n0 + kBK <= g.n);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(tS + ch * 32, rs);
+        tmem_ld32(tS + 64 + ch * 32, rd);
+        uint32_t dd[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            float pv = exp2f(fmaf(__uint_as_float(rs[x + u]), prm.scale_log2, -lse2));
+            if (!full) {
+              const int jj = n0 + ch * 32 + x + u;
+              if (jj < lo_i || jj > hi_i) pv = 0.f;
+            }
+            ds[u] = pv * (__uint_as_float(rd[x + u]) - Di);
+          }
+          dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_shared_v4(ds_base + sw128_row64(row, ch * 4 + u), dd[4 * u], dd[4 * u + 1], dd[4 * u + 2],
+                       dd[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_P + t));
+    }
+    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ + t), 0, abort_flag, prm.err));
+    tc_fence_after();
+    if (ok && NT > 0) {
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tS + 128 + c * 32, r);
+        if (valid) {
+          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 v;
+            const float sc = g.scale;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
+            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
+            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
+            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
+            dptr[u] = v;
+          }
+        }
+      }
+    } else if (NT == 0 && valid) {
+      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD);
+      for (int u = 0; u < kHD / 8; ++u) dptr[u] = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const MaskInfo &mk,
+                                const void *q, const void *k, const void *v, const void *o,
+                                const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                                float *Dv, cudaStream_t stream) {
+  const int qheads = g.P * g.B * g.hl, kvheads = g.P * g.B * g.gl;
+  uly_status st = attn_bwd_dot_launch(ULY_BF16, d->head_dim, o, dout, Dv, (long long)qheads * g.n, stream);
+  if (st != ULY_OK) return st;
+  CUtensorMap mK128, mV128, mQ64, mO64, mQ128, mO128, mK64, mV64;
+  if (!make_tmap_heads_bf16(&mK128, k, kHD, g.n, kvheads, 128) ||
+      !make_tmap_heads_bf16(&mV128, v, kHD, g.n, kvheads, 128) ||
+      !make_tmap_heads_bf16(&mQ64, q, kHD, g.n, qheads, 64) ||
+      !make_tmap_heads_bf16(&mO64, dout, kHD, g.n, qheads, 64) ||
+      !make_tmap_heads_bf16(&mQ128, q, kHD, g.n, qheads, 128) ||
+      !make_tmap_heads_bf16(&mO128, dout, kHD, g.n, qheads, 128) ||
+      !make_tmap_heads_bf16(&mK64, k, kHD, g.n, kvheads, 64) ||
+      !make_tmap_heads_bf16(&mV64, v, kHD, g.n, kvheads, 64))
+    return ULY_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_dkdv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kv::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             qk::kSmemBytes) != cudaSuccess)
+      return ULY_ERR_CUDA;
+    attr_set = true;
+  }
+  BwdParams prm;
+  prm.lse = lse;
+  prm.Dv = Dv;
+  prm.g = g;
+  prm.mk = mk;
+  prm.scale_log2 = g.scale * kLog2e;
+  prm.err = error_word();
+  prm.out0 = static_cast<__nv_bfloat16 *>(dv);
+  prm.out1 = static_cast<__nv_bfloat16 *>(dk);
+  dim3 gkv(kvheads, (g.n + kv::kBN - 1) / kv::kBN);
+  {
+    prof::Scope scope(prof::K_ATTN_DKDV_SM100, stream);
+    attn_dkdv_sm100_kernel<<<gkv, kThreads, kv::kSmemBytes, stream>>>(mK128, mV128, mQ64, mO64, prm);
+  }
+  prm.out0 = static_cast<__nv_bfloat16 *>(dq);
+  prm.out1 = nullptr;
+  dim3 gq(qheads / 2, (g.n + qk::kBM - 1) / qk::kBM);
+  {
+    prof::Scope scope(prof::K_ATTN_DQ_SM100, stream);
+    attn_dq_sm100_kernel<<<gq, kThreads, qk::kSmemBytes, stream>>>(mQ128, mO128, mK64, mV64, prm);
+  }
+  note_launches(2);
+  return last_launch_status();
 }
 
 }  // namespace uly

@@ -15,6 +15,7 @@
 // over the query rows of every query head of its group (deterministic, no
 // atomics).
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace uly {
 
@@ -281,6 +282,7 @@ uly_status attn_f32_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const 
   const float *Q = static_cast<const float *>(q), *K = static_cast<const float *>(k),
               *V = static_cast<const float *>(v);
   float *O = static_cast<float *>(o);
+  prof::Scope scope(prof::K_ATTN_FWD_F32, stream);
   if (d->head_dim == 64)
     attn_fwd_f32_kernel<64><<<grid, kThreads, 0, stream>>>(Q, K, V, O, lse, g, mk);
   else if (d->head_dim == 128)
@@ -295,6 +297,7 @@ uly_status attn_bwd_dot_launch(int dtype, int head_dim, const void *o, const voi
                                long long rows, cudaStream_t stream) {
   const unsigned blocks = (unsigned)((rows + 7) / 8);
   if (blocks == 0) return ULY_OK;
+  prof::Scope scope(prof::K_ATTN_BWD_DOT, stream);
   if (dtype == ULY_F32 && head_dim == 64)
     attn_bwd_dot_kernel<float, 64><<<blocks, 256, 0, stream>>>(
         static_cast<const float *>(o), static_cast<const float *>(dout), Dv, rows);
@@ -322,14 +325,20 @@ uly_status attn_f32_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const 
   float *dQ = static_cast<float *>(dq), *dK = static_cast<float *>(dk), *dV = static_cast<float *>(dv);
   dim3 gq((g.n + kRows - 1) / kRows, g.P * g.B * g.hl);
   dim3 gk((g.n + kRows - 1) / kRows, g.P * g.B * g.gl);
-  if (d->head_dim == 64) {
-    attn_dq_f32_kernel<64><<<gq, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dQ, g, mk);
-    attn_dkdv_f32_kernel<64><<<gk, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dK, dV, g, mk);
-  } else if (d->head_dim == 128) {
-    attn_dq_f32_kernel<128><<<gq, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dQ, g, mk);
-    attn_dkdv_f32_kernel<128><<<gk, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dK, dV, g, mk);
-  } else {
-    return ULY_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return ULY_ERR_UNSUPPORTED;
+  {
+    prof::Scope scope(prof::K_ATTN_DQ_F32, stream);
+    if (d->head_dim == 64)
+      attn_dq_f32_kernel<64><<<gq, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dQ, g, mk);
+    else
+      attn_dq_f32_kernel<128><<<gq, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dQ, g, mk);
+  }
+  {
+    prof::Scope scope(prof::K_ATTN_DKDV_F32, stream);
+    if (d->head_dim == 64)
+      attn_dkdv_f32_kernel<64><<<gk, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dK, dV, g, mk);
+    else
+      attn_dkdv_f32_kernel<128><<<gk, kThreads, 0, stream>>>(Q, K, V, dO, lse, Dv, dK, dV, g, mk);
   }
   note_launches(2);
   return last_launch_status();

@@ -25,6 +25,7 @@
 // when softmax sees S_j it also knows the previous PV finished (O may be
 // rescaled, P may be overwritten).  p_full[t] hands P_j back to the MMA warp.
 // Every wait is bounded (ULY_ERR_TIMEOUT), no wait can spin forever.
+#include "prof.cuh"
 #include "sm100.cuh"
 
 namespace uly {
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sb + kOffKV + slot * kTileBytes + c * 16384, map, bar(B_KVF + slot), c * 64, row0, kvhead);
         issued = idx + 1;
       }
-      if (*abort_flag, prm.err) {
+      if (*abort_flag) {
         // let the copies already in flight land before the CTA exits
         for (int idx = (issued > kSlots ? issued - kSlots : 0); idx < issued; ++idx) {
           mbar_wait(bar(B_KVF + idx % kSlots), (idx / kSlots) & 1, nullptr, prm.err);
@@ -326,7 +327,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (threadIdx.x == 0 && *abort_flag, prm.err) raise_error(prm.err, ULY_ERR_TIMEOUT);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -382,6 +382,7 @@ uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.scale_log2 = g.scale * kLog2e;
   prm.err = error_word();
   dim3 grid(g.P * g.B * (g.hl / 2), (g.n + kBM - 1) / kBM);
+  prof::Scope scope(prof::K_ATTN_FWD_SM100, stream);
   attn_fwd_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);
   note_launches(1);
   return last_launch_status();

@@ -11,11 +11,14 @@ namespace uly {
 
 // Data-dependent failures are OR-ed as (1 << status) into the device error
 // word of the current device (see error_word()); kernels never trap.
+// err[0] is the word; err[1..kErrInfoWords) describe the first bounded wait
+// that ran out (see ulysses_read_error_info).
+constexpr int kErrInfoWords = 16;
 __device__ __forceinline__ void raise_error(int *err, uly_status s) {
   if (err) atomicOr(err, 1 << (int)s);
 }
 
-// Device address of the error word of the current device (nullptr on failure).
+// Device address of the error record of the current device (nullptr on failure).
 int *error_word();
 
 // Host-side launch bookkeeping (counts every kernel launched by the library).

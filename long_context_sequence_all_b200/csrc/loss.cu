@@ -14,6 +14,7 @@
 // partials in a fixed order (deterministic) into S_r, C_r and L.
 // HBM-bound: each logits byte is read once.
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace uly {
 
@@ -194,6 +195,7 @@ uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, 
   double *psum = static_cast<double *>(ws);
   long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb * P);
   dim3 grid(nb, P);
+  prof::Scope s1(prof::K_LOSS_PARTIAL, stream);
   if (dtype == ULY_BF16)
     ce_partial_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(logits), labels, per, vocab, ignore_index, psum, pcnt,
@@ -202,6 +204,8 @@ uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, 
     ce_partial_kernel<float><<<grid, kThreads, 0, stream>>>(
         static_cast<const float *>(logits), labels, per, vocab, ignore_index, psum, pcnt,
         error_word());
+  s1.end();
+  prof::Scope s2(prof::K_LOSS_FINALIZE, stream);
   ce_finalize_kernel<<<1, 256, 0, stream>>>(psum, pcnt, P, nb, shard_sum, shard_count, loss);
   note_launches(2);
   return last_launch_status();

@@ -13,6 +13,7 @@
 // written in full 16-byte vectors by consecutive lanes (coalesced), and all
 // index arithmetic is per row, never per byte.
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace uly {
 
@@ -74,6 +75,7 @@ cudaError_t launch_permute(int B, int n, int P, int heads, int vpr, const void *
   dim3 grid((s + tok - 1) / tok, P * B);
   const uint4 *in = static_cast<const uint4 *>(src);
   uint4 *out = static_cast<uint4 *>(dst);
+  prof::Scope scope(TO_HEAD ? prof::K_SEQ_TO_HEAD : prof::K_HEAD_TO_SEQ, stream);
 #define ULY_PERMUTE_CASE(V)                                                                   \
   case V:                                                                                     \
     permute_rows_kernel<V, TO_HEAD><<<grid, kThreads, 0, stream>>>(in, out, B, n, s, heads, \

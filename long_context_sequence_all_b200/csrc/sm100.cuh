@@ -13,21 +13,18 @@
 namespace uly {
 namespace sm100 {
 
-// A bounded wait gives up after kWaitLimitNs and reports ULY_ERR_TIMEOUT.
-// A wait that has already lasted kPeerAbortNs also gives up as soon as some
-// other CTA has reported a timeout, so a failed launch ends quickly.  Correct
-// waits here last microseconds, far below both limits.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
-constexpr uint64_t kPeerAbortNs = 50000000ull;    // 50 ms
+// A bounded wait gives up after kWaitLimitCycles SM clock cycles (1-2 s at
+// the B200's clocks) and reports ULY_ERR_TIMEOUT.  A wait that has already
+// lasted kPeerAbortCycles (50-100 ms) also gives up as soon as some other CTA
+// has reported a timeout, so a failed launch ends quickly.  Correct waits here
+// last microseconds, far below both limits.  The per-SM cycle counter is used
+// because it is monotonic for a thread (the global nanosecond timer is not
+// guaranteed to be).
+constexpr long long kWaitLimitCycles = 2000000000ll;
+constexpr long long kPeerAbortCycles = 100000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -59,23 +56,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of `bar` to complete.  Returns false when the wait
-// runs out (see kWaitLimitNs / kPeerAbortNs) or when *abort is already set;
+// runs out (see kWaitLimitCycles / kPeerAbortCycles) or when *abort is already set;
 // then *abort is set so the CTA's other roles stop too.  abort == nullptr:
 // a drain wait that only honours the limits.  err: the device error word.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int *err) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 127u) == 0) {
       if (abort && *abort) return false;
-      const uint64_t dt = globaltimer() - t0;
+      const long long dt = clock64() - t0;
       bool give_up = false;
-      if (dt > kWaitLimitNs) {
+      if (dt > kWaitLimitCycles) {
         raise_error(err, ULY_ERR_TIMEOUT);
+        if (err && atomicCAS(err + 1, 0, 1) == 0) {
+          // first timeout of this device: where it happened
+          err[2] = blockIdx.x;
+          err[3] = blockIdx.y;
+          err[4] = threadIdx.x;
+          err[5] = (int)(bar & 0xFFFFF);
+          err[6] = (int)parity;
+          err[7] = (int)(dt >> 20);
+          err[8] = (int)it;
+          __threadfence();
+        }
         give_up = true;
-      } else if (dt > kPeerAbortNs && err &&
+      } else if (dt > kPeerAbortCycles && err &&
                  (*(volatile int *)err & (1 << (int)ULY_ERR_TIMEOUT))) {
         give_up = true;
       }

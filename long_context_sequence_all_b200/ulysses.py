@@ -25,7 +25,9 @@ STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE"
           8: "ULY_ERR_LABEL", 9: "ULY_ERR_TIMEOUT", 10: "ULY_ERR_WORKSPACE"}
 EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
-           "ulysses_loss_aggregate", "ulysses_read_error", "ulysses_status_string",
+           "ulysses_loss_aggregate", "ulysses_read_error", "ulysses_read_error_info",
+           "ulysses_status_string", "ulysses_profile_enable", "ulysses_profile_read",
+           "ulysses_kernel_count", "ulysses_kernel_name",
            "ulysses_launch_count"]
 
 
@@ -67,11 +69,20 @@ def lib() -> ctypes.CDLL:
             L.ulysses_loss_workspace_size.argtypes = [i32, i64, i32, ctypes.POINTER(sz)]
             L.ulysses_loss_aggregate.argtypes = [i32, i64, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
             L.ulysses_read_error.argtypes = [ctypes.POINTER(i32)]
+            L.ulysses_read_error_info.argtypes = [ctypes.POINTER(i32), i32]
             L.ulysses_status_string.argtypes = [ctypes.c_int]
             L.ulysses_status_string.restype = ctypes.c_char_p
             L.ulysses_launch_count.restype = ctypes.c_uint64
+            L.ulysses_profile_enable.argtypes = [i32]
+            L.ulysses_profile_enable.restype = ctypes.c_int
+            L.ulysses_profile_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
+            L.ulysses_profile_read.restype = ctypes.c_int
+            L.ulysses_kernel_count.restype = i32
+            L.ulysses_kernel_name.argtypes = [i32]
+            L.ulysses_kernel_name.restype = ctypes.c_char_p
             for name in ("ulysses_attn_fwd", "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd",
-                         "ulysses_loss_workspace_size", "ulysses_loss_aggregate", "ulysses_read_error"):
+                         "ulysses_loss_workspace_size", "ulysses_loss_aggregate", "ulysses_read_error",
+                         "ulysses_read_error_info"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -111,7 +122,8 @@ def make_desc(B, n, P, H, G, d, dtype_code, mask, cu_seqlens=None, scale=0.0) ->
 def ulysses_seq_to_head(x: torch.Tensor, P: int, out: torch.Tensor | None = None, stream=None):
     """[P][B][n/P][heads][d] -> [P][B][heads/P][n][d] (bit-exact copy)."""
     P_, B, s, heads, d = x.shape
-    assert P_ == P
+    if P_ != P or heads % P:
+        raise UlyssesError(2, f"ulysses_seq_to_head: shape {tuple(x.shape)} with P={P}")
     n = P * s
     if out is None:
         out = torch.empty((P, B, heads // P, n, d), dtype=x.dtype, device=x.device)
@@ -123,7 +135,8 @@ def ulysses_seq_to_head(x: torch.Tensor, P: int, out: torch.Tensor | None = None
 def ulysses_head_to_seq(x: torch.Tensor, P: int, out: torch.Tensor | None = None, stream=None):
     """[P][B][heads/P][n][d] -> [P][B][n/P][heads][d] (bit-exact copy)."""
     P_, B, hl, n, d = x.shape
-    assert P_ == P
+    if P_ != P or hl == 0 or n % P:
+        raise UlyssesError(2, f"ulysses_head_to_seq: shape {tuple(x.shape)} with P={P}")
     heads = hl * P
     if out is None:
         out = torch.empty((P, B, n // P, heads, d), dtype=x.dtype, device=x.device)
@@ -214,9 +227,33 @@ def ulysses_read_error() -> int:
     return w.value
 
 
+def ulysses_read_error_info() -> list:
+    """Read and clear the whole error record (16 words, see the header)."""
+    buf = (ctypes.c_int32 * 16)()
+    _check(lib().ulysses_read_error_info(buf, 16), "ulysses_read_error_info")
+    return list(buf)
+
+
 def ulysses_status_string(status: int) -> str:
     return lib().ulysses_status_string(status).decode()
 
 
 def ulysses_launch_count() -> int:
     return int(lib().ulysses_launch_count())
+
+
+def ulysses_profile_enable(on: bool = True):
+    _check(lib().ulysses_profile_enable(1 if on else 0), "ulysses_profile_enable")
+
+
+def ulysses_profile_read() -> dict:
+    """{kernel name: (total device ms, launches)} for every kernel timed since
+    the last ulysses_profile_enable(True)."""
+    L = lib()
+    out = {}
+    for k in range(L.ulysses_kernel_count()):
+        ms, n = ctypes.c_double(0), ctypes.c_int64(0)
+        _check(L.ulysses_profile_read(k, ctypes.byref(ms), ctypes.byref(n)), "ulysses_profile_read")
+        if n.value:
+            out[L.ulysses_kernel_name(k).decode()] = (ms.value, n.value)
+    return out

@@ -56,6 +56,7 @@ def _load():
             lib.oracle_ulysses_bwd.argtypes = uly + [P, P, P, P, P, P, P]
             lib.oracle_head_rows.argtypes = [i, i, i, P, i, dbl, P, P, P, P, P, i, P, P, P]
             lib.oracle_kv_cols.argtypes = [i, i, i, P, i, dbl, i, P, P, P, P, P, i, P, P]
+            lib.oracle_head_rows_step.argtypes = [i, i, i, P, i, dbl, P, P, P, P, P, i, P, P, P, P, P]
             lib.oracle_loss.argtypes = [i, l, i, P, P, i, P, P, P]
             lib.oracle_loss.restype = l
             _lib = lib
@@ -212,6 +213,25 @@ def kv_cols(qs, douts, k, v, cols, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0)
                            ctypes.cast(qp, ctypes.c_void_p), ctypes.cast(dp, ctypes.c_void_p),
                            _ptr(k), _ptr(v), _ptr(cols), cols.size, _ptr(dk), _ptr(dv))
     return dk, dv
+
+
+def head_rows_step(q, k, v, dout, rows, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0, dk=None, dv=None):
+    """All the work of the listed query rows of one head (q, k, v, dout [n][d]):
+    returns O, LSE, dQ at those rows and adds their dK, dV terms into dk, dv
+    ([n][d] fp64, zero-initialised if not given)."""
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    n, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    cu, nd = _cu(cu_seqlens)
+    o = np.empty((rows.size, d), np.float64)
+    lse = np.empty(rows.size, np.float64)
+    dq = np.empty((rows.size, d), np.float64)
+    dk = np.zeros((n, d), np.float64) if dk is None else dk
+    dv = np.zeros((n, d), np.float64) if dv is None else dv
+    _load().oracle_head_rows_step(n, d, mask, _ptr(cu), nd, scale, _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(dout), _ptr(rows), rows.size, _ptr(o), _ptr(lse), _ptr(dq),
+                                  _ptr(dk), _ptr(dv))
+    return o, lse, dq, dk, dv
 
 
 # --------------------------------------------------------------------------

@@ -518,6 +518,67 @@ void oracle_kv_cols(int n, int d, int mask, const int *cu_seqlens, int num_docs,
   free(lse); free(Dv); free(need); free(doc);
 }
 
+/*
+ * Everything one query row i of one head contributes to the layer: O_i,
+ * lse_i, dQ_i, and its terms of dK_j = scale * sum_i dS_ij q_i and
+ * dV_j = sum_i P_ij dO_i for every visible key j, added into dk, dv ([n][d],
+ * zeroed by the caller).  Summed over all rows this is the whole forward and
+ * backward of the head; the benchmark times it on a uniform sample of rows.
+ * Rows are processed one after another; the key loop of a row runs in
+ * parallel (each key j is updated by exactly one thread).
+ */
+void oracle_head_rows_step(int n, int d, int mask, const int *cu_seqlens, int num_docs, double scale,
+                           const float *q, const float *k, const float *v, const float *dout,
+                           const int *rows, int nrows, double *o, double *lse, double *dq,
+                           double *dk, double *dv) {
+  attn_cfg c = make_cfg(n, d, mask, cu_seqlens, num_docs, scale);
+  int *doc = doc_index(&c);
+  double *p = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  double *ds = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  for (int e = 0; e < nrows; ++e) {
+    const int i = rows[e];
+    int lo, hi;
+    key_range(&c, doc, i, &lo, &hi);
+    double *oi = o + (size_t)e * d, *dqi = dq + (size_t)e * d;
+    for (int x = 0; x < d; ++x) { oi[x] = 0.0; dqi[x] = 0.0; }
+    if (hi < lo) { lse[e] = -INFINITY; continue; }
+    const float *qi = q + (size_t)i * d, *doi = dout + (size_t)i * d;
+#pragma omp parallel for schedule(static)
+    for (int j = lo; j <= hi; ++j) p[j] = c.scale * dot_f(qi, k + (size_t)j * d, d);
+    double m = -INFINITY;
+    for (int j = lo; j <= hi; ++j) if (p[j] > m) m = p[j];
+    double l = 0.0;
+    for (int j = lo; j <= hi; ++j) { p[j] = exp(p[j] - m); l += p[j]; }
+#pragma omp parallel for schedule(static)
+    for (int x = 0; x < d; ++x) {
+      double acc = 0.0;
+      for (int j = lo; j <= hi; ++j) acc += p[j] * (double)v[(size_t)j * d + x];
+      oi[x] = acc / l;
+    }
+    lse[e] = m + log(l);
+    double D = 0.0;
+    for (int x = 0; x < d; ++x) D += (double)doi[x] * oi[x];
+#pragma omp parallel for schedule(static)
+    for (int j = lo; j <= hi; ++j) {
+      const double P = p[j] / l;
+      const double dP = dot_f(doi, v + (size_t)j * d, d);
+      ds[j] = P * (dP - D);
+      double *dkj = dk + (size_t)j * d, *dvj = dv + (size_t)j * d;
+      for (int x = 0; x < d; ++x) {
+        dkj[x] += c.scale * ds[j] * (double)qi[x];
+        dvj[x] += P * (double)doi[x];
+      }
+    }
+#pragma omp parallel for schedule(static)
+    for (int x = 0; x < d; ++x) {
+      double acc = 0.0;
+      for (int j = lo; j <= hi; ++j) acc += ds[j] * (double)k[(size_t)j * d + x];
+      dqi[x] = c.scale * acc;
+    }
+  }
+  free(p); free(ds); free(doc);
+}
+
 /* ------------------------------------------------------------------------- */
 /* Token-weighted loss aggregation over the P shards.                         */
 /* ------------------------------------------------------------------------- */

@@ -35,10 +35,22 @@ def max_abs(a, b):
     return float(np.abs(a - b).max()) if a.size else 0.0
 
 
+BF16_ULP_REL = 2.0 ** -7   # one bf16 ulp is at most 2^-7 |x| (8 significant bits)
+
+
 def assert_bf16_close(got, ref, what="", max_abs_tol=BF16_MAX_ABS, rel_tol=BF16_REL_L2):
-    ma, rl = max_abs(got, ref), rel_l2(got, ref)
-    assert np.isfinite(to64(got)).all(), f"{what}: non-finite values"
-    assert ma <= max_abs_tol and rl <= rel_tol, f"{what}: max_abs={ma:.3e} rel_l2={rl:.3e}"
+    """Element-wise |got - ref| <= max(2e-2, one bf16 ulp of |ref|) and
+    relative L2 <= 1e-2.  The ulp term only matters for |ref| > 2.56, where a
+    bf16 output cannot resolve 2e-2 (the exact value rounded to bf16 may
+    already be 2^-8 |ref| away); below that the bound is the plain 2e-2."""
+    g, r = to64(got), to64(ref)
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    err = np.abs(g - r)
+    bound = np.maximum(max_abs_tol, BF16_ULP_REL * np.abs(r))
+    worst = float((err / bound).max()) if err.size else 0.0
+    ma, rl = (float(err.max()) if err.size else 0.0), rel_l2(g, r)
+    assert worst <= 1.0 and rl <= rel_tol, \
+        f"{what}: max_abs={ma:.3e} (worst err/bound {worst:.2f}) rel_l2={rl:.3e}"
     return ma, rl
 
 

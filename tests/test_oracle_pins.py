@@ -336,6 +336,23 @@ def test_sampled_rows_and_columns_match_full(mask):
     assert np.abs(cv - dv[0, cols, 0]).max() < 1e-12
 
 
+@pytest.mark.parametrize("mask", [MASK_CAUSAL, MASK_DOC_CAUSAL, MASK_NONE])
+def test_row_step_sums_to_full_backward(mask):
+    """The per-row step (used to time the oracle on a row sample) summed over
+    every row gives exactly the full forward and backward of the head."""
+    n, d = 48, 8
+    q, k, v, do = _randn(1, n, 1, d), _randn(1, n, 1, d), _randn(1, n, 1, d), _randn(1, n, 1, d)
+    cu = np.array([0, 11, 30, n], np.int32) if mask == MASK_DOC_CAUSAL else None
+    o, lse = oracle.attention_fwd(q, k, v, mask=mask, cu_seqlens=cu)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, mask=mask, cu_seqlens=cu)
+    rows = np.arange(n)
+    so, sl, sdq, sdk, sdv = oracle.head_rows_step(q[0, :, 0], k[0, :, 0], v[0, :, 0], do[0, :, 0], rows,
+                                                  mask=mask, cu_seqlens=cu)
+    assert np.abs(so - o[0, :, 0]).max() < 1e-12 and np.abs(sl - lse[0, 0]).max() < 1e-12
+    assert np.abs(sdq - dq[0, :, 0]).max() < 1e-12
+    assert np.abs(sdk - dk[0, :, 0]).max() < 1e-12 and np.abs(sdv - dv[0, :, 0]).max() < 1e-12
+
+
 # ----------------------------------------------------------------------- loss
 
 def test_loss_uniform_logits_closed_form():
