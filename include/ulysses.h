@@ -148,6 +148,33 @@ uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab,
                                   float *shard_sum, int64_t *shard_count, float *loss,
                                   void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the fixed scratch array behind ulysses_loss_aggregate_noalloc. */
+#define ULYSSES_NOALLOC_LOSS_SCRATCH_BYTES 65536
+
+/*
+ * ulysses_loss_aggregate without a workspace argument, for callers that
+ * cannot allocate device memory: hosts that pass the library only their input
+ * and output buffers and own every allocation, or processes that allow no
+ * device allocation after start-up.  The method's pages have no counterpart
+ * of this call; it exists for those callers.
+ * Same arguments, results and errors as ulysses_loss_aggregate, except:
+ *  - the partial sums live in a fixed 64 KiB device array inside the library
+ *    (held on every GPU that loads it until the process exits); shapes whose
+ *    partials need more (more than 4096 of them: P * blocks per shard, about
+ *    P > 3500 ranks) return ULY_ERR_WORKSPACE and launch nothing;
+ *  - all calls share that array: calls that overlap on the GPU (unordered
+ *    streams) race and give wrong results; nothing in it needs clearing
+ *    between calls (every slot is written before it is read within a call);
+ *  - the first call on a device looks up the array's address on that device,
+ *    so make that first call before any stream capture.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+uly_status ulysses_loss_aggregate_noalloc(int32_t world, int64_t tokens, int32_t vocab,
+                                          int32_t logit_dtype, const void *logits,
+                                          const int32_t *labels, int32_t ignore_index,
+                                          float *shard_sum, int64_t *shard_count, float *loss,
+                                          void *stream);
+
 /* Asynchronous error word of the current device: reads it (synchronising the
  * device) into *word (bit s set <=> status s was raised) and clears it. */
 uly_status ulysses_read_error(int32_t *word);
