@@ -152,19 +152,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && T > 0) {
       bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
       tc_fence_after();
+      const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
       auto issue_sdp = [&](int t) -> bool {
         const int w = t & 1, s = t % kStages;
         if (!mbar_wait(bar(B_SF_ + s), (t / kStages) & 1, abort_flag, prm.err)) return false;
         tc_fence_after();
         const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
+        const uint64_t dQ = sdesc_sw128(st, 16, 1024), dO = sdesc_sw128(st + kQBytes, 16, 1024);
         const uint32_t tS = tmem + 256 + 128 * w;
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32, qo = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_bf16_ss(tS, sdesc_sw128(sb + kOffK + ko, 16, 1024), sdesc_sw128(st + qo, 16, 1024),
-                      kIdescN64, kk > 0);
-          mma_bf16_ss(tS + 64, sdesc_sw128(sb + kOffV + ko, 16, 1024),
-                      sdesc_sw128(st + kQBytes + qo, 16, 1024), kIdescN64, kk > 0);
+          mma_bf16_ss(tS, sdesc_add(dK, ko), sdesc_add(dQ, qo), kIdescN64, kk > 0);
+          mma_bf16_ss(tS + 64, sdesc_add(dV, ko), sdesc_add(dO, qo), kIdescN64, kk > 0);
         }
         tc_commit(bar(B_S + w));
         return true;
@@ -178,13 +178,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
         const uint32_t pt = sb + kOffPT + w * 32768, dst = pt + 16384;
+        const uint64_t dPt = sdesc_sw128(pt, 16, 1024), dSt = sdesc_sw128(dst, 16, 1024);
+        const uint64_t dOm = sdesc_sw128(st + kQBytes, 8192, 1024), dQm = sdesc_sw128(st, 8192, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk) {
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ss(tmem + 0, sdesc_sw128(pt + kk * 32, 16, 1024),
-                      sdesc_sw128(st + kQBytes + kk * 2048, 8192, 1024), kIdescN128MN, acc);
-          mma_bf16_ss(tmem + 128, sdesc_sw128(dst + kk * 32, 16, 1024),
-                      sdesc_sw128(st + kk * 2048, 8192, 1024), kIdescN128MN, acc);
+          mma_bf16_ss(tmem + 0, sdesc_add(dPt, kk * 32), sdesc_add(dOm, kk * 2048), kIdescN128MN, acc);
+          mma_bf16_ss(tmem + 128, sdesc_add(dSt, kk * 32), sdesc_add(dQm, kk * 2048), kIdescN128MN, acc);
         }
         tc_commit(bar(B_SE + s));
         if (t + 2 < T) ok = issue_sdp(t + 2);
@@ -206,27 +206,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + 256 + 128 * w;
     const uint32_t pt = sb + kOffPT + w * 32768, dst = pt + 16384;
     float *lsm = reinterpret_cast<float *>(smem + kOffLD + w * 512);  // [0,64) lse*log2e, [64,128) D
+    // this thread's share of the per-tile statistics: LSE (tid < 64) or D of
+    // query row i0 + (tid & 63); fetched one tile ahead of its use
+    auto fetch_stat = [&](int t) -> float {
+      if (t >= T) return 0.f;
+      const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
+      const int i = i0 + (tid & 63);
+      const long long idx = (long long)(qh_base + e) * g.n + i;
+      if (tid < 64) return (i < g.n) ? __ldg(prm.lse + idx) * kLog2e : INFINITY;
+      return (i < g.n) ? __ldg(prm.Dv + idx) : 0.f;
+    };
+    float stat_next = fetch_stat(w);
     bool ok = true;
     for (int t = w; t < T; t += 2) {
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
-      const int qh = qh_base + e;
       named_bar_sync(1 + w, 128);              // previous tile's LSE/D reads are done
-      {
-        const int c = tid & 63, i = i0 + c;
-        if (tid < 64) lsm[c] = (i < g.n) ? prm.lse[(long long)qh * g.n + i] * kLog2e : INFINITY;
-        else lsm[64 + c] = (i < g.n) ? prm.Dv[(long long)qh * g.n + i] : 0.f;
-      }
+      lsm[tid] = stat_next;
       named_bar_sync(1 + w, 128);
+      stat_next = fetch_stat(t + 2);           // in flight while this tile is processed
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + w), (t >> 1) & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + kBQ - 1 <= hi_a) && (i0 + kBQ <= g.n) &&
-                        (n0 + kBN <= g.n) && (prm.mk.mask != ULY_MASK_DOC_CAUSAL || i0 + kBQ - 1 <= hi_a);
+                        (n0 + kBN <= g.n);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        uint32_t rs[32], rd[32];
-        tmem_ld32(tS + ch * 32, rs);
-        tmem_ld32(tS + 64 + ch * 32, rd);
+        uint32_t r[64];                        // r[0..31] S^T, r[32..63] dP^T
+        tmem_ld32x2(tS + ch * 32, tS + 64 + ch * 32, r);
         uint32_t pp[16], dd[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
@@ -234,13 +240,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int c = ch * 32 + x + u;
-            float pv = exp2f(fmaf(__uint_as_float(rs[x + u]), prm.scale_log2, -lsm[c]));
+            float pv = ex2_approx(fmaf(__uint_as_float(r[x + u]), prm.scale_log2, -lsm[c]));
             if (!full) {
               const int i = i0 + c;
               if (i < lo_j || i > hi_j) pv = 0.f;
             }
             p[u] = pv;
-            ds[u] = pv * (__uint_as_float(rd[x + u]) - lsm[64 + c]);
+            ds[u] = pv * (__uint_as_float(r[32 + x + u]) - lsm[64 + c]);
           }
           pp[x >> 1] = pack_bf16x2(p[0], p[1]);
           dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
@@ -389,14 +395,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && NT > 0) {
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err);
       tc_fence_after();
+      const uint64_t dQ0 = sdesc_sw128(sb + kOffQ, 16, 1024), dQ1 = sdesc_sw128(sb + kOffQ + kQBytes, 16, 1024);
+      const uint64_t dO0 = sdesc_sw128(sb + kOffO, 16, 1024), dO1 = sdesc_sw128(sb + kOffO + kQBytes, 16, 1024);
+      const uint64_t dS0 = sdesc_sw128(sb + kOffDS, 16, 1024), dS1 = sdesc_sw128(sb + kOffDS + 16384, 16, 1024);
       auto issue_dq = [&](int t, int j) {
         // dQ_t += dS_t K_j   (A = dS K-major, B = K tile MN-major over d)
-        const uint32_t kst = sb + kOffKV + (j % kStages) * 2 * kKBytes;
-        const uint32_t ds = sb + kOffDS + t * 16384;
+        const uint64_t dKm = sdesc_sw128(sb + kOffKV + (j % kStages) * 2 * kKBytes, 8192, 1024);
+        const uint64_t dS = t ? dS1 : dS0;
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_bf16_ss(tmem + 256 * t + 128, sdesc_sw128(ds + kk * 32, 16, 1024),
-                      sdesc_sw128(kst + kk * 2048, 8192, 1024), kIdescN128MN, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ss(tmem + 256 * t + 128, sdesc_add(dS, kk * 32), sdesc_add(dKm, kk * 2048), kIdescN128MN,
+                      (j > 0 || kk > 0) ? 1u : 0u);
       };
       for (int j = 0; ok && j < NT; ++j) {
         const int s = j % kStages;
@@ -404,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t kst = sb + kOffKV + s * 2 * kKBytes;
+        const uint64_t dK = sdesc_sw128(kst, 16, 1024), dV = sdesc_sw128(kst + kKBytes, 16, 1024);
         for (int t = 0; t < 2 && ok; ++t) {
           if (j > 0) {
             ok = mbar_wait(bar(B_P + t), (j - 1) & 1, abort_flag, prm.err);
@@ -411,14 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             issue_dq(t, j - 1);
           }
-          const uint32_t q = sb + kOffQ + t * kQBytes, o = sb + kOffO + t * kQBytes;
+          const uint64_t dQ = t ? dQ1 : dQ0, dO = t ? dO1 : dO0;
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
             const uint32_t qo = (kk >> 2) * 16384 + (kk & 3) * 32, ko = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + 256 * t, sdesc_sw128(q + qo, 16, 1024), sdesc_sw128(kst + ko, 16, 1024),
-                        kIdescN64, kk > 0);
-            mma_bf16_ss(tmem + 256 * t + 64, sdesc_sw128(o + qo, 16, 1024),
-                        sdesc_sw128(kst + kKBytes + ko, 16, 1024), kIdescN64, kk > 0);
+            mma_bf16_ss(tmem + 256 * t, sdesc_add(dQ, qo), sdesc_add(dK, ko), kIdescN64, kk > 0);
+            mma_bf16_ss(tmem + 256 * t + 64, sdesc_add(dO, qo), sdesc_add(dV, ko), kIdescN64, kk > 0);
           }
           tc_commit(bar(B_S + t));
         }
@@ -460,21 +468,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (n0 >= lo_last) && (n0 + kBK - 1 <= hi_first) && (n0 + kBK <= g.n);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        uint32_t rs[32], rd[32];
-        tmem_ld32(tS + ch * 32, rs);
-        tmem_ld32(tS + 64 + ch * 32, rd);
+        uint32_t r[64];                        // r[0..31] S, r[32..63] dP
+        tmem_ld32x2(tS + ch * 32, tS + 64 + ch * 32, r);
         uint32_t dd[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           float ds[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            float pv = exp2f(fmaf(__uint_as_float(rs[x + u]), prm.scale_log2, -lse2));
+            float pv = ex2_approx(fmaf(__uint_as_float(r[x + u]), prm.scale_log2, -lse2));
             if (!full) {
               const int jj = n0 + ch * 32 + x + u;
               if (jj < lo_i || jj > hi_i) pv = 0.f;
             }
-            ds[u] = pv * (__uint_as_float(rd[x + u]) - Di);
+            ds[u] = pv * (__uint_as_float(r[32 + x + u]) - Di);
           }
           dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
         }

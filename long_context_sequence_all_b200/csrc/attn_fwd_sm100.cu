@@ -9,21 +9,25 @@
 // the same mask: K/V are loaded once for 256 query rows.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K_j, V_j into a 3-slot ring
+//   warp 0      TMA producer: Q tiles once, then K_j, V_j into a 5-slot ring
 //   warp 1      TMEM allocator and MMA issuer (one thread):
 //                 S_t = Q_t K_j^T          (M=128 N=128 K=128, SS, into TMEM)
-//                 O_t += P_t V_j           (M=128 N=128 K=128, SS, into TMEM)
+//                 O_t += P_t V_j           (M=128 N=128 K=128, P from TMEM, V from smem)
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread
 //               per query row reads its S row from TMEM, keeps the running
-//               max / sum, writes P (bf16) to shared memory in the MMA's
-//               swizzled layout, rescales O in TMEM when the max moved by more
+//               max / sum, writes P (bf16 pairs) back into the TMEM columns of
+//               S it has already read, rescales O in TMEM when the max moved by more
 //               than 2^8, and finally normalises O and writes O and LSE.
-// TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512) columns.
+// TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512) columns; P_t
+// occupies columns [0,64) of S_t.  P never touches shared memory, so the
+// P V product reads only V from shared memory.
 //
 // Ordering: s_full[t] is committed after S_j(t), which is issued after
 // O_t += P_{j-1} V_{j-1}; a commit tracks every earlier MMA of the thread, so
 // when softmax sees S_j it also knows the previous PV finished (O may be
-// rescaled, P may be overwritten).  p_full[t] hands P_j back to the MMA warp.
+// rescaled).  p_full[t] hands P_j to the MMA warp.  S_{j+1}(t) overwrites the
+// columns that O_t += P_j V_j reads; both are MMAs of this one issuing thread
+// and the tensor core executes them in issue order.
 // Every wait is bounded (ULY_ERR_TIMEOUT), no wait can spin forever.
 #include "prof.cuh"
 #include "sm100.cuh"
@@ -36,11 +40,10 @@ namespace {
 
 constexpr int kBM = 128, kBN = 128, kHD = 128;
 constexpr int kThreads = 384;
-constexpr int kSlots = 3;
+constexpr int kSlots = 5;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;       // one 128 x 128 bf16 tile
 constexpr uint32_t kOffQ = 0;                        // 2 tiles
-constexpr uint32_t kOffP = 2 * kTileBytes;           // 2 tiles
-constexpr uint32_t kOffKV = 4 * kTileBytes;          // kSlots tiles
+constexpr uint32_t kOffKV = 2 * kTileBytes;          // kSlots tiles
 constexpr uint32_t kOffBar = kOffKV + kSlots * kTileBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
 constexpr float kLog2e = 1.4426950408889634f;
@@ -142,6 +145,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && NT > 0) {
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err);
       tc_fence_after();
+      // descriptors of the fixed operands; per-k-step offsets are constants
+      const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dq1 = sdesc_sw128(sb + kOffQ + kTileBytes, 16, 1024);
+      auto issue_pv = [&](int t, uint32_t v_base, bool first) {
+        const uint64_t dv = sdesc_sw128(v_base, 16384, 1024);   // V: MN-major
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, sdesc_add(dv, kk * 2048), kIdescPV,
+                      (!first || kk > 0) ? 1u : 0u);
+      };
+      auto issue_s = [&](int t, uint32_t k_base) {
+        const uint64_t dk = sdesc_sw128(k_base, 16, 1024);
+        const uint64_t dq = t ? dq1 : dq0;
+#pragma unroll
+        for (int kk = 0; kk < kHD / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + t * 128, sdesc_add(dq, koff), sdesc_add(dk, koff), kIdescS, kk > 0 ? 1u : 0u);
+        }
+      };
       for (int it = 0; ok && it < NT; ++it) {
         const int idxK = 2 * it, slotK = idxK % kSlots;
         ok = mbar_wait(bar(B_KVF + slotK), (idxK / kSlots) & 1, abort_flag, prm.err);
@@ -159,21 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(bar(B_PF + t), (it - 1) & 1, abort_flag, prm.err);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t p_base = sb + kOffP + t * kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              const uint64_t ad = sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(v_base + kk * 2048, 16384, 1024);
-              mma_bf16_ss(tmem + 256 + t * 128, ad, bd, kIdescPV, (it > 1 || kk > 0) ? 1u : 0u);
-            }
+            issue_pv(t, v_base, it == 1);
           }
-          const uint32_t q_base = sb + kOffQ + t * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + t * 128, sdesc_sw128(q_base + koff, 16, 1024),
-                        sdesc_sw128(k_base + koff, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          }
+          issue_s(t, k_base);
           tc_commit(bar(B_SF + t));
         }
         if (!ok) break;
@@ -189,13 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(bar(B_PF + t), (NT - 1) & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t p_base = sb + kOffP + t * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(v_base + kk * 2048, 16384, 1024);
-            mma_bf16_ss(tmem + 256 + t * 128, ad, bd, kIdescPV, (NT > 1 || kk > 0) ? 1u : 0u);
-          }
+          issue_pv(t, v_base, NT == 1);
           tc_commit(bar(B_OF + t));
         }
         if (ok) tc_commit(bar(B_KVE + slotV));
@@ -218,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + wg * 128;
     const uint32_t tO = tmem + lane_off + 256 + wg * 128;
-    const uint32_t p_base = sb + kOffP + wg * kTileBytes;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int it = 0; it < NT; ++it) {
@@ -228,64 +231,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = (jt0 + it) * kBN;
       // the tile needs no element mask when every row of the CTA sees all of it
       const bool full = (n0 >= lo_last) && (n0 + kBN - 1 <= hi_first) && (n0 + kBN <= g.n);
-      uint32_t r[32];
-      float mx = -INFINITY;
+      // pass 1: row maximum of the raw scores (the scale is positive, so the
+      // maximum commutes with it); eight independent chains
+      uint32_t r[64];
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tS + c * 32, r);
+      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          float sv = __uint_as_float(r[x]) * prm.scale_log2;
+      for (int h2 = 0; h2 < 2; ++h2) {
+        tmem_ld32x2(tS + h2 * 64, tS + h2 * 64 + 32, r);
+#pragma unroll
+        for (int x = 0; x < 64; ++x) {
+          float sv = __uint_as_float(r[x]);
           if (!full) {
-            const int j = n0 + c * 32 + x;
+            const int j = n0 + h2 * 64 + x;
             if (j < lo_i || j > hi_i) sv = -INFINITY;
           }
-          mx = fmaxf(mx, sv);
+          mx8[x & 7] = fmaxf(mx8[x & 7], sv);
         }
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * prm.scale_log2;
       const float m_new = fmaxf(m_run, mx);
       const bool had = m_run != -INFINITY;
       const bool rescale = had && (m_new > m_run + kRescaleThreshold);
       if (!had) {
         m_run = m_new;
       } else if (rescale) {
-        l_run *= exp2f(m_run - m_new);
+        l_run *= ex2_approx(m_run - m_new);
       }
       if (__any_sync(0xffffffffu, rescale)) {
-        const float a = rescale ? exp2f(m_run - m_new) : 1.f;
+        const float a = rescale ? ex2_approx(m_run - m_new) : 1.f;
+        uint32_t ro[32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tO + c * 32, r);
+          tmem_ld32(tO + c * 32, ro);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * a);
-          tmem_st32(tO + c * 32, r);
+          for (int x = 0; x < 32; ++x) ro[x] = __float_as_uint(__uint_as_float(ro[x]) * a);
+          tmem_st32(tO + c * 32, ro);
         }
       }
       if (rescale) m_run = m_new;
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      // pass 2: P = 2^(s * scale * log2 e - m), written to shared memory as
+      // bf16 in the MMA's swizzled layout; eight independent sum chains
+      float ls8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tS + c * 32, r);
-        uint32_t pk[16];
+      for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float s0 = __uint_as_float(r[x]) * prm.scale_log2;
-          float s1 = __uint_as_float(r[x + 1]) * prm.scale_log2;
-          if (!full) {
-            const int j = n0 + c * 32 + x;
-            if (j < lo_i || j > hi_i) s0 = -INFINITY;
-            if (j + 1 < lo_i || j + 1 > hi_i) s1 = -INFINITY;
+      for (int h2 = 0; h2 < 2; ++h2) {
+        tmem_ld32x2(tS + h2 * 64, tS + h2 * 64 + 32, r);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = hh * 32; x < hh * 32 + 32; x += 2) {
+            float s0 = fmaf(__uint_as_float(r[x]), prm.scale_log2, -m_use);
+            float s1 = fmaf(__uint_as_float(r[x + 1]), prm.scale_log2, -m_use);
+            if (!full) {
+              const int j = n0 + h2 * 64 + x;
+              if (j < lo_i || j > hi_i) s0 = -INFINITY;
+              if (j + 1 < lo_i || j + 1 > hi_i) s1 = -INFINITY;
+            }
+            const float p0 = ex2_approx(s0), p1 = ex2_approx(s1);
+            ls8[x & 7] += p0;
+            ls8[(x & 7) + 1] += p1;
+            pk[(x - hh * 32) >> 1] = pack_bf16x2(p0, p1);
           }
-          const float p0 = exp2f(s0 - m_use), p1 = exp2f(s1 - m_use);
-          l_run += p0 + p1;
-          pk[x >> 1] = pack_bf16x2(p0, p1);
+          // P (bf16 pairs) overwrites S columns [32*h2 + 16*hh, +16), already read
+          tmem_st16_nowait(tS + h2 * 32 + hh * 16, pk);
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          st_shared_v4(p_base + sw128_offset(row, c * 4 + u), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                       pk[4 * u + 3]);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       tc_fence_before();
       mbar_arrive(bar(B_PF + wg));
     }
