@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import concurrent.futures as cf
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -37,14 +38,37 @@ def _deps_mtime() -> float:
     return max(os.path.getmtime(f) for f in files)
 
 
+# Kernels that split their register pool between warpgroups with setmaxnreg:
+# the split only adds up when the kernel launches with exactly this many
+# registers per thread; any other count would make setmaxnreg.inc wait forever.
+REGISTER_SPLIT_KERNELS = {"attn_fwd_sm100.cu": ("attn_fwd_sm100_kernel", 168)}
+
+
+def _check_register_split(src: str, ptxas_log: str):
+    kernel, want = REGISTER_SPLIT_KERNELS[src]
+    lines = ptxas_log.splitlines()
+    for i, line in enumerate(lines):
+        if "Compiling entry function" in line and kernel in line:
+            for nxt in lines[i + 1:i + 6]:
+                m = re.search(r"Used (\d+) registers", nxt)
+                if m:
+                    if int(m.group(1)) != want:
+                        raise RuntimeError(f"{kernel} uses {m.group(1)} registers, its warpgroup register "
+                                           f"split needs exactly {want}; refusing to build")
+                    return
+    raise RuntimeError(f"ptxas report for {kernel} not found; refusing to build")
+
+
 def _compile(src: str, verbose: bool) -> str:
     obj = os.path.join(BUILD, src.replace(".cu", ".o"))
     cmd = [nvcc(), *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
-    if verbose:
+    if verbose or src in REGISTER_SPLIT_KERNELS:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
+    if src in REGISTER_SPLIT_KERNELS:
+        _check_register_split(src, r.stdout + r.stderr)
     if verbose and (r.stdout or r.stderr):
         print(r.stdout + r.stderr, file=sys.stderr)
     return obj

@@ -49,6 +49,9 @@ constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment s
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
+constexpr int kRegsLaunch = 168, kRegsCtl = 88, kRegsSoftmax = 208;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax == kThreads * kRegsLaunch,
+              "register split must use exactly the launch pool");
 
 constexpr uint32_t kIdescS = sm100::idesc_bf16_f32(128, 128, false, false);   // Q K^T
 constexpr uint32_t kIdescPV = sm100::idesc_bf16_f32(128, 128, false, true);   // P V (V MN-major)
@@ -114,7 +117,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  // Registers: the producer / MMA warpgroup (warps 0-3) keeps 88 per thread,
+  // each softmax warpgroup gets 208 so a thread can hold a whole 128-column
+  // row of S.  128*88 + 256*208 = 384*168, the block's pool at launch.
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsCtl>();
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0 && NT > 0) {
@@ -210,7 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int wg = (warp - 4) >> 2;        // query tile 0 or 1
     const int wq = warp & 3;               // TMEM lane quarter of this warp
@@ -231,25 +240,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = (jt0 + it) * kBN;
       // the tile needs no element mask when every row of the CTA sees all of it
       const bool full = (n0 >= lo_last) && (n0 + kBN - 1 <= hi_first) && (n0 + kBN <= g.n);
-      // pass 1: row maximum of the raw scores (the scale is positive, so the
-      // maximum commutes with it); eight independent chains
-      uint32_t r[64];
+      // One read of the whole 128-column row of S from TMEM.
+      uint32_t r[128];
+      tmem_ld128(tS, r);
+      if (!full) {
+#pragma unroll
+        for (int x = 0; x < 128; ++x) {
+          const int j = n0 + x;
+          if (j < lo_i || j > hi_i) r[x] = __float_as_uint(-INFINITY);
+        }
+      }
+      // row maximum of the raw scores (the scale is positive, so the maximum
+      // commutes with it); eight independent chains
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        tmem_ld32x2(tS + h2 * 64, tS + h2 * 64 + 32, r);
-#pragma unroll
-        for (int x = 0; x < 64; ++x) {
-          float sv = __uint_as_float(r[x]);
-          if (!full) {
-            const int j = n0 + h2 * 64 + x;
-            if (j < lo_i || j > hi_i) sv = -INFINITY;
-          }
-          mx8[x & 7] = fmaxf(mx8[x & 7], sv);
-        }
-      }
+      for (int x = 0; x < 128; ++x) mx8[x & 7] = fmaxf(mx8[x & 7], __uint_as_float(r[x]));
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * prm.scale_log2;
       const float m_new = fmaxf(m_run, mx);
@@ -262,48 +269,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (__any_sync(0xffffffffu, rescale)) {
         const float a = rescale ? ex2_approx(m_run - m_new) : 1.f;
-        uint32_t ro[32];
+        uint32_t ro[16];
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          tmem_ld16(tO + c * 16, ro);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tO + c * 32, ro);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) ro[x] = __float_as_uint(__uint_as_float(ro[x]) * a);
-          tmem_st32(tO + c * 32, ro);
+          for (int x = 0; x < 16; ++x) ro[x] = __float_as_uint(__uint_as_float(ro[x]) * a);
+          tmem_st16_nowait(tO + c * 16, ro);
+          tmem_st_wait();
         }
       }
       if (rescale) m_run = m_new;
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2: P = 2^(s * scale * log2 e - m), written to shared memory as
-      // bf16 in the MMA's swizzled layout; eight independent sum chains
+      // P = 2^(s * scale * log2 e - m) as bf16 pairs into TMEM columns [0, 64)
+      // of S (already read); eight independent sum chains
       float ls8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        tmem_ld32x2(tS + h2 * 64, tS + h2 * 64 + 32, r);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = hh * 32; x < hh * 32 + 32; x += 2) {
-            float s0 = fmaf(__uint_as_float(r[x]), prm.scale_log2, -m_use);
-            float s1 = fmaf(__uint_as_float(r[x + 1]), prm.scale_log2, -m_use);
-            if (!full) {
-              const int j = n0 + h2 * 64 + x;
-              if (j < lo_i || j > hi_i) s0 = -INFINITY;
-              if (j + 1 < lo_i || j + 1 > hi_i) s1 = -INFINITY;
-            }
-            const float p0 = ex2_approx(s0), p1 = ex2_approx(s1);
-            ls8[x & 7] += p0;
-            ls8[(x & 7) + 1] += p1;
-            pk[(x - hh * 32) >> 1] = pack_bf16x2(p0, p1);
-          }
-          // P (bf16 pairs) overwrites S columns [32*h2 + 16*hh, +16), already read
-          tmem_st16_nowait(tS + h2 * 32 + hh * 16, pk);
+        for (int x = hh * 64; x < hh * 64 + 64; x += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[x]), prm.scale_log2, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[x + 1]), prm.scale_log2, -m_use));
+          ls8[x & 7] += p0;
+          ls8[(x & 7) + 1] += p1;
+          pk[(x - hh * 64) >> 1] = pack_bf16x2(p0, p1);
         }
+        tmem_st32_nowait(tS + hh * 32, pk);
       }
-      tmem_st_wait();
       l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_PF + wg));
     }
