@@ -41,22 +41,30 @@ def _deps_mtime() -> float:
 # Kernels that split their register pool between warpgroups with setmaxnreg:
 # the split only adds up when the kernel launches with exactly this many
 # registers per thread; any other count would make setmaxnreg.inc wait forever.
-REGISTER_SPLIT_KERNELS = {"attn_fwd_sm100.cu": ("attn_fwd_sm100_kernel", 168)}
+REGISTER_SPLIT_KERNELS = {
+    "attn_fwd_sm100.cu": [("attn_fwd_sm100_kernel", 168)],
+    "attn_bwd_sm100.cu": [("attn_dkdv_sm100_kernel", 168), ("attn_dq_sm100_kernel", 168)],
+}
 
 
 def _check_register_split(src: str, ptxas_log: str):
-    kernel, want = REGISTER_SPLIT_KERNELS[src]
     lines = ptxas_log.splitlines()
-    for i, line in enumerate(lines):
-        if "Compiling entry function" in line and kernel in line:
-            for nxt in lines[i + 1:i + 6]:
-                m = re.search(r"Used (\d+) registers", nxt)
-                if m:
-                    if int(m.group(1)) != want:
-                        raise RuntimeError(f"{kernel} uses {m.group(1)} registers, its warpgroup register "
-                                           f"split needs exactly {want}; refusing to build")
-                    return
-    raise RuntimeError(f"ptxas report for {kernel} not found; refusing to build")
+    for kernel, want in REGISTER_SPLIT_KERNELS[src]:
+        found = False
+        for i, line in enumerate(lines):
+            if "Compiling entry function" in line and kernel in line:
+                for nxt in lines[i + 1:i + 6]:
+                    m = re.search(r"Used (\d+) registers", nxt)
+                    if m:
+                        if int(m.group(1)) != want:
+                            raise RuntimeError(f"{kernel} uses {m.group(1)} registers, its warpgroup register "
+                                               f"split needs exactly {want}; refusing to build")
+                        found = True
+                        break
+            if found:
+                break
+        if not found:
+            raise RuntimeError(f"ptxas report for {kernel} not found; refusing to build")
 
 
 def _compile(src: str, verbose: bool) -> str:

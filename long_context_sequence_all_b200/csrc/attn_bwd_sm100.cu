@@ -40,6 +40,13 @@ constexpr int kHD = 128;
 constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCtlKV = 136, kRegsComputeKV = 184;  // dK/dV kernel
+constexpr int kRegsCtlQ = 120, kRegsComputeQ = 192;    // dQ kernel
+static_assert(128 * kRegsCtlKV + 256 * kRegsComputeKV == kThreads * kRegsLaunch &&
+                  128 * kRegsCtlQ + 256 * kRegsComputeQ == kThreads * kRegsLaunch,
+              "register split must use exactly the launch pool");
+
 constexpr uint32_t kIdescN64 = idesc_bf16_f32(128, 64, false, false);    // K-major A and B, N = 64
 constexpr uint32_t kIdescN128MN = idesc_bf16_f32(128, 128, false, true); // B MN-major, N = 128
 
@@ -123,7 +130,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: dV [0,128) dK [128,256); WG w: S^T [256+128w, +64), dP^T [+64, +64)
+  // Registers: producer / MMA warpgroup 136 per thread, the two compute
+  // warpgroups 184 (a thread holds its whole 128-column S^T | dP^T row).
 
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsCtlKV>();
   if (warp == 0) {
     if (lane == 0 && T > 0) {
       mbar_arrive_expect_tx(bar(B_KV), 2 * kKVBytes);
@@ -195,7 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsComputeKV>();
     const int w = (warp - 4) >> 2, wq = warp & 3;
     const int row = wq * 32 + lane;            // key row within the tile
     const int j = n0 + row;
@@ -229,10 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + kBQ - 1 <= hi_a) && (i0 + kBQ <= g.n) &&
                         (n0 + kBN <= g.n);
+      uint32_t r[128];                         // r[0..63] S^T, r[64..127] dP^T: one read
+      tmem_ld128(tS, r);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        uint32_t r[64];                        // r[0..31] S^T, r[32..63] dP^T
-        tmem_ld32x2(tS + ch * 32, tS + 64 + ch * 32, r);
         uint32_t pp[16], dd[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
@@ -240,13 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int c = ch * 32 + x + u;
-            float pv = ex2_approx(fmaf(__uint_as_float(r[x + u]), prm.scale_log2, -lsm[c]));
+            float pv = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lsm[c]));
             if (!full) {
               const int i = i0 + c;
               if (i < lo_j || i > hi_j) pv = 0.f;
             }
             p[u] = pv;
-            ds[u] = pv * (__uint_as_float(r[32 + x + u]) - lsm[64 + c]);
+            ds[u] = pv * (__uint_as_float(r[64 + c]) - lsm[64 + c]);
           }
           pp[x >> 1] = pack_bf16x2(p[0], p[1]);
           dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
@@ -365,7 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns, tile t: S [256t, +64), dP [256t+64, +64), dQ [256t+128, +128)
+  // Registers: producer / MMA warpgroup 120 per thread, the two compute
+  // warpgroups 192 (a thread holds its whole 128-column S | dP row).
 
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsCtlQ>();
   if (warp == 0) {
     if (lane == 0 && NT > 0) {
       mbar_arrive_expect_tx(bar(B_Q), 4 * kQBytes);
@@ -446,7 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsComputeQ>();
     const int t = (warp - 4) >> 2, wq = warp & 3;
     const int row = wq * 32 + lane;
     const int i = m0 + row;
@@ -466,22 +485,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int n0 = (jt0 + j) * kBK;
       const bool full = (n0 >= lo_last) && (n0 + kBK - 1 <= hi_first) && (n0 + kBK <= g.n);
+      uint32_t r[128];                         // r[0..63] S, r[64..127] dP: one read
+      tmem_ld128(tS, r);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        uint32_t r[64];                        // r[0..31] S, r[32..63] dP
-        tmem_ld32x2(tS + ch * 32, tS + 64 + ch * 32, r);
         uint32_t dd[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           float ds[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            float pv = ex2_approx(fmaf(__uint_as_float(r[x + u]), prm.scale_log2, -lse2));
+            const int c = ch * 32 + x + u;
+            float pv = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lse2));
             if (!full) {
-              const int jj = n0 + ch * 32 + x + u;
+              const int jj = n0 + c;
               if (jj < lo_i || jj > hi_i) pv = 0.f;
             }
-            ds[u] = pv * (__uint_as_float(r[32 + x + u]) - Di);
+            ds[u] = pv * (__uint_as_float(r[64 + c]) - Di);
           }
           dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
