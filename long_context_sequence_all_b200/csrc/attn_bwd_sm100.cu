@@ -17,9 +17,10 @@
 //       dV  += P^T dO, dK  += dS^T Q           (M=128 keys, N=128,      K=64)
 //     P^T and dS^T go through shared memory (bf16, swizzled); dK and dV stay
 //     in TMEM until the end.
-//  3. dQ kernel, query-stationary (like the forward: two query heads of one
-//     group at the same positions share K/V tiles of 64 keys):
+//  3. dQ kernel, query-stationary: a CTA owns 128 query rows of one head
+//     with Q and dO resident in TMEM, and streams K/V tiles of 64 keys:
 //       S = Q K^T, dP = dO V^T (M=128, N=64, K=128);  dQ += dS K (N=128, K=64)
+//     all with the A operand in TMEM (only K and V cross shared memory).
 //
 // TMA loads with 128-byte swizzle feed shared memory; one thread issues all
 // MMAs; every wait is bounded (ULY_ERR_TIMEOUT).
@@ -51,6 +52,8 @@ constexpr uint32_t kIdescN64 = idesc_bf16_f32(128, 64, false, false);    // K-ma
 constexpr uint32_t kIdescN128MN = idesc_bf16_f32(128, 128, false, true); // B MN-major, N = 128
 
 struct BwdParams {
+  const __nv_bfloat16 *q;     // [qheads][n][d] (dQ kernel: Q rows go into TMEM)
+  const __nv_bfloat16 *dout;  // [qheads][n][d]
   const float *lse;   // [qheads][n]
   const float *Dv;    // [qheads][n]
   __nv_bfloat16 *out0;  // dkdv: dV, dq: dQ
@@ -315,43 +318,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ================================================================== dQ
+// One CTA = one 128-row query tile of one query head.  Q and dO sit in TMEM
+// as the A operands of S = Q K^T and dP = dO V^T; S/dP are double-buffered
+// across 64-key tiles and the two compute warpgroups take alternate tiles;
+// dS goes back into the S columns of TMEM and dQ += dS K is also issued from
+// TMEM, so shared memory only carries K and V (six-stage ring).
 namespace qk {
-constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
+constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBK = 64;    // keys per K/V tile
-constexpr int kStages = 2;
-constexpr uint32_t kQBytes = 128 * 128 * 2;
-constexpr uint32_t kKBytes = 64 * 128 * 2;
-constexpr uint32_t kOffQ = 0;                      // Q_0, Q_1
-constexpr uint32_t kOffO = 2 * kQBytes;            // dO_0, dO_1
-constexpr uint32_t kOffKV = 4 * kQBytes;           // stage s: K at +s*2*kKBytes, V after it
-constexpr uint32_t kOffDS = kOffKV + kStages * 2 * kKBytes;   // dS_0, dS_1 (128 x 64 bf16)
-constexpr uint32_t kOffBar = kOffDS + 2 * (128 * 64 * 2);
-constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
+constexpr int kStages = 6;
+constexpr uint32_t kKBytes = 64 * 128 * 2;                 // one K or V tile
+constexpr uint32_t kOffBar = kStages * 2 * kKBytes;        // stage s: K at s*2*kKBytes, V after it
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+// TMEM columns: Q, dO (bf16 pairs), dQ (fp32), then S_b, dP_b for b = 0, 1
+constexpr uint32_t kTQ = 0, kTO = 64, kTdQ = 128, kTS = 256;
 }  // namespace qk
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                         const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    attn_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const BwdParams prm) {
   using namespace qk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  enum { B_Q = 0, B_KF = 1, B_KE = 1 + kStages, B_S = 1 + 2 * kStages, B_P = B_S + 2, B_DQ = B_P + 2,
-         B_DRAIN = B_DQ + 2, B_N = B_DRAIN + 1 };
+  enum { B_KF = 0, B_KE = kStages, B_S = 2 * kStages, B_P = B_S + 2, B_QO = B_P + 2, B_DQ = B_QO + 1,
+         B_DRAIN = B_DQ + 1, B_N = B_DRAIN + 1 };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = g.hl >> 1;
-  const int pair = blockIdx.x;
-  const int rb = pair / half, pp = pair - rb * half;
-  const int qhead0 = rb * g.hl + 2 * pp;
-  const int kvhead = rb * g.gl + (2 * pp) / g.group;
-  const int mt = gridDim.y - 1 - blockIdx.y;
+  const int qh = blockIdx.x;                     // (r*B + b)*hl + hh
+  const int rb = qh / g.hl, hh = qh - rb * g.hl;
+  const int kvhead = rb * g.gl + hh / g.group;
+  const int mt = gridDim.y - 1 - blockIdx.y;     // heaviest (latest) query tiles first
   const int m0 = mt * kBM;
 
   int lo_first, hi_first, lo_last, hi_last;
@@ -361,11 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NT = (hi_last >= lo_first) ? hi_last / kBK - jt0 + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
+    for (int i = 0; i < B_N; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_P || i == B_P + 1) cnt = 128;
+      if (i == B_QO) cnt = 256;
+      mbar_init(bar(i), cnt);
+    }
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmO);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
@@ -377,167 +382,159 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns, tile t: S [256t, +64), dP [256t+64, +64), dQ [256t+128, +128)
   // Registers: producer / MMA warpgroup 120 per thread, the two compute
   // warpgroups 192 (a thread holds its whole 128-column S | dP row).
 
   if (warp < 4) {
-  setmaxnreg_dec<kRegsCtlQ>();
-  if (warp == 0) {
-    if (lane == 0 && NT > 0) {
-      mbar_arrive_expect_tx(bar(B_Q), 4 * kQBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < 2; ++c) {
-          tma_load_3d(sb + kOffQ + t * kQBytes + c * 16384, &tmQ, bar(B_Q), c * 64, m0, qhead0 + t);
-          tma_load_3d(sb + kOffO + t * kQBytes + c * 16384, &tmO, bar(B_Q), c * 64, m0, qhead0 + t);
-        }
-      int issued = 0;
-      for (int j = 0; j < NT; ++j) {
-        const int s = j % kStages, use = j / kStages;
-        if (use > 0 && !mbar_wait(bar(B_KE + s), (use - 1) & 1, abort_flag, prm.err)) break;
-        const uint32_t st = sb + kOffKV + s * 2 * kKBytes;
-        const int row0 = (jt0 + j) * kBK;
-        mbar_arrive_expect_tx(bar(B_KF + s), 2 * kKBytes);
-        for (int c = 0; c < 2; ++c) {
-          tma_load_3d(st + c * 8192, &tmK, bar(B_KF + s), c * 64, row0, kvhead);
-          tma_load_3d(st + kKBytes + c * 8192, &tmV, bar(B_KF + s), c * 64, row0, kvhead);
-        }
-        issued = j + 1;
-      }
-      if (*abort_flag)
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_wait(bar(B_KF + j % kStages), (j / kStages) & 1, nullptr, prm.err);
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && NT > 0) {
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err);
-      tc_fence_after();
-      const uint64_t dQ0 = sdesc_sw128(sb + kOffQ, 16, 1024), dQ1 = sdesc_sw128(sb + kOffQ + kQBytes, 16, 1024);
-      const uint64_t dO0 = sdesc_sw128(sb + kOffO, 16, 1024), dO1 = sdesc_sw128(sb + kOffO + kQBytes, 16, 1024);
-      const uint64_t dS0 = sdesc_sw128(sb + kOffDS, 16, 1024), dS1 = sdesc_sw128(sb + kOffDS + 16384, 16, 1024);
-      auto issue_dq = [&](int t, int j) {
-        // dQ_t += dS_t K_j   (A = dS K-major, B = K tile MN-major over d)
-        const uint64_t dKm = sdesc_sw128(sb + kOffKV + (j % kStages) * 2 * kKBytes, 8192, 1024);
-        const uint64_t dS = t ? dS1 : dS0;
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_bf16_ss(tmem + 256 * t + 128, sdesc_add(dS, kk * 32), sdesc_add(dKm, kk * 2048), kIdescN128MN,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      for (int j = 0; ok && j < NT; ++j) {
-        const int s = j % kStages;
-        ok = mbar_wait(bar(B_KF + s), (j / kStages) & 1, abort_flag, prm.err);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kst = sb + kOffKV + s * 2 * kKBytes;
-        const uint64_t dK = sdesc_sw128(kst, 16, 1024), dV = sdesc_sw128(kst + kKBytes, 16, 1024);
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j > 0) {
-            ok = mbar_wait(bar(B_P + t), (j - 1) & 1, abort_flag, prm.err);
-            if (!ok) break;
-            tc_fence_after();
-            issue_dq(t, j - 1);
+    setmaxnreg_dec<kRegsCtlQ>();
+    if (warp == 0) {
+      if (lane == 0 && NT > 0) {
+        int issued = 0;
+        for (int j = 0; j < NT; ++j) {
+          const int s = j % kStages, use = j / kStages;
+          if (use > 0 && !mbar_wait(bar(B_KE + s), (use - 1) & 1, abort_flag, prm.err)) break;
+          const uint32_t st = sb + s * 2 * kKBytes;
+          const int row0 = (jt0 + j) * kBK;
+          mbar_arrive_expect_tx(bar(B_KF + s), 2 * kKBytes);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(st + c * 8192, &tmK, bar(B_KF + s), c * 64, row0, kvhead);
+            tma_load_3d(st + kKBytes + c * 8192, &tmV, bar(B_KF + s), c * 64, row0, kvhead);
           }
-          const uint64_t dQ = t ? dQ1 : dQ0, dO = t ? dO1 : dO0;
+          issued = j + 1;
+        }
+        if (*abort_flag)
+          for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+            mbar_wait(bar(B_KF + j % kStages), (j / kStages) & 1, nullptr, prm.err);
+      }
+    } else if (warp == 1) {
+      if (lane == 0 && NT > 0) {
+        bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err);
+        tc_fence_after();
+        // S_b = Q K_j^T and dP_b = dO V_j^T, A operands from TMEM
+        auto issue_sdp = [&](int j) -> bool {
+          const int b = j & 1, s = j % kStages;
+          if (!mbar_wait(bar(B_KF + s), (j / kStages) & 1, abort_flag, prm.err)) return false;
+          tc_fence_after();
+          const uint32_t kst = sb + s * 2 * kKBytes;
+          const uint64_t dK = sdesc_sw128(kst, 16, 1024), dV = sdesc_sw128(kst + kKBytes, 16, 1024);
+          const uint32_t tS = tmem + kTS + 128 * b;
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
-            const uint32_t qo = (kk >> 2) * 16384 + (kk & 3) * 32, ko = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + 256 * t, sdesc_add(dQ, qo), sdesc_add(dK, ko), kIdescN64, kk > 0);
-            mma_bf16_ss(tmem + 256 * t + 64, sdesc_add(dO, qo), sdesc_add(dV, ko), kIdescN64, kk > 0);
+            const uint32_t ko = (kk >> 2) * 8192 + (kk & 3) * 32;
+            mma_bf16_ts(tS, tmem + kTQ + kk * 8, sdesc_add(dK, ko), kIdescN64, kk > 0);
+            mma_bf16_ts(tS + 64, tmem + kTO + kk * 8, sdesc_add(dV, ko), kIdescN64, kk > 0);
           }
-          tc_commit(bar(B_S + t));
+          tc_commit(bar(B_S + b));
+          return true;
+        };
+        if (ok) ok = issue_sdp(0);
+        if (ok && NT > 1) ok = issue_sdp(1);
+        for (int j = 0; ok && j < NT; ++j) {
+          const int b = j & 1, s = j % kStages;
+          ok = mbar_wait(bar(B_P + b), (j >> 1) & 1, abort_flag, prm.err);
+          if (!ok) break;
+          tc_fence_after();
+          // dQ += dS_b K_j: A = dS (bf16 pairs in the S_b columns), B = K tile MN-major over d
+          const uint64_t dKm = sdesc_sw128(sb + s * 2 * kKBytes, 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16_ts(tmem + kTdQ, tmem + kTS + 128 * b + kk * 8, sdesc_add(dKm, kk * 2048), kIdescN128MN,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(B_KE + s));
+          if (j + 2 < NT) ok = issue_sdp(j + 2);
         }
-        if (!ok) break;
-        if (j > 0) tc_commit(bar(B_KE + (j - 1) % kStages));
-      }
-      for (int t = 0; t < 2 && ok; ++t) {
-        ok = mbar_wait(bar(B_P + t), (NT - 1) & 1, abort_flag, prm.err);
-        if (!ok) break;
-        tc_fence_after();
-        issue_dq(t, NT - 1);
-        tc_commit(bar(B_DQ + t));
-      }
-      if (ok) tc_commit(bar(B_KE + (NT - 1) % kStages));
-      if (!ok) {
-        tc_commit(bar(B_DRAIN));
-        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
+        if (ok) tc_commit(bar(B_DQ));
+        if (!ok) {
+          tc_commit(bar(B_DRAIN));
+          mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
+        }
       }
     }
-  }
   } else {
     setmaxnreg_inc<kRegsComputeQ>();
-    const int t = (warp - 4) >> 2, wq = warp & 3;
+    const int b = (warp - 4) >> 2, wq = warp & 3;   // b: even / odd key tiles
     const int row = wq * 32 + lane;
     const int i = m0 + row;
     const bool valid = i < g.n;
     int lo_i = 1, hi_i = 0;
     if (valid) prm.mk.row_range(i, lo_i, hi_i);
-    const long long qrow = (long long)(qhead0 + t) * g.n + i;
+    const long long qrow = (long long)qh * g.n + i;
     const float lse2 = valid ? prm.lse[qrow] * kLog2e : INFINITY;
     const float Di = valid ? prm.Dv[qrow] : 0.f;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + 256 * t;
-    const uint32_t ds_base = sb + kOffDS + t * 16384;
+    // warpgroup 0 puts this row of Q into TMEM, warpgroup 1 the row of dO
+    {
+      const __nv_bfloat16 *src = (b == 0) ? prm.q : prm.dout;
+      uint32_t v[64];
+      const uint4 *p4 = reinterpret_cast<const uint4 *>(src + (valid ? qrow : 0) * kHD);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const uint4 w4 = valid ? __ldg(p4 + u) : make_uint4(0, 0, 0, 0);
+        v[4 * u] = w4.x;
+        v[4 * u + 1] = w4.y;
+        v[4 * u + 2] = w4.z;
+        v[4 * u + 3] = w4.w;
+      }
+      tmem_st64_nowait(tmem + lane_off + (b == 0 ? kTQ : kTO), v);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_QO));
+    }
+    const uint32_t tS = tmem + lane_off + kTS + 128 * b;
     bool ok = true;
-    for (int j = 0; j < NT; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + t), j & 1, abort_flag, prm.err));
+    for (int j = b; j < NT; j += 2) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + b), (j >> 1) & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
       const int n0 = (jt0 + j) * kBK;
       const bool full = (n0 >= lo_last) && (n0 + kBK - 1 <= hi_first) && (n0 + kBK <= g.n);
       uint32_t r[128];                         // r[0..63] S, r[64..127] dP: one read
       tmem_ld128(tS, r);
+      uint32_t dd[32];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t dd[16];
+      for (int c = 0; c < 64; c += 2) {
+        float ds[2];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = ch * 32 + x + u;
-            float pv = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lse2));
-            if (!full) {
-              const int jj = n0 + c;
-              if (jj < lo_i || jj > hi_i) pv = 0.f;
-            }
-            ds[u] = pv * (__uint_as_float(r[64 + c]) - Di);
+        for (int u = 0; u < 2; ++u) {
+          float pv = ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lse2));
+          if (!full) {
+            const int jj = n0 + c + u;
+            if (jj < lo_i || jj > hi_i) pv = 0.f;
           }
-          dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
+          ds[u] = pv * (__uint_as_float(r[64 + c + u]) - Di);
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          st_shared_v4(ds_base + sw128_row64(row, ch * 4 + u), dd[4 * u], dd[4 * u + 1], dd[4 * u + 2],
-                       dd[4 * u + 3]);
+        dd[c >> 1] = pack_bf16x2(ds[0], ds[1]);
       }
-      fence_proxy_async_smem();
+      tmem_st32_nowait(tS, dd);                // dS (bf16 pairs) into S columns [0, 32)
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(B_P + t));
+      mbar_arrive(bar(B_P + b));
     }
-    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ + t), 0, abort_flag, prm.err));
+    // epilogue: warpgroup b writes dQ columns [64b, 64b + 64)
+    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, abort_flag, prm.err));
     tc_fence_after();
     if (ok && NT > 0) {
       uint32_t r[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tS + 128 + c * 32, r);
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(tmem + lane_off + kTdQ + 64 * b + 32 * c, r);
         if (valid) {
-          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + c * 32);
+          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * b + 32 * c);
+          const float sc = g.scale;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            uint4 v;
-            const float sc = g.scale;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
-            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
-            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
-            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
-            dptr[u] = v;
+            uint4 w4;
+            w4.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
+            w4.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
+            w4.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
+            w4.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
+            dptr[u] = w4;
           }
         }
       }
     } else if (NT == 0 && valid) {
-      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD);
-      for (int u = 0; u < kHD / 8; ++u) dptr[u] = make_uint4(0, 0, 0, 0);
+      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * b);
+      for (int u = 0; u < 8; ++u) dptr[u] = make_uint4(0, 0, 0, 0);
     }
   }
 
@@ -559,13 +556,11 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   const int qheads = g.P * g.B * g.hl, kvheads = g.P * g.B * g.gl;
   uly_status st = attn_bwd_dot_launch(ULY_BF16, d->head_dim, o, dout, Dv, (long long)qheads * g.n, stream);
   if (st != ULY_OK) return st;
-  CUtensorMap mK128, mV128, mQ64, mO64, mQ128, mO128, mK64, mV64;
+  CUtensorMap mK128, mV128, mQ64, mO64, mK64, mV64;
   if (!make_tmap_heads_bf16(&mK128, k, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&mV128, v, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&mQ64, q, kHD, g.n, qheads, 64) ||
       !make_tmap_heads_bf16(&mO64, dout, kHD, g.n, qheads, 64) ||
-      !make_tmap_heads_bf16(&mQ128, q, kHD, g.n, qheads, 128) ||
-      !make_tmap_heads_bf16(&mO128, dout, kHD, g.n, qheads, 128) ||
       !make_tmap_heads_bf16(&mK64, k, kHD, g.n, kvheads, 64) ||
       !make_tmap_heads_bf16(&mV64, v, kHD, g.n, kvheads, 64))
     return ULY_ERR_CUDA;
@@ -579,6 +574,8 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
     attr_set = true;
   }
   BwdParams prm;
+  prm.q = static_cast<const __nv_bfloat16 *>(q);
+  prm.dout = static_cast<const __nv_bfloat16 *>(dout);
   prm.lse = lse;
   prm.Dv = Dv;
   prm.g = g;
@@ -594,10 +591,10 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   }
   prm.out0 = static_cast<__nv_bfloat16 *>(dq);
   prm.out1 = nullptr;
-  dim3 gq(qheads / 2, (g.n + qk::kBM - 1) / qk::kBM);
+  dim3 gq(qheads, (g.n + qk::kBM - 1) / qk::kBM);
   {
     prof::Scope scope(prof::K_ATTN_DQ_SM100, stream);
-    attn_dq_sm100_kernel<<<gq, kThreads, qk::kSmemBytes, stream>>>(mQ128, mO128, mK64, mV64, prm);
+    attn_dq_sm100_kernel<<<gq, kThreads, qk::kSmemBytes, stream>>>(mK64, mV64, prm);
   }
   note_launches(2);
   return last_launch_status();
