@@ -10,13 +10,12 @@
 // Three launches, all deterministic (no atomics):
 //  1. D_i = <dO_i, O_i>   (one warp per row, HBM-bound)
 //  2. dK/dV kernel, KV-stationary: a CTA owns 128 keys of one KV head and
-//     visits every 64-row query tile (of every query head of the group) that
-//     sees them.  Two compute warpgroups take alternate query tiles (ping-
-//     pong) so one group's exp/dS work overlaps the other group's MMAs:
-//       S^T  = K Q^T,  dP^T = V dO^T          (M=128 keys, N=64 queries, K=128)
-//       dV  += P^T dO, dK  += dS^T Q           (M=128 keys, N=128,      K=64)
-//     P^T and dS^T go through shared memory (bf16, swizzled); dK and dV stay
-//     in TMEM until the end.
+//     visits every 128-row query tile (of every query head of the group) that
+//     sees them; the two compute warpgroups split each tile's query columns:
+//       S^T  = K Q^T,  dP^T = V dO^T          (M=128 keys, N=128 queries, K=128)
+//       dV  += P^T dO, dK  += dS^T Q           (M=128 keys, N=128,      K=128)
+//     P^T and dS^T stay in TMEM (A operand of dV / dK); dK and dV stay in
+//     TMEM until the end.
 //  3. dQ kernel, query-stationary: a CTA owns 128 query rows of one head
 //     with Q and dO resident in TMEM, and streams K/V tiles of 64 keys:
 //       S = Q K^T, dP = dO V^T (M=128, N=64, K=128);  dQ += dS K (N=128, K=64)
@@ -49,6 +48,7 @@ static_assert(128 * kRegsCtlKV + 256 * kRegsComputeKV == kThreads * kRegsLaunch 
               "register split must use exactly the launch pool");
 
 constexpr uint32_t kIdescN64 = idesc_bf16_f32(128, 64, false, false);    // K-major A and B, N = 64
+constexpr uint32_t kIdescN128 = idesc_bf16_f32(128, 128, false, false);  // K-major A and B, N = 128
 constexpr uint32_t kIdescN128MN = idesc_bf16_f32(128, 128, false, true); // B MN-major, N = 128
 
 struct BwdParams {
@@ -71,18 +71,26 @@ __device__ __forceinline__ uint32_t sw128_row64(int row, int chunk) {
 }
 
 // ============================================================== dK / dV
+// One CTA = 128 keys of one KV head; it visits every 128-row query tile (of
+// every query head of the group) that sees them, one tile at a time:
+//   S^T  = K Q^T,  dP^T = V dO^T   (M=128 keys, N=128 queries, K=128; A and B from smem)
+//   dV  += P^T dO, dK  += dS^T Q    (M=128, N=128, K=128 queries; A from TMEM)
+// The two compute warpgroups split the 128 query columns of a tile (64
+// each); each writes its half of P^T and dS^T (bf16 pairs) over TMEM columns
+// of S^T / dP^T that it has itself already read, so the halves never race.
+// All MMAs are N=128 (N=64 instructions run at two thirds of the rate).
 namespace kv {
 constexpr int kBN = 128;   // keys per CTA
-constexpr int kBQ = 64;    // query rows per tile
-constexpr int kStages = 3;
-constexpr uint32_t kKVBytes = 128 * 128 * 2;       // K or V tile
-constexpr uint32_t kQBytes = 64 * 128 * 2;         // Q or dO tile
-constexpr uint32_t kOffK = 0, kOffV = kKVBytes;
-constexpr uint32_t kOffStage = 2 * kKVBytes;       // stage s: Q at +s*2*kQBytes, dO after it
-constexpr uint32_t kOffPT = kOffStage + kStages * 2 * kQBytes;   // per WG: P^T then dS^T (16 KB each)
-constexpr uint32_t kOffLD = kOffPT + 2 * 2 * (128 * 64 * 2);     // per WG: 64 lse2 + 64 D floats
+constexpr int kBQ = 128;   // query rows per tile
+constexpr int kStages = 2;
+constexpr uint32_t kTile = 128 * 128 * 2;          // one 128 x 128 bf16 tile
+constexpr uint32_t kOffK = 0, kOffV = kTile;
+constexpr uint32_t kOffStage = 2 * kTile;          // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
+constexpr uint32_t kOffLD = kOffStage + kStages * 2 * kTile;   // per WG: 64 lse*log2e + 64 D
 constexpr uint32_t kOffBar = kOffLD + 2 * 512;
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
+// TMEM columns: dV, dK, S^T, dP^T
+constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTP = 384;
 }  // namespace kv
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -94,7 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  enum { B_KV = 0, B_SF_ = 1, B_SE = 1 + kStages, B_S = 1 + 2 * kStages, B_P = B_S + 2, B_DONE = B_P + 2,
+  enum { B_KV = 0, B_SF_ = 1, B_SE = 1 + kStages, B_S = 1 + 2 * kStages, B_P = B_S + 1, B_DONE = B_P + 1,
          B_DRAIN = B_DONE + 1, B_N = B_DRAIN + 1 };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
@@ -116,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = nqt * g.group;                   // tiles: head-major
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P) ? 256 : 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmK);
@@ -132,15 +140,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: dV [0,128) dK [128,256); WG w: S^T [256+128w, +64), dP^T [+64, +64)
   // Registers: producer / MMA warpgroup 136 per thread, the two compute
-  // warpgroups 184 (a thread holds its whole 128-column S^T | dP^T row).
+  // warpgroups 184 (a thread holds 64 columns of S^T and 64 of dP^T).
 
   if (warp < 4) {
   setmaxnreg_dec<kRegsCtlKV>();
   if (warp == 0) {
     if (lane == 0 && T > 0) {
-      mbar_arrive_expect_tx(bar(B_KV), 2 * kKVBytes);
+      mbar_arrive_expect_tx(bar(B_KV), 2 * kTile);
       for (int c = 0; c < 2; ++c) {
         tma_load_3d(sb + kOffK + c * 16384, &tmK, bar(B_KV), c * 64, n0, kvh);
         tma_load_3d(sb + kOffV + c * 16384, &tmV, bar(B_KV), c * 64, n0, kvh);
@@ -150,11 +157,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = t % kStages, use = t / kStages;
         if (use > 0 && !mbar_wait(bar(B_SE + s), (use - 1) & 1, abort_flag, prm.err)) break;
         const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
-        const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
-        mbar_arrive_expect_tx(bar(B_SF_ + s), 2 * kQBytes);
+        const uint32_t st = sb + kOffStage + s * 2 * kTile;
+        mbar_arrive_expect_tx(bar(B_SF_ + s), 2 * kTile);
         for (int c = 0; c < 2; ++c) {
-          tma_load_3d(st + c * 8192, &tmQ, bar(B_SF_ + s), c * 64, i0, qh_base + e);
-          tma_load_3d(st + kQBytes + c * 8192, &tmO, bar(B_SF_ + s), c * 64, i0, qh_base + e);
+          tma_load_3d(st + c * 16384, &tmQ, bar(B_SF_ + s), c * 64, i0, qh_base + e);
+          tma_load_3d(st + kTile + c * 16384, &tmO, bar(B_SF_ + s), c * 64, i0, qh_base + e);
         }
         issued = t + 1;
       }
@@ -167,41 +174,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
       tc_fence_after();
       const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
+      // S^T = K Q_t^T, dP^T = V dO_t^T (N = 128 query rows)
       auto issue_sdp = [&](int t) -> bool {
-        const int w = t & 1, s = t % kStages;
+        const int s = t % kStages;
         if (!mbar_wait(bar(B_SF_ + s), (t / kStages) & 1, abort_flag, prm.err)) return false;
         tc_fence_after();
-        const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
-        const uint64_t dQ = sdesc_sw128(st, 16, 1024), dO = sdesc_sw128(st + kQBytes, 16, 1024);
-        const uint32_t tS = tmem + 256 + 128 * w;
+        const uint32_t st = sb + kOffStage + s * 2 * kTile;
+        const uint64_t dQ = sdesc_sw128(st, 16, 1024), dO = sdesc_sw128(st + kTile, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32, qo = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_bf16_ss(tS, sdesc_add(dK, ko), sdesc_add(dQ, qo), kIdescN64, kk > 0);
-          mma_bf16_ss(tS + 64, sdesc_add(dV, ko), sdesc_add(dO, qo), kIdescN64, kk > 0);
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + kTS, sdesc_add(dK, ko), sdesc_add(dQ, ko), kIdescN128, kk > 0);
+          mma_bf16_ss(tmem + kTP, sdesc_add(dV, ko), sdesc_add(dO, ko), kIdescN128, kk > 0);
         }
-        tc_commit(bar(B_S + w));
+        tc_commit(bar(B_S));
         return true;
       };
       if (ok) ok = issue_sdp(0);
-      if (ok && T > 1) ok = issue_sdp(1);
       for (int t = 0; ok && t < T; ++t) {
-        const int w = t & 1, s = t % kStages;
-        ok = mbar_wait(bar(B_P + w), (t >> 1) & 1, abort_flag, prm.err);
+        const int s = t % kStages;
+        ok = mbar_wait(bar(B_P), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t st = sb + kOffStage + s * 2 * kQBytes;
-        const uint32_t pt = sb + kOffPT + w * 32768, dst = pt + 16384;
-        const uint64_t dPt = sdesc_sw128(pt, 16, 1024), dSt = sdesc_sw128(dst, 16, 1024);
-        const uint64_t dOm = sdesc_sw128(st + kQBytes, 8192, 1024), dQm = sdesc_sw128(st, 8192, 1024);
+        // dV += P^T dO_t, dK += dS^T Q_t: A from TMEM (query columns [0,64) in
+        // the S^T / dP^T columns [0,32), [64,128) in columns [64,96)), B = dO /
+        // Q tile, MN-major over d
+        const uint32_t st = sb + kOffStage + s * 2 * kTile;
+        const uint64_t dQm = sdesc_sw128(st, 16384, 1024), dOm = sdesc_sw128(st + kTile, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk) {
+          const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ss(tmem + 0, sdesc_add(dPt, kk * 32), sdesc_add(dOm, kk * 2048), kIdescN128MN, acc);
-          mma_bf16_ss(tmem + 128, sdesc_add(dSt, kk * 32), sdesc_add(dQm, kk * 2048), kIdescN128MN, acc);
+          mma_bf16_ts(tmem + kTdV, tmem + kTS + acol, sdesc_add(dOm, kk * 2048), kIdescN128MN, acc);
+          mma_bf16_ts(tmem + kTdK, tmem + kTP + acol, sdesc_add(dQm, kk * 2048), kIdescN128MN, acc);
         }
         tc_commit(bar(B_SE + s));
-        if (t + 2 < T) ok = issue_sdp(t + 2);
+        if (t + 1 < T) ok = issue_sdp(t + 1);
       }
       if (ok) tc_commit(bar(B_DONE));
       if (!ok) {
@@ -212,92 +220,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     setmaxnreg_inc<kRegsComputeKV>();
-    const int w = (warp - 4) >> 2, wq = warp & 3;
-    const int row = wq * 32 + lane;            // key row within the tile
+    const int w = (warp - 4) >> 2, wq = warp & 3;  // w: query columns [64w, 64w + 64)
+    const int row = wq * 32 + lane;                // key row within the tile
     const int j = n0 + row;
-    const int tid = threadIdx.x - 128 * (w + 1);  // 0..127 within the warpgroup
+    const int tid = threadIdx.x - 128 * (w + 1);   // 0..127 within the warpgroup
     int lo_j = 1, hi_j = 0;
     if (j < g.n) prm.mk.col_range(j, lo_j, hi_j);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + 256 + 128 * w;
-    const uint32_t pt = sb + kOffPT + w * 32768, dst = pt + 16384;
+    const uint32_t tS = tmem + lane_off + kTS + 64 * w, tP = tmem + lane_off + kTP + 64 * w;
     float *lsm = reinterpret_cast<float *>(smem + kOffLD + w * 512);  // [0,64) lse*log2e, [64,128) D
     // this thread's share of the per-tile statistics: LSE (tid < 64) or D of
-    // query row i0 + (tid & 63); fetched one tile ahead of its use
+    // query row i0 + 64w + (tid & 63); fetched one tile ahead of its use
     auto fetch_stat = [&](int t) -> float {
       if (t >= T) return 0.f;
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
-      const int i = i0 + (tid & 63);
+      const int i = i0 + 64 * w + (tid & 63);
       const long long idx = (long long)(qh_base + e) * g.n + i;
       if (tid < 64) return (i < g.n) ? __ldg(prm.lse + idx) * kLog2e : INFINITY;
       return (i < g.n) ? __ldg(prm.Dv + idx) : 0.f;
     };
-    float stat_next = fetch_stat(w);
+    float stat_next = fetch_stat(0);
     bool ok = true;
-    for (int t = w; t < T; t += 2) {
-      const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
+    for (int t = 0; t < T; ++t) {
+      const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ + 64 * w;  // this warpgroup's first query row
       named_bar_sync(1 + w, 128);              // previous tile's LSE/D reads are done
       lsm[tid] = stat_next;
       named_bar_sync(1 + w, 128);
-      stat_next = fetch_stat(t + 2);           // in flight while this tile is processed
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + w), (t >> 1) & 1, abort_flag, prm.err));
+      stat_next = fetch_stat(t + 1);           // in flight while this tile is processed
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S), t & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
-      const bool full = (i0 >= n0 + kBN - 1) && (i0 + kBQ - 1 <= hi_a) && (i0 + kBQ <= g.n) &&
-                        (n0 + kBN <= g.n);
-      uint32_t r[128];                         // r[0..63] S^T, r[64..127] dP^T: one read
-      tmem_ld128(tS, r);
+      const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
+      uint32_t r[128];                         // r[0..63] S^T, r[64..127] dP^T of this warpgroup's columns
+      tmem_ld64x2(tS, tP, r);
+      uint32_t pp[32], dd[32];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t pp[16], dd[16];
+      for (int c = 0; c < 64; c += 2) {
+        float p[2], ds[2];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float p[2], ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = ch * 32 + x + u;
-            float pv = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lsm[c]));
-            if (!full) {
-              const int i = i0 + c;
-              if (i < lo_j || i > hi_j) pv = 0.f;
-            }
-            p[u] = pv;
-            ds[u] = pv * (__uint_as_float(r[64 + c]) - lsm[64 + c]);
+        for (int u = 0; u < 2; ++u) {
+          float pv = ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lsm[c + u]));
+          if (!full) {
+            const int i = i0 + c + u;
+            if (i < lo_j || i > hi_j) pv = 0.f;
           }
-          pp[x >> 1] = pack_bf16x2(p[0], p[1]);
-          dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
+          p[u] = pv;
+          ds[u] = pv * (__uint_as_float(r[64 + c + u]) - lsm[64 + c + u]);
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t off = sw128_row64(row, ch * 4 + u);
-          st_shared_v4(pt + off, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-          st_shared_v4(dst + off, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-        }
+        pp[c >> 1] = pack_bf16x2(p[0], p[1]);
+        dd[c >> 1] = pack_bf16x2(ds[0], ds[1]);
       }
-      fence_proxy_async_smem();
+      // P^T and dS^T (bf16 pairs) over this warpgroup's first 32 columns of S^T / dP^T
+      tmem_st32_nowait(tS, pp);
+      tmem_st32_nowait(tP, dd);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(B_P + w));
+      mbar_arrive(bar(B_P));
     }
-    // epilogue: WG0 writes dV, WG1 writes dK (scaled)
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (scaled)
     if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err));
     tc_fence_after();
     __nv_bfloat16 *outp = (w == 0) ? prm.out0 : prm.out1;
     const float mul = (w == 0) ? 1.f : g.scale;
     const long long orow = (long long)kvh * g.n + j;
     if (ok && T > 0) {
-      uint32_t r[32];
+      uint32_t rr[32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_off + 128 * w + c * 32, r);
+        tmem_ld32(tmem + lane_off + (w == 0 ? kTdV : kTdK) + c * 32, rr);
         if (j < g.n) {
           uint4 *dptr = reinterpret_cast<uint4 *>(outp + orow * kHD + c * 32);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * mul, __uint_as_float(r[8 * u + 1]) * mul);
-            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * mul, __uint_as_float(r[8 * u + 3]) * mul);
-            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * mul, __uint_as_float(r[8 * u + 5]) * mul);
-            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * mul, __uint_as_float(r[8 * u + 7]) * mul);
+            v.x = pack_bf16x2(__uint_as_float(rr[8 * u + 0]) * mul, __uint_as_float(rr[8 * u + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(rr[8 * u + 2]) * mul, __uint_as_float(rr[8 * u + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(rr[8 * u + 4]) * mul, __uint_as_float(rr[8 * u + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(rr[8 * u + 6]) * mul, __uint_as_float(rr[8 * u + 7]) * mul);
             dptr[u] = v;
           }
         }
@@ -556,11 +555,11 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   const int qheads = g.P * g.B * g.hl, kvheads = g.P * g.B * g.gl;
   uly_status st = attn_bwd_dot_launch(ULY_BF16, d->head_dim, o, dout, Dv, (long long)qheads * g.n, stream);
   if (st != ULY_OK) return st;
-  CUtensorMap mK128, mV128, mQ64, mO64, mK64, mV64;
+  CUtensorMap mK128, mV128, mQ128, mO128, mK64, mV64;
   if (!make_tmap_heads_bf16(&mK128, k, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&mV128, v, kHD, g.n, kvheads, 128) ||
-      !make_tmap_heads_bf16(&mQ64, q, kHD, g.n, qheads, 64) ||
-      !make_tmap_heads_bf16(&mO64, dout, kHD, g.n, qheads, 64) ||
+      !make_tmap_heads_bf16(&mQ128, q, kHD, g.n, qheads, 128) ||
+      !make_tmap_heads_bf16(&mO128, dout, kHD, g.n, qheads, 128) ||
       !make_tmap_heads_bf16(&mK64, k, kHD, g.n, kvheads, 64) ||
       !make_tmap_heads_bf16(&mV64, v, kHD, g.n, kvheads, 64))
     return ULY_ERR_CUDA;
@@ -587,7 +586,7 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   dim3 gkv(kvheads, (g.n + kv::kBN - 1) / kv::kBN);
   {
     prof::Scope scope(prof::K_ATTN_DKDV_SM100, stream);
-    attn_dkdv_sm100_kernel<<<gkv, kThreads, kv::kSmemBytes, stream>>>(mK128, mV128, mQ64, mO64, prm);
+    attn_dkdv_sm100_kernel<<<gkv, kThreads, kv::kSmemBytes, stream>>>(mK128, mV128, mQ128, mO128, prm);
   }
   prm.out0 = static_cast<__nv_bfloat16 *>(dq);
   prm.out1 = nullptr;
