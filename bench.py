@@ -251,7 +251,7 @@ def run_ours(args, rank, world, dev):
     build.build()
     U.lib()
     w = WORKLOADS[args.workload]
-    inp = make_inputs(w, seed=1000 + w.index + 7919 * rank)
+    inp = make_inputs(w, seed=rank_seed(w, rank))
     work, pairs = algorithmic_work(inp)
     layer = Layer(inp, dev)
     U.ulysses_read_error()
@@ -300,7 +300,7 @@ def run_ours(args, rank, world, dev):
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
 
     tokens = inp["B"] * inp["n"]
-    value = world * tokens / (ms_max / 1e3)
+    value = job_throughput(tokens, world, ms_max)
     peaks, peak_src = load_peaks()
     kernels = {}
     for name, (tot_ms, cnt) in prof.items():
@@ -360,7 +360,7 @@ def run_ours(args, rank, world, dev):
         "roofline": roof,
         "kernels": kernels,
         "gpu_launches": launches,
-        "e2e": {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": job_throughput(tokens, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": io.h2d, "d2h_bytes_per_step": io.d2h},
         "clocks": clk.summary(),
     }
@@ -392,11 +392,25 @@ def _barrier(world):
 
 
 def _max_over_ranks(x, world, dev):
+    """Largest value of x over the ranks (the job is as slow as its slowest
+    replica).  dev: the device the collective's tensor lives on (cuda for
+    NCCL, cpu for gloo)."""
     if world == 1:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of the replica on `rank`: every GPU draws its own batch."""
+    return 1000 + w.index + 7919 * rank
+
+
+def job_throughput(tokens_per_replica: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every replica processes its own batch, the job
+    takes as long as the slowest one."""
+    return world * tokens_per_replica / (ms_max / 1e3)
 
 
 # ------------------------------------------------------ CPU oracle timings
