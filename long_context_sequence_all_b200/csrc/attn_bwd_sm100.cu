@@ -17,9 +17,10 @@
 //     P^T and dS^T stay in TMEM (A operand of dV / dK); dK and dV stay in
 //     TMEM until the end.
 //  3. dQ kernel, query-stationary: a CTA owns 128 query rows of one head
-//     with Q and dO resident in TMEM, and streams K/V tiles of 64 keys:
-//       S = Q K^T, dP = dO V^T (M=128, N=64, K=128);  dQ += dS K (N=128, K=64)
-//     all with the A operand in TMEM (only K and V cross shared memory).
+//     with Q and dO resident in TMEM, and streams K/V tiles of 128 keys:
+//       S = Q K^T, dP = dO V^T (M=128, N=128, K=128, A from TMEM)
+//       dQ += dS K             (M=128, N=128, K=128, dS through shared memory)
+//     The next tile's S, dP are issued while the current tile's dS is computed.
 //
 // TMA loads with 128-byte swizzle feed shared memory; one thread issues all
 // MMAs; every wait is bounded (ULY_ERR_TIMEOUT).
@@ -317,20 +318,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ================================================================== dQ
-// One CTA = one 128-row query tile of one query head.  Q and dO sit in TMEM
-// as the A operands of S = Q K^T and dP = dO V^T; S/dP are double-buffered
-// across 64-key tiles and the two compute warpgroups take alternate tiles;
-// dS goes back into the S columns of TMEM and dQ += dS K is also issued from
-// TMEM, so shared memory only carries K and V (six-stage ring).
+// One CTA = one 128-row query tile of one query head; Q and dO sit in TMEM
+// as the A operands of S = Q K^T and dP = dO V^T over K/V tiles of 128 keys
+// (all MMAs N=128).  The two compute warpgroups split each tile's key columns
+// (64 each).  As soon as both have copied S and dP into registers they
+// release the TMEM region, and the MMA thread issues the next tile's S and dP
+// while they compute dS; dS goes through shared memory to dQ += dS K.
 namespace qk {
 constexpr int kBM = 128;   // query rows per CTA
-constexpr int kBK = 64;    // keys per K/V tile
-constexpr int kStages = 6;
-constexpr uint32_t kKBytes = 64 * 128 * 2;                 // one K or V tile
-constexpr uint32_t kOffBar = kStages * 2 * kKBytes;        // stage s: K at s*2*kKBytes, V after it
+constexpr int kBK = 128;   // keys per K/V tile
+constexpr int kStages = 3;
+constexpr uint32_t kTile = 128 * 128 * 2;                  // one 128 x 128 bf16 tile
+constexpr uint32_t kOffKV = 0;                             // stage s: K at 2s*kTile, V at (2s+1)*kTile
+constexpr uint32_t kOffDS = kStages * 2 * kTile;           // dS [128 q][128 keys], K-major swizzled
+constexpr uint32_t kOffBar = kOffDS + kTile;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-// TMEM columns: Q, dO (bf16 pairs), dQ (fp32), then S_b, dP_b for b = 0, 1
-constexpr uint32_t kTQ = 0, kTO = 64, kTdQ = 128, kTS = 256;
+// TMEM columns: Q, dO (bf16 pairs), dQ (fp32), S, dP
+constexpr uint32_t kTQ = 0, kTO = 64, kTdQ = 128, kTS = 256, kTP = 384;
 }  // namespace qk
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -341,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  enum { B_KF = 0, B_KE = kStages, B_S = 2 * kStages, B_P = B_S + 2, B_QO = B_P + 2, B_DQ = B_QO + 1,
-         B_DRAIN = B_DQ + 1, B_N = B_DRAIN + 1 };
+  enum { B_KF = 0, B_KE = kStages, B_S = 2 * kStages, B_SR = B_S + 1, B_P = B_SR + 1, B_DSF = B_P + 1,
+         B_QO = B_DSF + 1, B_DQ = B_QO + 1, B_DRAIN = B_DQ + 1, B_N = B_DRAIN + 1 };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -364,8 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_N; ++i) {
       uint32_t cnt = 1;
-      if (i == B_P || i == B_P + 1) cnt = 128;
-      if (i == B_QO) cnt = 256;
+      if (i == B_SR || i == B_P || i == B_QO) cnt = 256;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Registers: producer / MMA warpgroup 120 per thread, the two compute
-  // warpgroups 192 (a thread holds its whole 128-column S | dP row).
+  // warpgroups 192 (a thread holds 64 columns of S and 64 of dP).
 
   if (warp < 4) {
     setmaxnreg_dec<kRegsCtlQ>();
@@ -392,12 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < NT; ++j) {
           const int s = j % kStages, use = j / kStages;
           if (use > 0 && !mbar_wait(bar(B_KE + s), (use - 1) & 1, abort_flag, prm.err)) break;
-          const uint32_t st = sb + s * 2 * kKBytes;
+          const uint32_t st = sb + kOffKV + s * 2 * kTile;
           const int row0 = (jt0 + j) * kBK;
-          mbar_arrive_expect_tx(bar(B_KF + s), 2 * kKBytes);
+          mbar_arrive_expect_tx(bar(B_KF + s), 2 * kTile);
           for (int c = 0; c < 2; ++c) {
-            tma_load_3d(st + c * 8192, &tmK, bar(B_KF + s), c * 64, row0, kvhead);
-            tma_load_3d(st + kKBytes + c * 8192, &tmV, bar(B_KF + s), c * 64, row0, kvhead);
+            tma_load_3d(st + c * 16384, &tmK, bar(B_KF + s), c * 64, row0, kvhead);
+            tma_load_3d(st + kTile + c * 16384, &tmV, bar(B_KF + s), c * 64, row0, kvhead);
           }
           issued = j + 1;
         }
@@ -409,38 +412,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && NT > 0) {
         bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err);
         tc_fence_after();
-        // S_b = Q K_j^T and dP_b = dO V_j^T, A operands from TMEM
+        // S = Q K_j^T, dP = dO V_j^T: A from TMEM, B = K / V tile (K-major), N = 128
         auto issue_sdp = [&](int j) -> bool {
-          const int b = j & 1, s = j % kStages;
+          const int s = j % kStages;
           if (!mbar_wait(bar(B_KF + s), (j / kStages) & 1, abort_flag, prm.err)) return false;
           tc_fence_after();
-          const uint32_t kst = sb + s * 2 * kKBytes;
-          const uint64_t dK = sdesc_sw128(kst, 16, 1024), dV = sdesc_sw128(kst + kKBytes, 16, 1024);
-          const uint32_t tS = tmem + kTS + 128 * b;
+          const uint32_t kst = sb + kOffKV + s * 2 * kTile;
+          const uint64_t dK = sdesc_sw128(kst, 16, 1024), dV = sdesc_sw128(kst + kTile, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
-            const uint32_t ko = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16_ts(tS, tmem + kTQ + kk * 8, sdesc_add(dK, ko), kIdescN64, kk > 0);
-            mma_bf16_ts(tS + 64, tmem + kTO + kk * 8, sdesc_add(dV, ko), kIdescN64, kk > 0);
+            const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ts(tmem + kTS, tmem + kTQ + kk * 8, sdesc_add(dK, ko), kIdescN128, kk > 0);
+            mma_bf16_ts(tmem + kTP, tmem + kTO + kk * 8, sdesc_add(dV, ko), kIdescN128, kk > 0);
           }
-          tc_commit(bar(B_S + b));
+          tc_commit(bar(B_S));
           return true;
         };
+        const uint64_t dS = sdesc_sw128(sb + kOffDS, 16, 1024);
         if (ok) ok = issue_sdp(0);
-        if (ok && NT > 1) ok = issue_sdp(1);
         for (int j = 0; ok && j < NT; ++j) {
-          const int b = j & 1, s = j % kStages;
-          ok = mbar_wait(bar(B_P + b), (j >> 1) & 1, abort_flag, prm.err);
+          const int s = j % kStages;
+          // both warpgroups hold S_j and dP_j in registers: the region is free
+          ok = mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          // dQ += dS_b K_j: A = dS (bf16 pairs in the S_b columns), B = K tile MN-major over d
-          const uint64_t dKm = sdesc_sw128(sb + s * 2 * kKBytes, 8192, 1024);
+          if (j + 1 < NT) {
+            ok = issue_sdp(j + 1);
+            if (!ok) break;
+          }
+          ok = mbar_wait(bar(B_P), j & 1, abort_flag, prm.err);
+          if (!ok) break;
+          tc_fence_after();
+          // dQ += dS K_j: A = dS (shared memory, K-major), B = K tile MN-major over d
+          const uint64_t dKm = sdesc_sw128(sb + kOffKV + s * 2 * kTile, 16384, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ts(tmem + kTdQ, tmem + kTS + 128 * b + kk * 8, sdesc_add(dKm, kk * 2048), kIdescN128MN,
-                        (j > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ss(tmem + kTdQ, sdesc_add(dS, (kk >> 2) * 16384 + (kk & 3) * 32),
+                        sdesc_add(dKm, kk * 2048), kIdescN128MN, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(B_DSF));
           tc_commit(bar(B_KE + s));
-          if (j + 2 < NT) ok = issue_sdp(j + 2);
         }
         if (ok) tc_commit(bar(B_DQ));
         if (!ok) {
@@ -451,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     setmaxnreg_inc<kRegsComputeQ>();
-    const int b = (warp - 4) >> 2, wq = warp & 3;   // b: even / odd key tiles
+    const int w = (warp - 4) >> 2, wq = warp & 3;   // w: key columns [64w, 64w + 64) of each tile
     const int row = wq * 32 + lane;
     const int i = m0 + row;
     const bool valid = i < g.n;
@@ -463,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     // warpgroup 0 puts this row of Q into TMEM, warpgroup 1 the row of dO
     {
-      const __nv_bfloat16 *src = (b == 0) ? prm.q : prm.dout;
+      const __nv_bfloat16 *src = (w == 0) ? prm.q : prm.dout;
       uint32_t v[64];
       const uint4 *p4 = reinterpret_cast<const uint4 *>(src + (valid ? qrow : 0) * kHD);
 #pragma unroll
@@ -474,21 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         v[4 * u + 2] = w4.z;
         v[4 * u + 3] = w4.w;
       }
-      tmem_st64_nowait(tmem + lane_off + (b == 0 ? kTQ : kTO), v);
+      tmem_st64_nowait(tmem + lane_off + (w == 0 ? kTQ : kTO), v);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_QO));
     }
-    const uint32_t tS = tmem + lane_off + kTS + 128 * b;
+    const uint32_t ds_base = sb + kOffDS;
     bool ok = true;
-    for (int j = b; j < NT; j += 2) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S + b), (j >> 1) & 1, abort_flag, prm.err));
+    for (int j = 0; j < NT; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S), j & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
-      const int n0 = (jt0 + j) * kBK;
-      const bool full = (n0 >= lo_last) && (n0 + kBK - 1 <= hi_first) && (n0 + kBK <= g.n);
-      uint32_t r[128];                         // r[0..63] S, r[64..127] dP: one read
-      tmem_ld128(tS, r);
+      uint32_t r[128];                         // r[0..63] S, r[64..127] dP of this warpgroup's keys
+      tmem_ld64x2(tmem + lane_off + kTS + 64 * w, tmem + lane_off + kTP + 64 * w, r);
+      tc_fence_before();
+      mbar_arrive(bar(B_SR));                  // the MMA thread may now overwrite S and dP
+      const int n0 = (jt0 + j) * kBK + 64 * w;
+      const bool full = (n0 >= lo_last) && (n0 + 63 <= hi_first) && (n0 + 64 <= g.n);
       uint32_t dd[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
@@ -504,35 +516,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         dd[c >> 1] = pack_bf16x2(ds[0], ds[1]);
       }
-      tmem_st32_nowait(tS, dd);                // dS (bf16 pairs) into S columns [0, 32)
-      tmem_st_wait();
+      // dS of the previous tile must have been consumed by its dQ MMA
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSF), (j - 1) & 1, abort_flag, prm.err));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(ds_base + sw128_offset(row, 8 * w + u), dd[4 * u], dd[4 * u + 1], dd[4 * u + 2],
+                     dd[4 * u + 3]);
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(B_P + b));
+      mbar_arrive(bar(B_P));
     }
-    // epilogue: warpgroup b writes dQ columns [64b, 64b + 64)
+    // epilogue: warpgroup w writes dQ columns [64w, 64w + 64)
     if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, abort_flag, prm.err));
     tc_fence_after();
     if (ok && NT > 0) {
-      uint32_t r[32];
+      uint32_t rr[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        tmem_ld32(tmem + lane_off + kTdQ + 64 * b + 32 * c, r);
+        tmem_ld32(tmem + lane_off + kTdQ + 64 * w + 32 * c, rr);
         if (valid) {
-          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * b + 32 * c);
+          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * w + 32 * c);
           const float sc = g.scale;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 w4;
-            w4.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
-            w4.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
-            w4.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
-            w4.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
+            w4.x = pack_bf16x2(__uint_as_float(rr[8 * u + 0]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
+            w4.y = pack_bf16x2(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
+            w4.z = pack_bf16x2(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
+            w4.w = pack_bf16x2(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
             dptr[u] = w4;
           }
         }
       }
     } else if (NT == 0 && valid) {
-      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * b);
+      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * w);
       for (int u = 0; u < 8; ++u) dptr[u] = make_uint4(0, 0, 0, 0);
     }
   }
@@ -593,7 +613,7 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   dim3 gq(qheads, (g.n + qk::kBM - 1) / qk::kBM);
   {
     prof::Scope scope(prof::K_ATTN_DQ_SM100, stream);
-    attn_dq_sm100_kernel<<<gq, kThreads, qk::kSmemBytes, stream>>>(mK64, mV64, prm);
+    attn_dq_sm100_kernel<<<gq, kThreads, qk::kSmemBytes, stream>>>(mK128, mV128, prm);
   }
   note_launches(2);
   return last_launch_status();
