@@ -14,8 +14,9 @@
 //     sees them; the two compute warpgroups split each tile's query columns:
 //       S^T  = K Q^T,  dP^T = V dO^T          (M=128 keys, N=128 queries, K=128)
 //       dV  += P^T dO, dK  += dS^T Q           (M=128 keys, N=128,      K=128)
-//     P^T and dS^T stay in TMEM (A operand of dV / dK); dK and dV stay in
-//     TMEM until the end.
+//     P^T goes through shared memory (A of dV), dS^T stays in TMEM (A of
+//     dK); dK and dV stay in TMEM until the end.  The next tile's S^T and dP^T
+//     are issued while the current tile's P^T and dS^T are computed.
 //  3. dQ kernel, query-stationary: a CTA owns 128 query rows of one head
 //     with Q and dO resident in TMEM, and streams K/V tiles of 128 keys:
 //       S = Q K^T, dP = dO V^T (M=128, N=128, K=128, A from TMEM)
@@ -42,7 +43,7 @@ constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsCtlKV = 136, kRegsComputeKV = 184;  // dK/dV kernel
+constexpr int kRegsCtlKV = 120, kRegsComputeKV = 192;  // dK/dV kernel
 constexpr int kRegsCtlQ = 120, kRegsComputeQ = 192;    // dQ kernel
 static_assert(128 * kRegsCtlKV + 256 * kRegsComputeKV == kThreads * kRegsLaunch &&
                   128 * kRegsCtlQ + 256 * kRegsComputeQ == kThreads * kRegsLaunch,
@@ -73,13 +74,21 @@ __device__ __forceinline__ uint32_t sw128_row64(int row, int chunk) {
 
 // ============================================================== dK / dV
 // One CTA = 128 keys of one KV head; it visits every 128-row query tile (of
-// every query head of the group) that sees them, one tile at a time:
+// every query head of the group) that sees them:
 //   S^T  = K Q^T,  dP^T = V dO^T   (M=128 keys, N=128 queries, K=128; A and B from smem)
-//   dV  += P^T dO, dK  += dS^T Q    (M=128, N=128, K=128 queries; A from TMEM)
+//   dV  += P^T dO                  (M=128, N=128, K=128 queries; P^T from smem)
+//   dK  += dS^T Q                  (M=128, N=128, K=128 queries; dS^T from TMEM)
 // The two compute warpgroups split the 128 query columns of a tile (64
-// each); each writes its half of P^T and dS^T (bf16 pairs) over TMEM columns
-// of S^T / dP^T that it has itself already read, so the halves never race.
-// All MMAs are N=128 (N=64 instructions run at two thirds of the rate).
+// each).  A tile is processed in two phases so that the tensor cores always
+// have the next MMA queued:
+//   a/b. read S^T into registers (the S^T columns are then free and the next
+//        tile's S^T is issued), P^T = exp2(S^T scale log2e - LSE log2e),
+//        P^T (bf16) to shared memory  -> dV MMA
+//   c.   read dP^T, dS^T = P^T (dP^T - D), dS^T (bf16 pairs) over this
+//        warpgroup's own dP^T columns -> dK MMA, then the next tile's dP^T.
+// TMEM: dV [0,128), dK [128,256), S^T [256,384), dP^T / dS^T [384,512).
+// Writes to a TMEM region that an earlier MMA reads (the next S^T over S^T,
+// the next dP^T over dS^T) rely on tcgen05.mma executing in issue order.
 namespace kv {
 constexpr int kBN = 128;   // keys per CTA
 constexpr int kBQ = 128;   // query rows per tile
@@ -87,10 +96,11 @@ constexpr int kStages = 2;
 constexpr uint32_t kTile = 128 * 128 * 2;          // one 128 x 128 bf16 tile
 constexpr uint32_t kOffK = 0, kOffV = kTile;
 constexpr uint32_t kOffStage = 2 * kTile;          // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
-constexpr uint32_t kOffLD = kOffStage + kStages * 2 * kTile;   // per WG: 64 lse*log2e + 64 D
+constexpr uint32_t kOffPT = kOffStage + kStages * 2 * kTile;   // P^T [128 keys][128 q], K-major swizzled
+constexpr uint32_t kOffLD = kOffPT + kTile;        // per WG: 64 lse*log2e + 64 D
 constexpr uint32_t kOffBar = kOffLD + 2 * 512;
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
-// TMEM columns: dV, dK, S^T, dP^T
+static_assert(kSmemBytes <= 232448, "dK/dV kernel exceeds the shared memory of one SM");
 constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTP = 384;
 }  // namespace kv
 
@@ -103,8 +113,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  enum { B_KV = 0, B_SF_ = 1, B_SE = 1 + kStages, B_S = 1 + 2 * kStages, B_P = B_S + 1, B_DONE = B_P + 1,
-         B_DRAIN = B_DONE + 1, B_N = B_DRAIN + 1 };
+  enum { B_KV = 0, B_QF = 1, B_QE = 1 + kStages, B_SF = 1 + 2 * kStages, B_SR = B_SF + 1, B_PS = B_SR + 1,
+         B_PE = B_PS + 1, B_DPF = B_PE + 1, B_DS = B_DPF + 1, B_DONE = B_DS + 1, B_DRAIN = B_DONE + 1,
+         B_N = B_DRAIN + 1 };
+  static_assert(8 * B_N + 8 <= 128, "barrier area");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -125,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = nqt * g.group;                   // tiles: head-major
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P) ? 256 : 1);
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_SR || i == B_PS || i == B_DS) ? 256 : 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmK);
@@ -141,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Registers: producer / MMA warpgroup 136 per thread, the two compute
-  // warpgroups 184 (a thread holds 64 columns of S^T and 64 of dP^T).
+  // Registers: producer / MMA warpgroup 120 per thread, the two compute
+  // warpgroups 192 (a thread holds 64 values of P^T and 64 of dP^T).
 
   if (warp < 4) {
   setmaxnreg_dec<kRegsCtlKV>();
@@ -156,61 +168,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int t = 0; t < T; ++t) {
         const int s = t % kStages, use = t / kStages;
-        if (use > 0 && !mbar_wait(bar(B_SE + s), (use - 1) & 1, abort_flag, prm.err)) break;
+        if (use > 0 && !mbar_wait(bar(B_QE + s), (use - 1) & 1, abort_flag, prm.err)) break;
         const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
         const uint32_t st = sb + kOffStage + s * 2 * kTile;
-        mbar_arrive_expect_tx(bar(B_SF_ + s), 2 * kTile);
+        mbar_arrive_expect_tx(bar(B_QF + s), 2 * kTile);
         for (int c = 0; c < 2; ++c) {
-          tma_load_3d(st + c * 16384, &tmQ, bar(B_SF_ + s), c * 64, i0, qh_base + e);
-          tma_load_3d(st + kTile + c * 16384, &tmO, bar(B_SF_ + s), c * 64, i0, qh_base + e);
+          tma_load_3d(st + c * 16384, &tmQ, bar(B_QF + s), c * 64, i0, qh_base + e);
+          tma_load_3d(st + kTile + c * 16384, &tmO, bar(B_QF + s), c * 64, i0, qh_base + e);
         }
         issued = t + 1;
       }
       if (*abort_flag)
         for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
-          mbar_wait(bar(B_SF_ + t % kStages), (t / kStages) & 1, nullptr, prm.err);
+          mbar_wait(bar(B_QF + t % kStages), (t / kStages) & 1, nullptr, prm.err);
     }
   } else if (warp == 1) {
     if (lane == 0 && T > 0) {
       bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
-      tc_fence_after();
       const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
-      // S^T = K Q_t^T, dP^T = V dO_t^T (N = 128 query rows)
-      auto issue_sdp = [&](int t) -> bool {
-        const int s = t % kStages;
-        if (!mbar_wait(bar(B_SF_ + s), (t / kStages) & 1, abort_flag, prm.err)) return false;
+      const uint64_t dPT = sdesc_sw128(sb + kOffPT, 16, 1024);
+      auto stage_ready = [&](int t) -> bool {
+        const bool r = mbar_wait(bar(B_QF + t % kStages), (t / kStages) & 1, abort_flag, prm.err);
         tc_fence_after();
-        const uint32_t st = sb + kOffStage + s * 2 * kTile;
-        const uint64_t dQ = sdesc_sw128(st, 16, 1024), dO = sdesc_sw128(st + kTile, 16, 1024);
+        return r;
+      };
+      // S^T = K Q_t^T (N = 128 query rows)
+      auto issue_s = [&](int t) {
+        const uint64_t dQ = sdesc_sw128(sb + kOffStage + (t % kStages) * 2 * kTile, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
           mma_bf16_ss(tmem + kTS, sdesc_add(dK, ko), sdesc_add(dQ, ko), kIdescN128, kk > 0);
+        }
+        tc_commit(bar(B_SF));
+      };
+      // dP^T = V dO_t^T
+      auto issue_dp = [&](int t) {
+        const uint64_t dO = sdesc_sw128(sb + kOffStage + (t % kStages) * 2 * kTile + kTile, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kHD / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
           mma_bf16_ss(tmem + kTP, sdesc_add(dV, ko), sdesc_add(dO, ko), kIdescN128, kk > 0);
         }
-        tc_commit(bar(B_S));
-        return true;
+        tc_commit(bar(B_DPF));
       };
-      if (ok) ok = issue_sdp(0);
+      if (ok) ok = stage_ready(0);
+      if (ok) {
+        issue_s(0);
+        issue_dp(0);
+      }
       for (int t = 0; ok && t < T; ++t) {
         const int s = t % kStages;
-        ok = mbar_wait(bar(B_P), t & 1, abort_flag, prm.err);
+        const uint32_t st = sb + kOffStage + s * 2 * kTile;
+        // both warpgroups hold S^T_t in registers: issue S^T_{t+1}
+        if (t + 1 < T) {
+          ok = mbar_wait(bar(B_SR), t & 1, abort_flag, prm.err) && stage_ready(t + 1);
+          if (!ok) break;
+          issue_s(t + 1);
+        }
+        // dV += P^T dO_t: A = P^T (shared memory, K-major), B = dO tile MN-major over d
+        ok = mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dO_t, dK += dS^T Q_t: A from TMEM (query columns [0,64) in
-        // the S^T / dP^T columns [0,32), [64,128) in columns [64,96)), B = dO /
-        // Q tile, MN-major over d
-        const uint32_t st = sb + kOffStage + s * 2 * kTile;
-        const uint64_t dQm = sdesc_sw128(st, 16384, 1024), dOm = sdesc_sw128(st + kTile, 16384, 1024);
+        const uint64_t dOm = sdesc_sw128(st + kTile, 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kBQ / 16; ++kk)
+          mma_bf16_ss(tmem + kTdV, sdesc_add(dPT, (kk >> 2) * 16384 + (kk & 3) * 32),
+                      sdesc_add(dOm, kk * 2048), kIdescN128MN, (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(B_PE));
+        // dK += dS^T Q_t: A from TMEM (query columns [0,64) in the dP^T
+        // columns [0,32), [64,128) in [64,96)), B = Q tile MN-major over d
+        ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dQm = sdesc_sw128(st, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk) {
           const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ts(tmem + kTdV, tmem + kTS + acol, sdesc_add(dOm, kk * 2048), kIdescN128MN, acc);
-          mma_bf16_ts(tmem + kTdK, tmem + kTP + acol, sdesc_add(dQm, kk * 2048), kIdescN128MN, acc);
+          mma_bf16_ts(tmem + kTdK, tmem + kTP + acol, sdesc_add(dQm, kk * 2048), kIdescN128MN,
+                      (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(B_SE + s));
-        if (t + 1 < T) ok = issue_sdp(t + 1);
+        tc_commit(bar(B_QE + s));
+        if (t + 1 < T) issue_dp(t + 1);
       }
       if (ok) tc_commit(bar(B_DONE));
       if (!ok) {
@@ -229,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (j < g.n) prm.mk.col_range(j, lo_j, hi_j);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + kTS + 64 * w, tP = tmem + lane_off + kTP + 64 * w;
+    const uint32_t pt_base = sb + kOffPT;
     float *lsm = reinterpret_cast<float *>(smem + kOffLD + w * 512);  // [0,64) lse*log2e, [64,128) D
     // this thread's share of the per-tile statistics: LSE (tid < 64) or D of
     // query row i0 + 64w + (tid & 63); fetched one tile ahead of its use
@@ -248,16 +288,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       lsm[tid] = stat_next;
       named_bar_sync(1 + w, 128);
       stat_next = fetch_stat(t + 1);           // in flight while this tile is processed
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S), t & 1, abort_flag, prm.err));
+      // phase a/b: P^T
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
-      uint32_t r[128];                         // r[0..63] S^T, r[64..127] dP^T of this warpgroup's columns
-      tmem_ld64x2(tS, tP, r);
-      uint32_t pp[32], dd[32];
+      uint32_t r[64];
+      tmem_ld64(tS, r);
+      tc_fence_before();
+      mbar_arrive(bar(B_SR));                  // the MMA thread may now overwrite S^T
+      uint32_t pp[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        float p[2], ds[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           float pv = ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lsm[c + u]));
@@ -265,18 +307,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = i0 + c + u;
             if (i < lo_j || i > hi_j) pv = 0.f;
           }
-          p[u] = pv;
-          ds[u] = pv * (__uint_as_float(r[64 + c + u]) - lsm[64 + c + u]);
+          r[c + u] = __float_as_uint(pv);
         }
-        pp[c >> 1] = pack_bf16x2(p[0], p[1]);
-        dd[c >> 1] = pack_bf16x2(ds[0], ds[1]);
+        pp[c >> 1] = pack_bf16x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
       }
-      // P^T and dS^T (bf16 pairs) over this warpgroup's first 32 columns of S^T / dP^T
-      tmem_st32_nowait(tS, pp);
+      // the previous tile's P^T must have been consumed by its dV MMA
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PE), (t - 1) & 1, abort_flag, prm.err));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(pt_base + sw128_offset(row, 8 * w + u), pp[4 * u], pp[4 * u + 1], pp[4 * u + 2],
+                     pp[4 * u + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_PS));
+      // phase c: dS^T
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dp[64];
+      tmem_ld64(tP, dp);
+      uint32_t dd[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float d0 = __uint_as_float(r[c]) * (__uint_as_float(dp[c]) - lsm[64 + c]);
+        const float d1 = __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - lsm[64 + c + 1]);
+        dd[c >> 1] = pack_bf16x2(d0, d1);
+      }
+      // dS^T (bf16 pairs) over this warpgroup's first 32 columns of dP^T
       tmem_st32_nowait(tP, dd);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(B_P));
+      mbar_arrive(bar(B_DS));
     }
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (scaled)
     if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err));
