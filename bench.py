@@ -76,7 +76,8 @@ def algorithmic_work(inp):
         "attn_fwd_sm100": ("flops", 4.0 * B * H * d * pairs),
         "attn_dkdv_sm100": ("flops", 8.0 * B * H * d * pairs),   # S, dP, dV, dK
         "attn_dq_sm100": ("flops", 2.0 * B * H * d * pairs),     # dQ (S, dP recomputed)
-        "attn_bwd_dot": ("bytes", 2.0 * qb + B * n * H * 4),
+        # bf16: reads O, dO, LSE; writes D and LSE log2(e)
+        "attn_bwd_dot": ("bytes", 2.0 * qb + 3 * B * n * H * 4),
     }
     if "logits" in inp:
         valid = int((inp["labels"] != -100).sum())
@@ -222,7 +223,7 @@ def load_peaks():
 def kernel_source_hash(kernel: str) -> str:
     files = {"attn_fwd_sm100": "attn_fwd_sm100.cu", "attn_dkdv_sm100": "attn_bwd_sm100.cu",
              "attn_dq_sm100": "attn_bwd_sm100.cu", "seq_to_head": "permute.cu", "head_to_seq": "permute.cu",
-             "loss_partial": "loss.cu", "attn_bwd_dot": "attn_f32.cu"}
+             "loss_partial": "loss.cu", "attn_bwd_dot": "attn_bwd_sm100.cu"}
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_sequence_all_b200", "csrc")
     for f in [files.get(kernel, ""), "sm100.cuh", "common.cuh"]:

@@ -158,7 +158,13 @@ uly_status ulysses_attn_bwd_workspace_size(const uly_attn_desc *d, size_t *bytes
   if (!bytes) return ULY_ERR_NULL;
   uly_status st = check_desc(d, g, mk);
   if (st != ULY_OK) return st;
-  *bytes = align256(lse_bytes(d));  // D_i = <dO_i, O_i> for every query row
+  if (d->dtype == ULY_BF16) {
+    // D_i and LSE_i log2(e), query rows padded per head
+    const long long rows_pad = (long long)d->batch * d->n_q_heads * bwd_rows_padded(d->seq_len);
+    *bytes = 2 * sizeof(float) * (size_t)bwd_stats_stride(rows_pad);
+  } else {
+    *bytes = align256(lse_bytes(d));  // D_i = <dO_i, O_i> for every query row
+  }
   return ULY_OK;
 }
 

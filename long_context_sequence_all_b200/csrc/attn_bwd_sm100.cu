@@ -8,7 +8,9 @@
 // with dK, dV summed over the query heads that share a KV head (GQA).
 //
 // Three launches, all deterministic (no atomics):
-//  1. D_i = <dO_i, O_i>   (one warp per row, HBM-bound)
+//  1. D_i = <dO_i, O_i> and LSE_i log2(e) into arrays whose query rows are
+//     padded to a multiple of 128 (zeros past n), so that every 128-row tile
+//     of them is one aligned 512-byte block (HBM-bound)
 //  2. dK/dV kernel, KV-stationary: a CTA owns 128 keys of one KV head and
 //     visits every 128-row query tile (of every query head of the group) that
 //     sees them; the two compute warpgroups split each tile's query columns:
@@ -33,8 +35,6 @@ namespace uly {
 using namespace sm100;
 
 bool make_tmap_heads_bf16(CUtensorMap *map, const void *base, int d, int n, int heads, int box_rows);
-uly_status attn_bwd_dot_launch(int dtype, int head_dim, const void *o, const void *dout, float *Dv,
-                               long long rows, cudaStream_t stream);
 
 namespace {
 
@@ -49,27 +49,56 @@ static_assert(128 * kRegsCtlKV + 256 * kRegsComputeKV == kThreads * kRegsLaunch 
                   128 * kRegsCtlQ + 256 * kRegsComputeQ == kThreads * kRegsLaunch,
               "register split must use exactly the launch pool");
 
-constexpr uint32_t kIdescN64 = idesc_bf16_f32(128, 64, false, false);    // K-major A and B, N = 64
 constexpr uint32_t kIdescN128 = idesc_bf16_f32(128, 128, false, false);  // K-major A and B, N = 128
 constexpr uint32_t kIdescN128MN = idesc_bf16_f32(128, 128, false, true); // B MN-major, N = 128
 
 struct BwdParams {
   const __nv_bfloat16 *q;     // [qheads][n][d] (dQ kernel: Q rows go into TMEM)
   const __nv_bfloat16 *dout;  // [qheads][n][d]
-  const float *lse;   // [qheads][n]
-  const float *Dv;    // [qheads][n]
+  const float *lse2;  // [qheads][n_pad]: LSE log2(e), 0 past n
+  const float *Dv;    // [qheads][n_pad]: D, 0 past n
   __nv_bfloat16 *out0;  // dkdv: dV, dq: dQ
   __nv_bfloat16 *out1;  // dkdv: dK
   HeadGeom g;
   MaskInfo mk;
   float scale_log2;
+  int n_pad;          // n rounded up to a multiple of 128
   int *err;
 };
 
-// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a [rows][64]
-// bf16 operand stored as one 128-byte-swizzled span per row.
-__device__ __forceinline__ uint32_t sw128_row64(int row, int chunk) {
-  return (uint32_t)(row * 128 + (((chunk ^ (row & 7))) << 4));
+// D_i = <dO_i, O_i> and LSE_i log2(e) of every query row (two rows per warp,
+// 16-byte loads), written to the padded per-head arrays; rows n..n_pad-1 get 0.
+__global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                             const __nv_bfloat16 *__restrict__ dout,
+                                                             const float *__restrict__ lse,
+                                                             float *__restrict__ Dpad,
+                                                             float *__restrict__ L2pad, int n, int n_pad,
+                                                             long long rows_pad) {
+  const long long r = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const int l = threadIdx.x & 15;
+  const long long h = r / n_pad;
+  const int i = (int)(r - h * n_pad);
+  const bool valid = r < rows_pad && i < n;
+  float acc = 0.f;
+  if (valid) {
+    const long long src = (h * n + i) * kHD;
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(o + src) + l);
+    const uint4 b = __ldg(reinterpret_cast<const uint4 *>(dout + src) + l);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&av[u]));
+      const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bv[u]));
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (l == 0 && r < rows_pad) {
+    Dpad[r] = acc;
+    L2pad[r] = valid ? __ldg(lse + h * n + i) * kLog2e : 0.f;
+  }
 }
 
 // ============================================================== dK / dV
@@ -97,10 +126,16 @@ constexpr uint32_t kTile = 128 * 128 * 2;          // one 128 x 128 bf16 tile
 constexpr uint32_t kOffK = 0, kOffV = kTile;
 constexpr uint32_t kOffStage = 2 * kTile;          // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
 constexpr uint32_t kOffPT = kOffStage + kStages * 2 * kTile;   // P^T [128 keys][128 q], K-major swizzled
-constexpr uint32_t kOffLD = kOffPT + kTile;        // per WG: 64 lse*log2e + 64 D
-constexpr uint32_t kOffBar = kOffLD + 2 * 512;
-constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
-static_assert(kSmemBytes <= 232448, "dK/dV kernel exceeds the shared memory of one SM");
+constexpr uint32_t kOffStats = kOffPT + kTile;     // stage s: 128 LSE log2(e), then 128 D of its tile
+constexpr uint32_t kStatBytes = 2 * kBQ * 4;
+constexpr uint32_t kBarBytes = 128;
+// The tiles need a 1024-byte-aligned base.  The barriers go in front of it
+// when the alignment gap can hold them, else after the statistics; either
+// way the whole fits the 227 KB an SM offers one CTA.
+constexpr uint32_t kSmemBytes = 232448;
+static_assert(1023 + kOffStats + kStages * kStatBytes <= kSmemBytes &&
+                  (kBarBytes - 1) + kOffStats + kStages * kStatBytes + kBarBytes <= kSmemBytes,
+              "dK/dV shared memory layout");
 constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTP = 384;
 }  // namespace kv
 
@@ -109,16 +144,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                            const BwdParams prm) {
   using namespace kv;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t gap = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t *smem = smem_raw + gap;
   const uint32_t sb = smem_u32(smem);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint8_t *bar_area = (gap >= kBarBytes) ? smem_raw : smem + kOffStats + kStages * kStatBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(bar_area);
   enum { B_KV = 0, B_QF = 1, B_QE = 1 + kStages, B_SF = 1 + 2 * kStages, B_SR = B_SF + 1, B_PS = B_SR + 1,
          B_PE = B_PS + 1, B_DPF = B_PE + 1, B_DS = B_DPF + 1, B_DONE = B_DS + 1, B_DRAIN = B_DONE + 1,
          B_N = B_DRAIN + 1 };
-  static_assert(8 * B_N + 8 <= 128, "barrier area");
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
+  static_assert(8 * B_N + 8 <= kBarBytes, "barrier area");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + 8 * B_N);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + 8 * B_N + 4);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const HeadGeom &g = prm.g;
@@ -171,11 +208,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (use > 0 && !mbar_wait(bar(B_QE + s), (use - 1) & 1, abort_flag, prm.err)) break;
         const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
         const uint32_t st = sb + kOffStage + s * 2 * kTile;
-        mbar_arrive_expect_tx(bar(B_QF + s), 2 * kTile);
+        const long long srow = (long long)(qh_base + e) * prm.n_pad + i0;
+        const uint32_t sst = sb + kOffStats + s * kStatBytes;
+        mbar_arrive_expect_tx(bar(B_QF + s), 2 * kTile + kStatBytes);
         for (int c = 0; c < 2; ++c) {
           tma_load_3d(st + c * 16384, &tmQ, bar(B_QF + s), c * 64, i0, qh_base + e);
           tma_load_3d(st + kTile + c * 16384, &tmO, bar(B_QF + s), c * 64, i0, qh_base + e);
         }
+        bulk_load(sst, prm.lse2 + srow, kBQ * 4, bar(B_QF + s));
+        bulk_load(sst + kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_QF + s));
         issued = t + 1;
       }
       if (*abort_flag)
@@ -263,33 +304,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int w = (warp - 4) >> 2, wq = warp & 3;  // w: query columns [64w, 64w + 64)
     const int row = wq * 32 + lane;                // key row within the tile
     const int j = n0 + row;
-    const int tid = threadIdx.x - 128 * (w + 1);   // 0..127 within the warpgroup
     int lo_j = 1, hi_j = 0;
     if (j < g.n) prm.mk.col_range(j, lo_j, hi_j);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + kTS + 64 * w, tP = tmem + lane_off + kTP + 64 * w;
     const uint32_t pt_base = sb + kOffPT;
-    float *lsm = reinterpret_cast<float *>(smem + kOffLD + w * 512);  // [0,64) lse*log2e, [64,128) D
-    // this thread's share of the per-tile statistics: LSE (tid < 64) or D of
-    // query row i0 + 64w + (tid & 63); fetched one tile ahead of its use
-    auto fetch_stat = [&](int t) -> float {
-      if (t >= T) return 0.f;
-      const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
-      const int i = i0 + 64 * w + (tid & 63);
-      const long long idx = (long long)(qh_base + e) * g.n + i;
-      if (tid < 64) return (i < g.n) ? __ldg(prm.lse + idx) * kLog2e : INFINITY;
-      return (i < g.n) ? __ldg(prm.Dv + idx) : 0.f;
-    };
-    float stat_next = fetch_stat(0);
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ + 64 * w;  // this warpgroup's first query row
-      named_bar_sync(1 + w, 128);              // previous tile's LSE/D reads are done
-      lsm[tid] = stat_next;
-      named_bar_sync(1 + w, 128);
-      stat_next = fetch_stat(t + 1);           // in flight while this tile is processed
+      // LSE log2(e) and D of this warpgroup's 64 query rows (loaded with Q / dO)
+      const float *lsm = reinterpret_cast<const float *>(smem + kOffStats + (t % kStages) * kStatBytes) + 64 * w;
+      const float *dsm = lsm + kBQ;
       // phase a/b: P^T
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + t % kStages), (t / kStages) & 1, abort_flag, prm.err) &&
+                                       mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
@@ -331,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t dd[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float d0 = __uint_as_float(r[c]) * (__uint_as_float(dp[c]) - lsm[64 + c]);
-        const float d1 = __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - lsm[64 + c + 1]);
+        const float d0 = __uint_as_float(r[c]) * (__uint_as_float(dp[c]) - dsm[c]);
+        const float d1 = __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - dsm[c + 1]);
         dd[c >> 1] = pack_bf16x2(d0, d1);
       }
       // dS^T (bf16 pairs) over this warpgroup's first 32 columns of dP^T
@@ -531,8 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lo_i = 1, hi_i = 0;
     if (valid) prm.mk.row_range(i, lo_i, hi_i);
     const long long qrow = (long long)qh * g.n + i;
-    const float lse2 = valid ? prm.lse[qrow] * kLog2e : INFINITY;
-    const float Di = valid ? prm.Dv[qrow] : 0.f;
+    const long long srow = (long long)qh * prm.n_pad + i;
+    const float lse2 = valid ? prm.lse2[srow] : INFINITY;
+    const float Di = valid ? prm.Dv[srow] : 0.f;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     // warpgroup 0 puts this row of Q into TMEM, warpgroup 1 the row of dO
     {
@@ -634,10 +663,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const MaskInfo &mk,
                                 const void *q, const void *k, const void *v, const void *o,
                                 const float *lse, const void *dout, void *dq, void *dk, void *dv,
-                                float *Dv, cudaStream_t stream) {
+                                float *workspace, cudaStream_t stream) {
   const int qheads = g.P * g.B * g.hl, kvheads = g.P * g.B * g.gl;
-  uly_status st = attn_bwd_dot_launch(ULY_BF16, d->head_dim, o, dout, Dv, (long long)qheads * g.n, stream);
-  if (st != ULY_OK) return st;
+  const int n_pad = bwd_rows_padded(g.n);
+  const long long rows_pad = (long long)qheads * n_pad;
+  float *Dv = workspace;
+  float *L2 = workspace + bwd_stats_stride(rows_pad);
+  if (rows_pad > 0) {
+    prof::Scope scope(prof::K_ATTN_BWD_DOT, stream);
+    attn_bwd_stats_kernel<<<(unsigned)((rows_pad + 15) / 16), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, Dv, L2, g.n,
+        n_pad, rows_pad);
+    note_launches(1);
+  }
   CUtensorMap mK128, mV128, mQ128, mO128, mK64, mV64;
   if (!make_tmap_heads_bf16(&mK128, k, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&mV128, v, kHD, g.n, kvheads, 128) ||
@@ -658,8 +696,9 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   BwdParams prm;
   prm.q = static_cast<const __nv_bfloat16 *>(q);
   prm.dout = static_cast<const __nv_bfloat16 *>(dout);
-  prm.lse = lse;
+  prm.lse2 = L2;
   prm.Dv = Dv;
+  prm.n_pad = n_pad;
   prm.g = g;
   prm.mk = mk;
   prm.scale_log2 = g.scale * kLog2e;

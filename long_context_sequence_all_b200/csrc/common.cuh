@@ -74,6 +74,12 @@ struct MaskInfo {
   }
 };
 
+// Workspace of the bf16 backward: D_i and LSE_i log2(e) per query row, each
+// head's rows padded to a multiple of 128 so every 128-row tile of them is one
+// aligned 512-byte block; the LSE array starts bwd_stats_stride floats after D.
+__host__ __device__ inline int bwd_rows_padded(int n) { return (n + 127) / 128 * 128; }
+__host__ __device__ inline long long bwd_stats_stride(long long rows_pad) { return (rows_pad + 63) / 64 * 64; }
+
 // Per-launch geometry of the head layout shared by the attention kernels.
 struct HeadGeom {
   int B, n, P, hl, gl, group;  // hl = H/P, gl = G/P, group = H/G
