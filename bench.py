@@ -77,7 +77,7 @@ def algorithmic_work(inp):
         "attn_dkdv_sm100": ("flops", 8.0 * B * H * d * pairs),   # S, dP, dV, dK
         "attn_dq_sm100": ("flops", 2.0 * B * H * d * pairs),     # dQ (S, dP recomputed)
         # bf16: reads O, dO, LSE; writes D and LSE log2(e)
-        "attn_bwd_dot": ("bytes", 2.0 * qb + 3 * B * n * H * 4),
+        "attn_bwd_stats": ("bytes", 2.0 * qb + 3 * B * n * H * 4),
     }
     if "logits" in inp:
         valid = int((inp["labels"] != -100).sum())
@@ -223,7 +223,7 @@ def load_peaks():
 def kernel_source_hash(kernel: str) -> str:
     files = {"attn_fwd_sm100": "attn_fwd_sm100.cu", "attn_dkdv_sm100": "attn_bwd_sm100.cu",
              "attn_dq_sm100": "attn_bwd_sm100.cu", "seq_to_head": "permute.cu", "head_to_seq": "permute.cu",
-             "loss_partial": "loss.cu", "attn_bwd_dot": "attn_bwd_sm100.cu"}
+             "loss_partial": "loss.cu", "attn_bwd_stats": "attn_bwd_sm100.cu"}
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_sequence_all_b200", "csrc")
     for f in [files.get(kernel, ""), "sm100.cuh", "common.cuh"]:
@@ -356,7 +356,7 @@ def run_ours(args, rank, world, dev):
         "attn_fwd_tflops": kernels.get("attn_fwd_sm100", {}).get("tflops"),
         "attn_bwd_tflops": (10.0 * inp["B"] * inp["H"] * inp["d"] * pairs) /
                            (sum(kernels[k]["ms_per_step"] for k in ("attn_dkdv_sm100", "attn_dq_sm100",
-                                                                   "attn_bwd_dot") if k in kernels) / 1e3) / 1e12,
+                                                                   "attn_bwd_stats") if k in kernels) / 1e3) / 1e12,
         "permute_gbs": {k: kernels[k]["gbs"] for k in ("seq_to_head", "head_to_seq") if k in kernels},
         "roofline": roof,
         "kernels": kernels,

@@ -670,7 +670,7 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   float *Dv = workspace;
   float *L2 = workspace + bwd_stats_stride(rows_pad);
   if (rows_pad > 0) {
-    prof::Scope scope(prof::K_ATTN_BWD_DOT, stream);
+    prof::Scope scope(prof::K_ATTN_BWD_STATS, stream);
     attn_bwd_stats_kernel<<<(unsigned)((rows_pad + 15) / 16), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, Dv, L2, g.n,
         n_pad, rows_pad);

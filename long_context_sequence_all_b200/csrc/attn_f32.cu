@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kThreads) attn_dkdv_f32_kernel(
   }
 }
 
-// D_i = <dO_i, O_i> (fp32), one warp per row; T = float or bf16.
+// D_i = <dO_i, O_i> (fp32 path), one warp per row.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_bwd_dot_kernel(const T *__restrict__ o,
                                                            const T *__restrict__ dout,
@@ -304,9 +304,6 @@ uly_status attn_bwd_dot_launch(int dtype, int head_dim, const void *o, const voi
   else if (dtype == ULY_F32 && head_dim == 128)
     attn_bwd_dot_kernel<float, 128><<<blocks, 256, 0, stream>>>(
         static_cast<const float *>(o), static_cast<const float *>(dout), Dv, rows);
-  else if (dtype == ULY_BF16 && head_dim == 128)
-    attn_bwd_dot_kernel<__nv_bfloat16, 128><<<blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), Dv, rows);
   else
     return ULY_ERR_UNSUPPORTED;
   note_launches(1);

@@ -22,6 +22,7 @@ enum Kernel {
   K_ATTN_FWD_SM100,
   K_ATTN_DKDV_SM100,
   K_ATTN_DQ_SM100,
+  K_ATTN_BWD_STATS,
   K_COUNT
 };
 
