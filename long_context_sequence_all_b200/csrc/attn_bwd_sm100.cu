@@ -16,9 +16,8 @@
 //     sees them; the two compute warpgroups split each tile's query columns:
 //       S^T  = K Q^T,  dP^T = V dO^T          (M=128 keys, N=128 queries, K=128)
 //       dV  += P^T dO, dK  += dS^T Q           (M=128 keys, N=128,      K=128)
-//     P^T goes through shared memory (A of dV), dS^T stays in TMEM (A of
-//     dK); dK and dV stay in TMEM until the end.  The next tile's S^T and dP^T
-//     are issued while the current tile's P^T and dS^T are computed.
+//     P^T and dS^T stay in TMEM over S^T / dP^T (A of dV and dK), as do dK
+//     and dV; Q tiles have three shared-memory stages, dO tiles two.
 //  3. dQ kernel, query-stationary: a CTA owns 128 query rows of one head
 //     with Q and dO resident in TMEM, and streams K/V tiles of 128 keys:
 //       S = Q K^T, dP = dO V^T (M=128, N=128, K=128, A from TMEM)
@@ -105,37 +104,35 @@ __global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const __nv_bfloat16
 // One CTA = 128 keys of one KV head; it visits every 128-row query tile (of
 // every query head of the group) that sees them:
 //   S^T  = K Q^T,  dP^T = V dO^T   (M=128 keys, N=128 queries, K=128; A and B from smem)
-//   dV  += P^T dO                  (M=128, N=128, K=128 queries; P^T from smem)
-//   dK  += dS^T Q                  (M=128, N=128, K=128 queries; dS^T from TMEM)
+//   dV  += P^T dO, dK  += dS^T Q    (M=128, N=128, K=128 queries; A from TMEM)
 // The two compute warpgroups split the 128 query columns of a tile (64
-// each).  A tile is processed in two phases so that the tensor cores always
-// have the next MMA queued:
-//   a/b. read S^T into registers (the S^T columns are then free and the next
-//        tile's S^T is issued), P^T = exp2(S^T scale log2e - LSE log2e),
-//        P^T (bf16) to shared memory  -> dV MMA
-//   c.   read dP^T, dS^T = P^T (dP^T - D), dS^T (bf16 pairs) over this
-//        warpgroup's own dP^T columns -> dK MMA, then the next tile's dP^T.
-// TMEM: dV [0,128), dK [128,256), S^T [256,384), dP^T / dS^T [384,512).
-// Writes to a TMEM region that an earlier MMA reads (the next S^T over S^T,
-// the next dP^T over dS^T) rely on tcgen05.mma executing in issue order.
+// each); each writes its half of P^T and dS^T (bf16 pairs) over TMEM columns
+// of S^T / dP^T that it has itself already read, so shared memory holds only
+// operand tiles: K, V, three Q stages (a Q tile is needed until the tile's dK
+// MMA, and the next tiles' Q loads must not sit on the critical path) and two
+// dO stages.  Each tile's LSE log2(e) and D travel with its Q and dO tiles.
+// TMEM: dV [0,128), dK [128,256), S^T / P^T [256,384), dP^T / dS^T [384,512).
+// The next tile's S^T is issued right after this tile's dV MMA and its dP^T
+// right after the dK MMA: they overwrite the P^T / dS^T those MMAs read, which
+// relies on tcgen05.mma executing in issue order.
 namespace kv {
 constexpr int kBN = 128;   // keys per CTA
 constexpr int kBQ = 128;   // query rows per tile
-constexpr int kStages = 2;
+constexpr int kQStages = 3, kOStages = 2;
 constexpr uint32_t kTile = 128 * 128 * 2;          // one 128 x 128 bf16 tile
 constexpr uint32_t kOffK = 0, kOffV = kTile;
-constexpr uint32_t kOffStage = 2 * kTile;          // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
-constexpr uint32_t kOffPT = kOffStage + kStages * 2 * kTile;   // P^T [128 keys][128 q], K-major swizzled
-constexpr uint32_t kOffStats = kOffPT + kTile;     // stage s: 128 LSE log2(e), then 128 D of its tile
-constexpr uint32_t kStatBytes = 2 * kBQ * 4;
-constexpr uint32_t kBarBytes = 128;
+constexpr uint32_t kOffQ = 2 * kTile;                          // Q stage s at kOffQ + s * kTile
+constexpr uint32_t kOffO = kOffQ + kQStages * kTile;           // dO stage s at kOffO + s * kTile
+constexpr uint32_t kOffLse = kOffO + kOStages * kTile;         // per Q stage: 128 LSE log2(e)
+constexpr uint32_t kOffD = kOffLse + kQStages * kBQ * 4;       // per dO stage: 128 D
+constexpr uint32_t kEnd = kOffD + kOStages * kBQ * 4;
+constexpr uint32_t kBarBytes = 160;
+constexpr uint32_t kSmemBytes = 232448;                        // all an SM offers one CTA
 // The tiles need a 1024-byte-aligned base.  The barriers go in front of it
-// when the alignment gap can hold them, else after the statistics; either
-// way the whole fits the 227 KB an SM offers one CTA.
-constexpr uint32_t kSmemBytes = 232448;
-static_assert(1023 + kOffStats + kStages * kStatBytes <= kSmemBytes &&
-                  (kBarBytes - 1) + kOffStats + kStages * kStatBytes + kBarBytes <= kSmemBytes,
-              "dK/dV shared memory layout");
+// when the alignment gap can hold them, else after the statistics; a gap
+// larger than kMaxGap would not fit and is reported (ULY_ERR_UNSUPPORTED).
+constexpr uint32_t kMaxGap = kSmemBytes - kEnd;
+static_assert(kEnd + kBarBytes <= kSmemBytes && kMaxGap >= kBarBytes, "dK/dV shared memory layout");
 constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTP = 384;
 }  // namespace kv
 
@@ -146,13 +143,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   using namespace kv;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t gap = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (gap > kMaxGap) {   // uniform over the CTA: nothing has been started
+    if (threadIdx.x == 0) raise_error(prm.err, ULY_ERR_UNSUPPORTED);
+    return;
+  }
   uint8_t *smem = smem_raw + gap;
   const uint32_t sb = smem_u32(smem);
-  uint8_t *bar_area = (gap >= kBarBytes) ? smem_raw : smem + kOffStats + kStages * kStatBytes;
+  uint8_t *bar_area = (gap >= kBarBytes) ? smem_raw : smem + kEnd;
   uint64_t *bars = reinterpret_cast<uint64_t *>(bar_area);
-  enum { B_KV = 0, B_QF = 1, B_QE = 1 + kStages, B_SF = 1 + 2 * kStages, B_SR = B_SF + 1, B_PS = B_SR + 1,
-         B_PE = B_PS + 1, B_DPF = B_PE + 1, B_DS = B_DPF + 1, B_DONE = B_DS + 1, B_DRAIN = B_DONE + 1,
-         B_N = B_DRAIN + 1 };
+  enum { B_KV = 0, B_QF = 1, B_QE = B_QF + kQStages, B_OF = B_QE + kQStages, B_OE = B_OF + kOStages,
+         B_SF = B_OE + kOStages, B_PS, B_DPF, B_DS, B_DONE, B_DRAIN, B_N };
   static_assert(8 * B_N + 8 <= kBarBytes, "barrier area");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + 8 * B_N + 4);
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = nqt * g.group;                   // tiles: head-major
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_SR || i == B_PS || i == B_DS) ? 256 : 1);
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_PS || i == B_DS) ? 256 : 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmK);
@@ -202,40 +202,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sb + kOffK + c * 16384, &tmK, bar(B_KV), c * 64, n0, kvh);
         tma_load_3d(sb + kOffV + c * 16384, &tmV, bar(B_KV), c * 64, n0, kvh);
       }
-      int issued = 0;
+      int issued_q = 0, issued_o = 0;
       for (int t = 0; t < T; ++t) {
-        const int s = t % kStages, use = t / kStages;
-        if (use > 0 && !mbar_wait(bar(B_QE + s), (use - 1) & 1, abort_flag, prm.err)) break;
         const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
-        const uint32_t st = sb + kOffStage + s * 2 * kTile;
         const long long srow = (long long)(qh_base + e) * prm.n_pad + i0;
-        const uint32_t sst = sb + kOffStats + s * kStatBytes;
-        mbar_arrive_expect_tx(bar(B_QF + s), 2 * kTile + kStatBytes);
-        for (int c = 0; c < 2; ++c) {
-          tma_load_3d(st + c * 16384, &tmQ, bar(B_QF + s), c * 64, i0, qh_base + e);
-          tma_load_3d(st + kTile + c * 16384, &tmO, bar(B_QF + s), c * 64, i0, qh_base + e);
-        }
-        bulk_load(sst, prm.lse2 + srow, kBQ * 4, bar(B_QF + s));
-        bulk_load(sst + kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_QF + s));
-        issued = t + 1;
+        // Q tile and its LSE
+        const int sq = t % kQStages, uq = t / kQStages;
+        if (uq > 0 && !mbar_wait(bar(B_QE + sq), (uq - 1) & 1, abort_flag, prm.err)) break;
+        mbar_arrive_expect_tx(bar(B_QF + sq), kTile + kBQ * 4);
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(sb + kOffQ + sq * kTile + c * 16384, &tmQ, bar(B_QF + sq), c * 64, i0, qh_base + e);
+        bulk_load(sb + kOffLse + sq * kBQ * 4, prm.lse2 + srow, kBQ * 4, bar(B_QF + sq));
+        issued_q = t + 1;
+        // dO tile and its D
+        const int so = t % kOStages, uo = t / kOStages;
+        if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err)) break;
+        mbar_arrive_expect_tx(bar(B_OF + so), kTile + kBQ * 4);
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(sb + kOffO + so * kTile + c * 16384, &tmO, bar(B_OF + so), c * 64, i0, qh_base + e);
+        bulk_load(sb + kOffD + so * kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_OF + so));
+        issued_o = t + 1;
       }
-      if (*abort_flag)
-        for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
-          mbar_wait(bar(B_QF + t % kStages), (t / kStages) & 1, nullptr, prm.err);
+      if (*abort_flag) {
+        for (int t = (issued_q > kQStages ? issued_q - kQStages : 0); t < issued_q; ++t)
+          mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, nullptr, prm.err);
+        for (int t = (issued_o > kOStages ? issued_o - kOStages : 0); t < issued_o; ++t)
+          mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, nullptr, prm.err);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && T > 0) {
       bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
       const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
-      const uint64_t dPT = sdesc_sw128(sb + kOffPT, 16, 1024);
-      auto stage_ready = [&](int t) -> bool {
-        const bool r = mbar_wait(bar(B_QF + t % kStages), (t / kStages) & 1, abort_flag, prm.err);
+      auto q_ready = [&](int t) -> bool {
+        const bool r = mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, abort_flag, prm.err);
         tc_fence_after();
         return r;
       };
-      // S^T = K Q_t^T (N = 128 query rows)
+      auto o_ready = [&](int t) -> bool {
+        const bool r = mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, abort_flag, prm.err);
+        tc_fence_after();
+        return r;
+      };
+      // S^T = K Q_t^T
       auto issue_s = [&](int t) {
-        const uint64_t dQ = sdesc_sw128(sb + kOffStage + (t % kStages) * 2 * kTile, 16, 1024);
+        const uint64_t dQ = sdesc_sw128(sb + kOffQ + (t % kQStages) * kTile, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -245,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // dP^T = V dO_t^T
       auto issue_dp = [&](int t) {
-        const uint64_t dO = sdesc_sw128(sb + kOffStage + (t % kStages) * 2 * kTile + kTile, 16, 1024);
+        const uint64_t dO = sdesc_sw128(sb + kOffO + (t % kOStages) * kTile, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -253,44 +264,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(B_DPF));
       };
-      if (ok) ok = stage_ready(0);
-      if (ok) {
-        issue_s(0);
-        issue_dp(0);
-      }
+      if (ok) ok = q_ready(0);
+      if (ok) issue_s(0);
+      if (ok) ok = o_ready(0);
+      if (ok) issue_dp(0);
       for (int t = 0; ok && t < T; ++t) {
-        const int s = t % kStages;
-        const uint32_t st = sb + kOffStage + s * 2 * kTile;
-        // both warpgroups hold S^T_t in registers: issue S^T_{t+1}
-        if (t + 1 < T) {
-          ok = mbar_wait(bar(B_SR), t & 1, abort_flag, prm.err) && stage_ready(t + 1);
-          if (!ok) break;
-          issue_s(t + 1);
-        }
-        // dV += P^T dO_t: A = P^T (shared memory, K-major), B = dO tile MN-major over d
+        // dV += P^T dO_t: A from TMEM (query columns [0,64) in the S^T
+        // columns [0,32), [64,128) in [64,96)), B = dO tile MN-major over d
         ok = mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dOm = sdesc_sw128(st + kTile, 16384, 1024);
+        const uint64_t dOm = sdesc_sw128(sb + kOffO + (t % kOStages) * kTile, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kBQ / 16; ++kk)
-          mma_bf16_ss(tmem + kTdV, sdesc_add(dPT, (kk >> 2) * 16384 + (kk & 3) * 32),
-                      sdesc_add(dOm, kk * 2048), kIdescN128MN, (t > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_PE));
-        // dK += dS^T Q_t: A from TMEM (query columns [0,64) in the dP^T
-        // columns [0,32), [64,128) in [64,96)), B = Q tile MN-major over d
+        for (int kk = 0; kk < kBQ / 16; ++kk) {
+          const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+          mma_bf16_ts(tmem + kTdV, tmem + kTS + acol, sdesc_add(dOm, kk * 2048), kIdescN128MN,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        // the next tile's S^T over this tile's P^T (after the dV MMA in issue order)
+        if (t + 1 < T) {
+          ok = q_ready(t + 1);
+          if (!ok) break;
+          issue_s(t + 1);
+        }
+        // dK += dS^T Q_t: A from TMEM (dS^T over the dP^T columns), B = Q tile MN-major over d
         ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dQm = sdesc_sw128(st, 16384, 1024);
+        const uint64_t dQm = sdesc_sw128(sb + kOffQ + (t % kQStages) * kTile, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk) {
           const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
           mma_bf16_ts(tmem + kTdK, tmem + kTP + acol, sdesc_add(dQm, kk * 2048), kIdescN128MN,
                       (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(B_QE + s));
-        if (t + 1 < T) issue_dp(t + 1);
+        // both stages of tile t are free once dK is done (the compute
+        // warpgroups read the tile's LSE and D before they released dS^T)
+        tc_commit(bar(B_QE + t % kQStages));
+        tc_commit(bar(B_OE + t % kOStages));
+        if (t + 1 < T) {
+          ok = o_ready(t + 1);
+          if (!ok) break;
+          issue_dp(t + 1);
+        }
       }
       if (ok) tc_commit(bar(B_DONE));
       if (!ok) {
@@ -308,23 +324,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (j < g.n) prm.mk.col_range(j, lo_j, hi_j);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + kTS + 64 * w, tP = tmem + lane_off + kTP + 64 * w;
-    const uint32_t pt_base = sb + kOffPT;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ + 64 * w;  // this warpgroup's first query row
+      const int sq = t % kQStages, so = t % kOStages;
       // LSE log2(e) and D of this warpgroup's 64 query rows (loaded with Q / dO)
-      const float *lsm = reinterpret_cast<const float *>(smem + kOffStats + (t % kStages) * kStatBytes) + 64 * w;
-      const float *dsm = lsm + kBQ;
-      // phase a/b: P^T
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + t % kStages), (t / kStages) & 1, abort_flag, prm.err) &&
+      const float *lsm = reinterpret_cast<const float *>(smem + kOffLse + sq * kBQ * 4) + 64 * w;
+      const float *dsm = reinterpret_cast<const float *>(smem + kOffD + so * kBQ * 4) + 64 * w;
+      // phase a/b: P^T over this warpgroup's first 32 columns of S^T
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err) &&
                                        mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
       uint32_t r[64];
       tmem_ld64(tS, r);
-      tc_fence_before();
-      mbar_arrive(bar(B_SR));                  // the MMA thread may now overwrite S^T
       uint32_t pp[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
@@ -339,19 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         pp[c >> 1] = pack_bf16x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
       }
-      // the previous tile's P^T must have been consumed by its dV MMA
-      if (t > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PE), (t - 1) & 1, abort_flag, prm.err));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        st_shared_v4(pt_base + sw128_offset(row, 8 * w + u), pp[4 * u], pp[4 * u + 1], pp[4 * u + 2],
-                     pp[4 * u + 3]);
-      fence_proxy_async_smem();
+      tmem_st32_nowait(tS, pp);
+      tmem_st_wait();
+      tc_fence_before();
       mbar_arrive(bar(B_PS));
-      // phase c: dS^T
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err));
+      // phase c: dS^T over this warpgroup's first 32 columns of dP^T
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + so), (t / kOStages) & 1, abort_flag, prm.err) &&
+                                       mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
       uint32_t dp[64];
@@ -363,7 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float d1 = __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - dsm[c + 1]);
         dd[c >> 1] = pack_bf16x2(d0, d1);
       }
-      // dS^T (bf16 pairs) over this warpgroup's first 32 columns of dP^T
       tmem_st32_nowait(tP, dd);
       tmem_st_wait();
       tc_fence_before();
