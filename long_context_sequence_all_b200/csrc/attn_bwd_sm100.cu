@@ -21,8 +21,8 @@
 //  3. dQ kernel, query-stationary: a CTA owns 128 query rows of one head
 //     with Q and dO resident in TMEM, and streams K/V tiles of 128 keys:
 //       S = Q K^T, dP = dO V^T (M=128, N=128, K=128, A from TMEM)
-//       dQ += dS K             (M=128, N=128, K=128, dS through shared memory)
-//     The next tile's S, dP are issued while the current tile's dS is computed.
+//       dQ += dS K             (M=128, N=128, K=128, dS from TMEM)
+//     The next tile's S is issued as soon as the current S has been read.
 //
 // TMA loads with 128-byte swizzle feed shared memory; one thread issues all
 // MMAs; every wait is bounded (ULY_ERR_TIMEOUT).
@@ -419,19 +419,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One CTA = one 128-row query tile of one query head; Q and dO sit in TMEM
 // as the A operands of S = Q K^T and dP = dO V^T over K/V tiles of 128 keys
 // (all MMAs N=128).  The two compute warpgroups split each tile's key columns
-// (64 each).  As soon as both have copied S and dP into registers they
-// release the TMEM region, and the MMA thread issues the next tile's S and dP
-// while they compute dS; dS goes through shared memory to dQ += dS K.
+// (64 each).  A tile is processed in two phases:
+//   a. read S into registers (the S columns are then free and the next tile's
+//      S is issued), P = exp2(S scale log2e - LSE log2e)
+//   b. read dP, dS = P (dP - D), dS (bf16 pairs) over this warpgroup's own
+//      dP columns -> dQ += dS K (A from TMEM), then the next tile's dP.
+// TMEM: Q [0,64), dO [64,128) (bf16 pairs), dQ [128,256), S [256,384),
+// dP / dS [384,512).  The next dP overwrites the dS the dQ MMA reads, which
+// relies on tcgen05.mma executing in issue order.
 namespace qk {
 constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBK = 128;   // keys per K/V tile
 constexpr int kStages = 3;
 constexpr uint32_t kTile = 128 * 128 * 2;                  // one 128 x 128 bf16 tile
 constexpr uint32_t kOffKV = 0;                             // stage s: K at 2s*kTile, V at (2s+1)*kTile
-constexpr uint32_t kOffDS = kStages * 2 * kTile;           // dS [128 q][128 keys], K-major swizzled
-constexpr uint32_t kOffBar = kOffDS + kTile;
+constexpr uint32_t kOffBar = kStages * 2 * kTile;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-// TMEM columns: Q, dO (bf16 pairs), dQ (fp32), S, dP
 constexpr uint32_t kTQ = 0, kTO = 64, kTdQ = 128, kTS = 256, kTP = 384;
 }  // namespace qk
 
@@ -443,8 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  enum { B_KF = 0, B_KE = kStages, B_S = 2 * kStages, B_SR = B_S + 1, B_P = B_SR + 1, B_DSF = B_P + 1,
-         B_QO = B_DSF + 1, B_DQ = B_QO + 1, B_DRAIN = B_DQ + 1, B_N = B_DRAIN + 1 };
+  enum { B_KF = 0, B_KE = kStages, B_SF = 2 * kStages, B_SR, B_DPF, B_DS, B_QO, B_DQ, B_DRAIN, B_N };
+  static_assert(8 * B_N + 8 <= 256, "barrier area");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -464,11 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NT = (hi_last >= lo_first) ? hi_last / kBK - jt0 + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_N; ++i) {
-      uint32_t cnt = 1;
-      if (i == B_SR || i == B_P || i == B_QO) cnt = 256;
-      mbar_init(bar(i), cnt);
-    }
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_SR || i == B_DS || i == B_QO) ? 256 : 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmK);
@@ -483,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Registers: producer / MMA warpgroup 120 per thread, the two compute
-  // warpgroups 192 (a thread holds 64 columns of S and 64 of dP).
+  // warpgroups 192 (a thread holds 64 columns of P and 64 of dP).
 
   if (warp < 4) {
     setmaxnreg_dec<kRegsCtlQ>();
@@ -510,45 +509,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && NT > 0) {
         bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err);
         tc_fence_after();
-        // S = Q K_j^T, dP = dO V_j^T: A from TMEM, B = K / V tile (K-major), N = 128
-        auto issue_sdp = [&](int j) -> bool {
+        // S = Q K_j^T: A = Q from TMEM, B = K tile (K-major); waits for the K/V stage
+        auto issue_s = [&](int j) -> bool {
           const int s = j % kStages;
           if (!mbar_wait(bar(B_KF + s), (j / kStages) & 1, abort_flag, prm.err)) return false;
           tc_fence_after();
-          const uint32_t kst = sb + kOffKV + s * 2 * kTile;
-          const uint64_t dK = sdesc_sw128(kst, 16, 1024), dV = sdesc_sw128(kst + kTile, 16, 1024);
+          const uint64_t dK = sdesc_sw128(sb + kOffKV + s * 2 * kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk) {
-            const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ts(tmem + kTS, tmem + kTQ + kk * 8, sdesc_add(dK, ko), kIdescN128, kk > 0);
-            mma_bf16_ts(tmem + kTP, tmem + kTO + kk * 8, sdesc_add(dV, ko), kIdescN128, kk > 0);
-          }
-          tc_commit(bar(B_S));
+          for (int kk = 0; kk < kHD / 16; ++kk)
+            mma_bf16_ts(tmem + kTS, tmem + kTQ + kk * 8, sdesc_add(dK, (kk >> 2) * 16384 + (kk & 3) * 32),
+                        kIdescN128, kk > 0);
+          tc_commit(bar(B_SF));
           return true;
         };
-        const uint64_t dS = sdesc_sw128(sb + kOffDS, 16, 1024);
-        if (ok) ok = issue_sdp(0);
+        // dP = dO V_j^T: A = dO from TMEM, B = V tile (its stage already waited for by issue_s)
+        auto issue_dp = [&](int j) {
+          const uint64_t dV = sdesc_sw128(sb + kOffKV + (j % kStages) * 2 * kTile + kTile, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk)
+            mma_bf16_ts(tmem + kTP, tmem + kTO + kk * 8, sdesc_add(dV, (kk >> 2) * 16384 + (kk & 3) * 32),
+                        kIdescN128, kk > 0);
+          tc_commit(bar(B_DPF));
+        };
+        if (ok) ok = issue_s(0);
+        if (ok) issue_dp(0);
         for (int j = 0; ok && j < NT; ++j) {
           const int s = j % kStages;
-          // both warpgroups hold S_j and dP_j in registers: the region is free
+          // both warpgroups hold S_j in registers: the next tile's S
           ok = mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
           if (j + 1 < NT) {
-            ok = issue_sdp(j + 1);
+            ok = issue_s(j + 1);
             if (!ok) break;
           }
-          ok = mbar_wait(bar(B_P), j & 1, abort_flag, prm.err);
+          // dQ += dS K_j: A = dS from TMEM (key columns [0,64) in the dP
+          // columns [0,32), [64,128) in [64,96)), B = K tile MN-major over d
+          ok = mbar_wait(bar(B_DS), j & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          // dQ += dS K_j: A = dS (shared memory, K-major), B = K tile MN-major over d
           const uint64_t dKm = sdesc_sw128(sb + kOffKV + s * 2 * kTile, 16384, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ss(tmem + kTdQ, sdesc_add(dS, (kk >> 2) * 16384 + (kk & 3) * 32),
-                        sdesc_add(dKm, kk * 2048), kIdescN128MN, (j > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(B_DSF));
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+            mma_bf16_ts(tmem + kTdQ, tmem + kTP + acol, sdesc_add(dKm, kk * 2048), kIdescN128MN,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit(bar(B_KE + s));
+          if (j + 1 < NT) issue_dp(j + 1);
         }
         if (ok) tc_commit(bar(B_DQ));
         if (!ok) {
@@ -570,6 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float lse2 = valid ? prm.lse2[srow] : INFINITY;
     const float Di = valid ? prm.Dv[srow] : 0.f;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kTS + 64 * w, tP = tmem + lane_off + kTP + 64 * w;
     // warpgroup 0 puts this row of Q into TMEM, warpgroup 1 the row of dO
     {
       const __nv_bfloat16 *src = (w == 0) ? prm.q : prm.dout;
@@ -588,45 +597,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_QO));
     }
-    const uint32_t ds_base = sb + kOffDS;
     bool ok = true;
     for (int j = 0; j < NT; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S), j & 1, abort_flag, prm.err));
+      // phase a: P
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF), j & 1, abort_flag, prm.err));
       if (!ok) break;
       tc_fence_after();
-      uint32_t r[128];                         // r[0..63] S, r[64..127] dP of this warpgroup's keys
-      tmem_ld64x2(tmem + lane_off + kTS + 64 * w, tmem + lane_off + kTP + 64 * w, r);
+      uint32_t r[64];
+      tmem_ld64(tS, r);
       tc_fence_before();
-      mbar_arrive(bar(B_SR));                  // the MMA thread may now overwrite S and dP
+      mbar_arrive(bar(B_SR));                  // the MMA thread may now overwrite S
       const int n0 = (jt0 + j) * kBK + 64 * w;
       const bool full = (n0 >= lo_last) && (n0 + 63 <= hi_first) && (n0 + 64 <= g.n);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float pv = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lse2));
+        if (!full) {
+          const int jj = n0 + c;
+          if (jj < lo_i || jj > hi_i) pv = 0.f;
+        }
+        r[c] = __float_as_uint(pv);
+      }
+      // phase b: dS over this warpgroup's first 32 columns of dP
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), j & 1, abort_flag, prm.err));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dp[64];
+      tmem_ld64(tP, dp);
       uint32_t dd[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        float ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          float pv = ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lse2));
-          if (!full) {
-            const int jj = n0 + c + u;
-            if (jj < lo_i || jj > hi_i) pv = 0.f;
-          }
-          ds[u] = pv * (__uint_as_float(r[64 + c + u]) - Di);
-        }
-        dd[c >> 1] = pack_bf16x2(ds[0], ds[1]);
+        const float d0 = __uint_as_float(r[c]) * (__uint_as_float(dp[c]) - Di);
+        const float d1 = __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - Di);
+        dd[c >> 1] = pack_bf16x2(d0, d1);
       }
-      // dS of the previous tile must have been consumed by its dQ MMA
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSF), (j - 1) & 1, abort_flag, prm.err));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        st_shared_v4(ds_base + sw128_offset(row, 8 * w + u), dd[4 * u], dd[4 * u + 1], dd[4 * u + 2],
-                     dd[4 * u + 3]);
-      fence_proxy_async_smem();
+      tmem_st32_nowait(tP, dd);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(B_P));
+      mbar_arrive(bar(B_DS));
     }
     // epilogue: warpgroup w writes dQ columns [64w, 64w + 64)
     if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, abort_flag, prm.err));
