@@ -268,10 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) issue_s(0);
       if (ok) ok = o_ready(0);
       if (ok) issue_dp(0);
+      // The dV group waits at one point for P^T and the next Q tile (fewer
+      // waits between MMA groups keep the tensor pipe busy).
       for (int t = 0; ok && t < T; ++t) {
+        const bool more = t + 1 < T;
         // dV += P^T dO_t: A from TMEM (query columns [0,64) in the S^T
         // columns [0,32), [64,128) in [64,96)), B = dO tile MN-major over d
-        ok = mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
+        ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + (t + 1) % kQStages), ((t + 1) / kQStages) & 1,
+                               abort_flag, prm.err)
+                  : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dOm = sdesc_sw128(sb + kOffO + (t % kOStages) * kTile, 16384, 1024);
@@ -282,11 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (t > 0 || kk > 0) ? 1u : 0u);
         }
         // the next tile's S^T over this tile's P^T (after the dV MMA in issue order)
-        if (t + 1 < T) {
-          ok = q_ready(t + 1);
-          if (!ok) break;
-          issue_s(t + 1);
-        }
+        if (more) issue_s(t + 1);
         // dK += dS^T Q_t: A from TMEM (dS^T over the dP^T columns), B = Q tile MN-major over d
         ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err);
         if (!ok) break;
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // warpgroups read the tile's LSE and D before they released dS^T)
         tc_commit(bar(B_QE + t % kQStages));
         tc_commit(bar(B_OE + t % kOStages));
-        if (t + 1 < T) {
+        if (more) {
           ok = o_ready(t + 1);
           if (!ok) break;
           issue_dp(t + 1);
@@ -509,18 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && NT > 0) {
         bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err);
         tc_fence_after();
-        // S = Q K_j^T: A = Q from TMEM, B = K tile (K-major); waits for the K/V stage
-        auto issue_s = [&](int j) -> bool {
-          const int s = j % kStages;
-          if (!mbar_wait(bar(B_KF + s), (j / kStages) & 1, abort_flag, prm.err)) return false;
-          tc_fence_after();
-          const uint64_t dK = sdesc_sw128(sb + kOffKV + s * 2 * kTile, 16, 1024);
+        // S = Q K_j^T: A = Q from TMEM, B = K tile (K-major); the caller has
+        // waited for the K/V stage
+        auto issue_s = [&](int j) {
+          const uint64_t dK = sdesc_sw128(sb + kOffKV + (j % kStages) * 2 * kTile, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk)
             mma_bf16_ts(tmem + kTS, tmem + kTQ + kk * 8, sdesc_add(dK, (kk >> 2) * 16384 + (kk & 3) * 32),
                         kIdescN128, kk > 0);
           tc_commit(bar(B_SF));
-          return true;
         };
         // dP = dO V_j^T: A = dO from TMEM, B = V tile (its stage already waited for by issue_s)
         auto issue_dp = [&](int j) {
@@ -531,18 +529,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         kIdescN128, kk > 0);
           tc_commit(bar(B_DPF));
         };
-        if (ok) ok = issue_s(0);
-        if (ok) issue_dp(0);
+        if (ok) ok = mbar_wait(bar(B_KF), 0, abort_flag, prm.err);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
+        }
         for (int j = 0; ok && j < NT; ++j) {
           const int s = j % kStages;
-          // both warpgroups hold S_j in registers: the next tile's S
-          ok = mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
+          // both warpgroups hold S_j in registers, and the next K/V stage has
+          // landed: the next tile's S (one wait point for both)
+          ok = (j + 1 < NT) ? mbar_wait2(bar(B_SR), j & 1, bar(B_KF + (j + 1) % kStages), ((j + 1) / kStages) & 1,
+                                         abort_flag, prm.err)
+                            : mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          if (j + 1 < NT) {
-            ok = issue_s(j + 1);
-            if (!ok) break;
-          }
+          if (j + 1 < NT) issue_s(j + 1);
           // dQ += dS K_j: A = dS from TMEM (key columns [0,64) in the dP
           // columns [0,32), [64,128) in [64,96)), B = K tile MN-major over d
           ok = mbar_wait(bar(B_DS), j & 1, abort_flag, prm.err);

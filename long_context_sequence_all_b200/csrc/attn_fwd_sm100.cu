@@ -173,13 +173,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int it = 0; ok && it < NT; ++it) {
         const int idxK = 2 * it, slotK = idxK % kSlots;
-        ok = mbar_wait(bar(B_KVF + slotK), (idxK / kSlots) & 1, abort_flag, prm.err);
-        if (!ok) break;
         const int idxV = 2 * (it - 1) + 1, slotV = (idxV + kSlots) % kSlots;
-        if (it > 0) {
-          ok = mbar_wait(bar(B_KVF + slotV), (idxV / kSlots) & 1, abort_flag, prm.err);
-          if (!ok) break;
-        }
+        ok = (it > 0) ? mbar_wait2(bar(B_KVF + slotK), (idxK / kSlots) & 1, bar(B_KVF + slotV), (idxV / kSlots) & 1,
+                                   abort_flag, prm.err)
+                      : mbar_wait(bar(B_KVF + slotK), (idxK / kSlots) & 1, abort_flag, prm.err);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t k_base = sb + kOffKV + slotK * kTileBytes;
         const uint32_t v_base = sb + kOffKV + slotV * kTileBytes;
