@@ -234,19 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && T > 0) {
       bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
       const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
-      auto q_ready = [&](int t) -> bool {
-        const bool r = mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, abort_flag, prm.err);
-        tc_fence_after();
-        return r;
-      };
-      auto o_ready = [&](int t) -> bool {
-        const bool r = mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, abort_flag, prm.err);
-        tc_fence_after();
-        return r;
-      };
-      // S^T = K Q_t^T
-      auto issue_s = [&](int t) {
-        const uint64_t dQ = sdesc_sw128(sb + kOffQ + (t % kQStages) * kTile, 16, 1024);
+      // S^T = K Q^T into the S^T columns; dP^T = V dO^T into the dP^T columns
+      auto issue_s = [&](uint64_t dQ) {
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -254,9 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(B_SF));
       };
-      // dP^T = V dO_t^T
-      auto issue_dp = [&](int t) {
-        const uint64_t dO = sdesc_sw128(sb + kOffO + (t % kOStages) * kTile, 16, 1024);
+      auto issue_dp = [&](uint64_t dO) {
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -264,22 +251,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(B_DPF));
       };
-      if (ok) ok = q_ready(0);
-      if (ok) issue_s(0);
-      if (ok) ok = o_ready(0);
-      if (ok) issue_dp(0);
-      // The dV group waits at one point for P^T and the next Q tile (fewer
-      // waits between MMA groups keep the tensor pipe busy).
+      if (ok) ok = mbar_wait2(bar(B_QF), 0, bar(B_OF), 0, abort_flag, prm.err);
+      if (ok) {
+        tc_fence_after();
+        issue_s(sdesc_sw128(sb + kOffQ, 16, 1024));
+        issue_dp(sdesc_sw128(sb + kOffO, 16, 1024));
+      }
+      // Stages and parities roll forward; every descriptor of an iteration
+      // is computed before its waits, so that nothing but the MMAs follows a
+      // completed wait (the issue queue is shallow, so any latency there idles
+      // the tensor pipe).  The dV group waits at one point for P^T and the
+      // next Q tile.
+      int sq = 0, so = 0;
+      uint32_t pq = 0, po = 0;
       for (int t = 0; ok && t < T; ++t) {
         const bool more = t + 1 < T;
+        const int sq1 = (sq + 1 == kQStages) ? 0 : sq + 1, so1 = (so + 1 == kOStages) ? 0 : so + 1;
+        const uint32_t pq1 = (sq1 == 0) ? (pq ^ 1u) : pq, po1 = (so1 == 0) ? (po ^ 1u) : po;
+        const uint64_t dOm = sdesc_sw128(sb + kOffO + so * kTile, 16384, 1024);   // dV: B = dO, MN-major
+        const uint64_t dQm = sdesc_sw128(sb + kOffQ + sq * kTile, 16384, 1024);   // dK: B = Q, MN-major
+        const uint64_t dQn = sdesc_sw128(sb + kOffQ + sq1 * kTile, 16, 1024);     // next S^T: B = next Q
+        const uint64_t dOn = sdesc_sw128(sb + kOffO + so1 * kTile, 16, 1024);     // next dP^T: B = next dO
         // dV += P^T dO_t: A from TMEM (query columns [0,64) in the S^T
-        // columns [0,32), [64,128) in [64,96)), B = dO tile MN-major over d
-        ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + (t + 1) % kQStages), ((t + 1) / kQStages) & 1,
-                               abort_flag, prm.err)
+        // columns [0,32), [64,128) in [64,96))
+        ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + sq1), pq1, abort_flag, prm.err)
                   : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dOm = sdesc_sw128(sb + kOffO + (t % kOStages) * kTile, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk) {
           const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -287,12 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (t > 0 || kk > 0) ? 1u : 0u);
         }
         // the next tile's S^T over this tile's P^T (after the dV MMA in issue order)
-        if (more) issue_s(t + 1);
-        // dK += dS^T Q_t: A from TMEM (dS^T over the dP^T columns), B = Q tile MN-major over d
+        if (more) issue_s(dQn);
+        // dK += dS^T Q_t: A from TMEM (dS^T over the dP^T columns)
         ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dQm = sdesc_sw128(sb + kOffQ + (t % kQStages) * kTile, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk) {
           const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -301,13 +298,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // both stages of tile t are free once dK is done (the compute
         // warpgroups read the tile's LSE and D before they released dS^T)
-        tc_commit(bar(B_QE + t % kQStages));
-        tc_commit(bar(B_OE + t % kOStages));
+        tc_commit(bar(B_QE + sq));
+        tc_commit(bar(B_OE + so));
         if (more) {
-          ok = o_ready(t + 1);
+          ok = mbar_wait(bar(B_OF + so1), po1, abort_flag, prm.err);
           if (!ok) break;
-          issue_dp(t + 1);
+          tc_fence_after();
+          issue_dp(dOn);
         }
+        sq = sq1; so = so1; pq = pq1; po = po1;
       }
       if (ok) tc_commit(bar(B_DONE));
       if (!ok) {
@@ -510,19 +509,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && NT > 0) {
         bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err);
         tc_fence_after();
-        // S = Q K_j^T: A = Q from TMEM, B = K tile (K-major); the caller has
-        // waited for the K/V stage
-        auto issue_s = [&](int j) {
-          const uint64_t dK = sdesc_sw128(sb + kOffKV + (j % kStages) * 2 * kTile, 16, 1024);
+        // S = Q K_j^T (A = Q from TMEM), dP = dO V_j^T (A = dO from TMEM); B tiles K-major
+        auto issue_s = [&](uint64_t dK) {
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk)
             mma_bf16_ts(tmem + kTS, tmem + kTQ + kk * 8, sdesc_add(dK, (kk >> 2) * 16384 + (kk & 3) * 32),
                         kIdescN128, kk > 0);
           tc_commit(bar(B_SF));
         };
-        // dP = dO V_j^T: A = dO from TMEM, B = V tile (its stage already waited for by issue_s)
-        auto issue_dp = [&](int j) {
-          const uint64_t dV = sdesc_sw128(sb + kOffKV + (j % kStages) * 2 * kTile + kTile, 16, 1024);
+        auto issue_dp = [&](uint64_t dV) {
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk)
             mma_bf16_ts(tmem + kTP, tmem + kTO + kk * 8, sdesc_add(dV, (kk >> 2) * 16384 + (kk & 3) * 32),
@@ -532,25 +527,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = mbar_wait(bar(B_KF), 0, abort_flag, prm.err);
         if (ok) {
           tc_fence_after();
-          issue_s(0);
-          issue_dp(0);
+          issue_s(sdesc_sw128(sb + kOffKV, 16, 1024));
+          issue_dp(sdesc_sw128(sb + kOffKV + kTile, 16, 1024));
         }
+        // Stages and parities roll forward; every descriptor of an iteration
+        // is computed before its waits (nothing but MMAs right after a wait).
+        int s = 0;
+        uint32_t ps = 0;
         for (int j = 0; ok && j < NT; ++j) {
-          const int s = j % kStages;
+          const bool more = j + 1 < NT;
+          const int s1 = (s + 1 == kStages) ? 0 : s + 1;
+          const uint32_t ps1 = (s1 == 0) ? (ps ^ 1u) : ps;
+          const uint32_t st = sb + kOffKV + s * 2 * kTile, st1 = sb + kOffKV + s1 * 2 * kTile;
+          const uint64_t dKn = sdesc_sw128(st1, 16, 1024), dVn = sdesc_sw128(st1 + kTile, 16, 1024);
+          const uint64_t dKm = sdesc_sw128(st, 16384, 1024);   // dQ: B = K tile, MN-major over d
           // both warpgroups hold S_j in registers, and the next K/V stage has
           // landed: the next tile's S (one wait point for both)
-          ok = (j + 1 < NT) ? mbar_wait2(bar(B_SR), j & 1, bar(B_KF + (j + 1) % kStages), ((j + 1) / kStages) & 1,
-                                         abort_flag, prm.err)
-                            : mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
+          ok = more ? mbar_wait2(bar(B_SR), j & 1, bar(B_KF + s1), ps1, abort_flag, prm.err)
+                    : mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          if (j + 1 < NT) issue_s(j + 1);
+          if (more) issue_s(dKn);
           // dQ += dS K_j: A = dS from TMEM (key columns [0,64) in the dP
-          // columns [0,32), [64,128) in [64,96)), B = K tile MN-major over d
+          // columns [0,32), [64,128) in [64,96))
           ok = mbar_wait(bar(B_DS), j & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t dKm = sdesc_sw128(sb + kOffKV + s * 2 * kTile, 16384, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -558,7 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (j > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(bar(B_KE + s));
-          if (j + 1 < NT) issue_dp(j + 1);
+          if (more) issue_dp(dVn);
+          s = s1;
+          ps = ps1;
         }
         if (ok) tc_commit(bar(B_DQ));
         if (!ok) {

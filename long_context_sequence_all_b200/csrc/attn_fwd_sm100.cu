@@ -155,15 +155,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors of the fixed operands; per-k-step offsets are constants
       const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
       const uint64_t dq1 = sdesc_sw128(sb + kOffQ + kTileBytes, 16, 1024);
-      auto issue_pv = [&](int t, uint32_t v_base, bool first) {
-        const uint64_t dv = sdesc_sw128(v_base, 16384, 1024);   // V: MN-major
+      auto issue_pv = [&](int t, uint64_t dv, bool first) {   // dv: V tile, MN-major
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, sdesc_add(dv, kk * 2048), kIdescPV,
                       (!first || kk > 0) ? 1u : 0u);
       };
-      auto issue_s = [&](int t, uint32_t k_base) {
-        const uint64_t dk = sdesc_sw128(k_base, 16, 1024);
+      auto issue_s = [&](int t, uint64_t dk) {
         const uint64_t dq = t ? dq1 : dq0;
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
@@ -171,40 +169,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ss(tmem + t * 128, sdesc_add(dq, koff), sdesc_add(dk, koff), kIdescS, kk > 0 ? 1u : 0u);
         }
       };
+      // K/V slots and their phases roll forward (K of tile it at ring index
+      // 2 it, V at 2 it + 1); descriptors are computed before the waits so
+      // that nothing but MMAs follows a completed wait.
+      int slotK = 0, slotV = kSlots - 1;
+      uint32_t parK = 0, parV = 1;
       for (int it = 0; ok && it < NT; ++it) {
-        const int idxK = 2 * it, slotK = idxK % kSlots;
-        const int idxV = 2 * (it - 1) + 1, slotV = (idxV + kSlots) % kSlots;
-        ok = (it > 0) ? mbar_wait2(bar(B_KVF + slotK), (idxK / kSlots) & 1, bar(B_KVF + slotV), (idxV / kSlots) & 1,
-                                   abort_flag, prm.err)
-                      : mbar_wait(bar(B_KVF + slotK), (idxK / kSlots) & 1, abort_flag, prm.err);
+        const uint64_t dk = sdesc_sw128(sb + kOffKV + slotK * kTileBytes, 16, 1024);
+        const uint64_t dv = sdesc_sw128(sb + kOffKV + slotV * kTileBytes, 16384, 1024);   // V: MN-major
+        ok = (it > 0) ? mbar_wait2(bar(B_KVF + slotK), parK, bar(B_KVF + slotV), parV, abort_flag, prm.err)
+                      : mbar_wait(bar(B_KVF + slotK), parK, abort_flag, prm.err);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t k_base = sb + kOffKV + slotK * kTileBytes;
-        const uint32_t v_base = sb + kOffKV + slotV * kTileBytes;
         for (int t = 0; t < 2 && ok; ++t) {
           if (it > 0) {
             ok = mbar_wait(bar(B_PF + t), (it - 1) & 1, abort_flag, prm.err);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(t, v_base, it == 1);
+            issue_pv(t, dv, it == 1);
           }
-          issue_s(t, k_base);
+          issue_s(t, dk);
           tc_commit(bar(B_SF + t));
         }
         if (!ok) break;
         tc_commit(bar(B_KVE + slotK));
         if (it > 0) tc_commit(bar(B_KVE + slotV));
+        slotK += 2;
+        if (slotK >= kSlots) { slotK -= kSlots; parK ^= 1u; }
+        slotV += 2;
+        if (slotV >= kSlots) { slotV -= kSlots; parV ^= 1u; }
       }
       if (ok) {
-        const int idxV = 2 * (NT - 1) + 1, slotV = idxV % kSlots;
-        ok = mbar_wait(bar(B_KVF + slotV), (idxV / kSlots) & 1, abort_flag, prm.err);
+        // the last tile's V (ring index 2 NT - 1: where slotV has rolled to)
+        const uint64_t dv = sdesc_sw128(sb + kOffKV + slotV * kTileBytes, 16384, 1024);
+        ok = mbar_wait(bar(B_KVF + slotV), parV, abort_flag, prm.err);
         tc_fence_after();
-        const uint32_t v_base = sb + kOffKV + slotV * kTileBytes;
         for (int t = 0; t < 2 && ok; ++t) {
           ok = mbar_wait(bar(B_PF + t), (NT - 1) & 1, abort_flag, prm.err);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, v_base, NT == 1);
+          issue_pv(t, dv, NT == 1);
           tc_commit(bar(B_OF + t));
         }
         if (ok) tc_commit(bar(B_KVE + slotV));
