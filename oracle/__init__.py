@@ -59,6 +59,8 @@ def _load():
             lib.oracle_head_rows_step.argtypes = [i, i, i, P, i, dbl, P, P, P, P, P, i, P, P, P, P, P]
             lib.oracle_loss.argtypes = [i, l, i, P, P, i, P, P, P]
             lib.oracle_loss.restype = l
+            lib.oracle_loss_grad.argtypes = [l, i, P, P, i, P]
+            lib.oracle_loss_grad.restype = ctypes.c_longlong
             _lib = lib
     return _lib
 
@@ -249,3 +251,14 @@ def loss_aggregate(logits, labels, P, ignore_index=-100):
     L = np.empty(1, np.float64)
     bad = _load().oracle_loss(P, T, V, _ptr(z), _ptr(y), ignore_index, _ptr(S), _ptr(C), _ptr(L))
     return S, C, float(L[0]), int(bad)
+
+
+def loss_grad(logits, labels, ignore_index=-100):
+    """dL/dlogits of the aggregated loss L = sum S_r / sum C_r: logits [T][V],
+    labels [T] -> (dlogits [T][V] fp64, global count C)."""
+    z = _f32(logits)
+    T, V = z.shape
+    y = np.ascontiguousarray(labels, dtype=np.int32)
+    g = np.empty((T, V), np.float64)
+    C = _load().oracle_loss_grad(T, V, _ptr(z), _ptr(y), ignore_index, _ptr(g))
+    return g, int(C)

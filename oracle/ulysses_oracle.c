@@ -626,3 +626,40 @@ long oracle_loss(int P, long T, int V, const float *logits, const int *labels,
   *loss = Ssum / (double)Csum;
   return bad;
 }
+
+/*
+ * Gradient of the aggregated loss with respect to the logits -- the step that
+ * follows the aggregation in training.  L = sum_r S_r / sum_r C_r has one
+ * denominator for every shard, the global count C = sum_r C_r
+ * [P3 "Integrarea cu Accelerate": the loss is weighted by the tokens each rank
+ * holds], so for a counted token t:
+ *     dL/dz_tv = (softmax(z_t)_v - [v == y_t]) / C,
+ * and dL/dz_tv = 0 for an ignored or invalid token.  softmax in fp64 with the
+ * maximum subtracted.  logits [T][V] (the shards stacked), labels [T]; writes
+ * dlogits [T][V] (fp64) and returns C.  With C = 0 every row is 0.
+ */
+long long oracle_loss_grad(long T, int V, const float *logits, const int *labels, int ignore_index,
+                           double *dlogits) {
+  long long C = 0;
+  for (long t = 0; t < T; ++t) {
+    const int y = labels[t];
+    if (y != ignore_index && y >= 0 && y < V) ++C;
+  }
+#pragma omp parallel for schedule(static)
+  for (long t = 0; t < T; ++t) {
+    double *g = dlogits + (size_t)t * V;
+    const int y = labels[t];
+    if (C == 0 || y == ignore_index || y < 0 || y >= V) {
+      for (int e = 0; e < V; ++e) g[e] = 0.0;
+      continue;
+    }
+    const float *z = logits + (size_t)t * V;
+    double m = -INFINITY;
+    for (int e = 0; e < V; ++e) if ((double)z[e] > m) m = (double)z[e];
+    double acc = 0.0;
+    for (int e = 0; e < V; ++e) acc += exp((double)z[e] - m);
+    for (int e = 0; e < V; ++e) g[e] = exp((double)z[e] - m) / acc / (double)C;
+    g[y] -= 1.0 / (double)C;
+  }
+  return C;
+}

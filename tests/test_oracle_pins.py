@@ -423,6 +423,70 @@ def test_loss_edge_cases():
     assert math.isfinite(L) and abs(L - _ce_ref(z2, y2)) < 1e-9 * max(1, abs(L))
 
 
+def test_loss_grad_equals_torch_autograd():
+    """dL/dz of the aggregated loss equals torch's float64 autograd gradient of
+    the unsharded mean cross-entropy (ignore_index -100): one global count."""
+    T, V = 48, 77
+    z = _randn(T, V, scale=2.0)
+    y = rng.integers(0, V, T).astype(np.int32)
+    y[rng.random(T) < 0.25] = -100
+    g, C = oracle.loss_grad(z, y)
+    zt = torch.tensor(z, dtype=torch.float64, requires_grad=True)
+    F.cross_entropy(zt, torch.tensor(y, dtype=torch.int64), ignore_index=-100, reduction="mean").backward()
+    assert C == int((y != -100).sum())
+    assert np.abs(g - zt.grad.numpy()).max() < 1e-15
+
+
+def test_loss_grad_finite_differences():
+    """Central differences of the oracle's own aggregated loss (P shards, one
+    shard without valid tokens) match dL/dz at label and non-label entries."""
+    T, V, P = 24, 40, 4
+    z = _randn(T, V)
+    y = rng.integers(0, V, T).astype(np.int32)
+    y[: T // P] = -100
+    y[rng.random(T) < 0.2] = -100
+    g, C = oracle.loss_grad(z, y)
+    h = np.float32(1.0 / 256)   # a power of two: z +- h is exact in float32
+    picks = [(t, int(y[t])) for t in range(T) if y[t] >= 0][:6]
+    picks += [(int(rng.integers(0, T)), int(rng.integers(0, V))) for _ in range(20)]
+    for t, v in picks:
+        zp, zm = z.copy(), z.copy()
+        zp[t, v] += h
+        zm[t, v] -= h
+        Lp = oracle.loss_aggregate(zp, y, P)[2]
+        Lm = oracle.loss_aggregate(zm, y, P)[2]
+        fd = (Lp - Lm) / (float(zp[t, v]) - float(zm[t, v]))
+        assert abs(fd - g[t, v]) < 1e-6, (t, v, fd, g[t, v])
+
+
+def test_loss_grad_closed_forms_and_invariants():
+    T, V = 32, 64
+    z = _randn(T, V, scale=3.0)
+    y = rng.integers(0, V, T).astype(np.int32)
+    y[::4] = -100
+    y[5], y[6] = V, -7               # invalid labels: not counted, zero rows
+    g, C = oracle.loss_grad(z, y)
+    counted = (y >= 0) & (y < V)
+    assert C == int(counted.sum())
+    # softmax sums to one: every counted row of dL/dz sums to zero
+    assert np.abs(g[counted].sum(axis=1)).max() < 1e-15
+    assert not g[~counted].any()
+    # the label entry is the only negative one: (p_y - 1) / C < 0 < p_v / C
+    for t in np.flatnonzero(counted):
+        assert g[t, y[t]] < 0 and (np.delete(g[t], y[t]) > 0).all()
+    # uniform logits: (1/V - [v == y]) / C exactly
+    zu = np.full((T, V), -1.25, np.float32)
+    gu, Cu = oracle.loss_grad(zu, y)
+    ref = np.zeros((T, V))
+    for t in np.flatnonzero(counted):
+        ref[t] = 1.0 / V / Cu
+        ref[t, y[t]] -= 1.0 / Cu
+    assert np.abs(gu - ref).max() < 1e-16
+    # nothing counted: all zero (no NaN)
+    g0, C0 = oracle.loss_grad(z, np.full(T, -100, np.int32))
+    assert C0 == 0 and not g0.any()
+
+
 def test_pages_loss_parity_bound_is_met_by_sharding():
     """The pages report SP and DP losses within 1e-5 of each other; with exact
     token weighting the oracle's sharded loss equals the unsharded mean to
