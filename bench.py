@@ -121,6 +121,16 @@ class Layer:
             self.C = torch.empty(P, dtype=torch.int64, device=dev)
             self.L = torch.empty(1, dtype=torch.float32, device=dev)
             self.lws = torch.empty(max(256, U.ulysses_loss_workspace_size(P, T, V)), dtype=torch.uint8, device=dev)
+            self.dlogits = torch.empty_like(self.logits)
+            self.lbws = torch.empty(max(256, U.ulysses_loss_bwd_workspace_size(P, T, V)), dtype=torch.uint8,
+                                    device=dev)
+
+    def loss_bwd(self):
+        """The loss with its gradient dL/dlogits (the step after the layer's
+        loss in training; measured on its own, not part of the layer step)."""
+        self.U.ulysses_loss_aggregate_bwd(self.logits, self.labels, self.P, dlogits=self.dlogits,
+                                          shard_sum=self.S, shard_count=self.C, loss=self.L,
+                                          workspace=self.lbws)
 
     def step(self):
         U, P = self.U, self.P
@@ -300,6 +310,27 @@ def run_ours(args, rank, world, dev):
     _barrier(world)
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
 
+    # the fused loss + gradient, timed on its own (it follows the layer's loss
+    # in training and is not part of the layer step)
+    loss_bwd = None
+    if layer.logits is not None:
+        layer.loss_bwd()
+        torch.cuda.synchronize()
+        U.ulysses_profile_enable(True)
+        for _ in range(args.steps):
+            layer.loss_bwd()
+        torch.cuda.synchronize()
+        lprof = U.ulysses_profile_read()
+        U.ulysses_profile_enable(False)
+        if "loss_fwd_bwd" in lprof:
+            tot, cnt = lprof["loss_fwd_bwd"]
+            T, V = layer.logits.shape
+            nbytes = 2.0 * T * V * layer.logits.element_size() + 2.0 * T * 4
+            loss_bwd = {"ms_per_launch": tot / cnt, "gbs": nbytes / (tot / cnt / 1e3) / 1e9,
+                        "note": "logits read once, dlogits written once; timed outside the layer step"}
+        if U.ulysses_read_error():
+            raise RuntimeError("device error word set by the loss gradient")
+
     tokens = inp["B"] * inp["n"]
     value = job_throughput(tokens, world, ms_max)
     peaks, peak_src = load_peaks()
@@ -320,6 +351,8 @@ def run_ours(args, rank, world, dev):
                 k["gbs"] = amount / (tot_ms / args.steps / 1e3) / 1e9
                 k["frac_hbm"] = k["gbs"] / peaks["hbm_gbs"]
         kernels[name] = k
+    if loss_bwd is not None:
+        loss_bwd["frac_hbm"] = loss_bwd["gbs"] / peaks["hbm_gbs"]
     dominant = max(kernels, key=lambda n: kernels[n]["ms_per_step"])
     dk = kernels[dominant]
     kind, amount = work.get(dominant, ("flops", float("nan")))
@@ -360,6 +393,7 @@ def run_ours(args, rank, world, dev):
         "permute_gbs": {k: kernels[k]["gbs"] for k in ("seq_to_head", "head_to_seq") if k in kernels},
         "roofline": roof,
         "kernels": kernels,
+        "loss_grad": loss_bwd,
         "gpu_launches": launches,
         "e2e": {"value": job_throughput(tokens, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": io.h2d, "d2h_bytes_per_step": io.d2h},

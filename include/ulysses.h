@@ -148,6 +148,31 @@ uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab,
                                   float *shard_sum, int64_t *shard_count, float *loss,
                                   void *workspace, size_t workspace_bytes, void *stream);
 
+/* Bytes of device workspace ulysses_loss_aggregate_bwd needs. */
+uly_status ulysses_loss_bwd_workspace_size(int32_t world, int64_t tokens, int32_t vocab,
+                                           size_t *bytes);
+
+/*
+ * The aggregated loss and its gradient in one pass over the logits (the
+ * training step after the aggregation; "Integrarea cu Accelerate": every
+ * shard's loss is weighted by its valid-token count, so the gradient of
+ * L = sum_r S_r / sum_r C_r has the global count C = sum_r C_r as its only
+ * denominator):
+ *   dlogits[t][v] = (softmax(z_t)_v - [v == y_t]) / C  for counted tokens,
+ *   dlogits[t][v] = 0                                   for ignored or invalid ones.
+ * shard_sum, shard_count and *loss as ulysses_loss_aggregate (bitwise the same
+ * values).  dlogits: same shape and dtype as logits, written in full; it must
+ * not overlap any other argument.  Logits are read once from HBM and dlogits
+ * written once.  Errors as ulysses_loss_aggregate; with no counted token
+ * every dlogits row is 0 and *loss is NaN.
+ */
+uly_status ulysses_loss_aggregate_bwd(int32_t world, int64_t tokens, int32_t vocab,
+                                      int32_t logit_dtype, const void *logits,
+                                      const int32_t *labels, int32_t ignore_index,
+                                      void *dlogits, float *shard_sum, int64_t *shard_count,
+                                      float *loss, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
 /* Size of the fixed scratch array behind ulysses_loss_aggregate_noalloc. */
 #define ULYSSES_NOALLOC_LOSS_SCRATCH_BYTES 65536
 

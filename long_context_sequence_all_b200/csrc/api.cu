@@ -52,6 +52,9 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *, const HeadGeom &, const M
                                 const float *, const void *, void *, void *, void *, float *,
                                 cudaStream_t);
 size_t loss_workspace_bytes(int P, long long per_shard);
+size_t loss_bwd_workspace_bytes(int P, long long per_shard);
+uly_status loss_bwd_launch(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *, int32_t,
+                           void *, float *, int64_t *, float *, void *, cudaStream_t);
 uly_status loss_validate(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *,
                          const float *, const int64_t *, const float *);
 uly_status loss_launch(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *, int32_t,
@@ -225,6 +228,40 @@ uly_status ulysses_loss_aggregate(int32_t world, int64_t tokens, int32_t vocab, 
       return ULY_ERR_ALIAS;
   return loss_launch(world, tokens, vocab, logit_dtype, logits, labels, ignore_index, shard_sum,
                      shard_count, loss, workspace, static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_loss_bwd_workspace_size(int32_t world, int64_t tokens, int32_t vocab, size_t *bytes) {
+  if (!bytes) return ULY_ERR_NULL;
+  if (world <= 0 || tokens < 0 || vocab <= 0 || tokens % world) return ULY_ERR_SHAPE;
+  *bytes = align256(loss_bwd_workspace_bytes(world, tokens / world));
+  return ULY_OK;
+}
+
+uly_status ulysses_loss_aggregate_bwd(int32_t world, int64_t tokens, int32_t vocab, int32_t logit_dtype,
+                                      const void *logits, const int32_t *labels, int32_t ignore_index,
+                                      void *dlogits, float *shard_sum, int64_t *shard_count, float *loss,
+                                      void *workspace, size_t workspace_bytes, void *stream) {
+  uly_status st = loss_validate(world, tokens, vocab, logit_dtype, logits, labels, shard_sum,
+                                shard_count, loss);
+  if (st != ULY_OK) return st;
+  if (!dlogits) return ULY_ERR_NULL;
+  if (!aligned16(dlogits)) return ULY_ERR_ALIGN;
+  size_t need = 0;
+  ulysses_loss_bwd_workspace_size(world, tokens, vocab, &need);
+  if (!workspace || workspace_bytes < need) return ULY_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ULY_ERR_ALIGN;
+  const size_t zb = (size_t)tokens * vocab * (logit_dtype == ULY_BF16 ? 2 : 4);
+  const size_t yb = (size_t)tokens * 4;
+  const void *outs[5] = {dlogits, shard_sum, shard_count, loss, workspace};
+  const size_t outb[5] = {zb, (size_t)world * 4, (size_t)world * 8, 4, need};
+  for (int a = 0; a < 5; ++a) {
+    if (overlap(outs[a], outb[a], logits, zb) || overlap(outs[a], outb[a], labels, yb))
+      return ULY_ERR_ALIAS;
+    for (int b = a + 1; b < 5; ++b)
+      if (overlap(outs[a], outb[a], outs[b], outb[b])) return ULY_ERR_ALIAS;
+  }
+  return loss_bwd_launch(world, tokens, vocab, logit_dtype, logits, labels, ignore_index, dlogits,
+                         shard_sum, shard_count, loss, workspace, static_cast<cudaStream_t>(stream));
 }
 
 uly_status ulysses_read_error_info(int32_t *info, int32_t n) {

@@ -13,6 +13,14 @@
 // its shard into the workspace.  Pass 2: one CTA per launch folds the
 // partials in a fixed order (deterministic) into S_r, C_r and L.
 // HBM-bound: each logits byte is read once.
+//
+// The gradient (the training step after the aggregation) has the global
+// count C = sum_r C_r as its only denominator:
+//   dL/dz_tv = (softmax(z_t)_v - [v == y_t]) / C   (counted tokens; else 0)
+// The fused forward+backward counts the valid labels first (one CTA, labels
+// only), then each token's warp computes the row's logsumexp exactly as the
+// forward does, re-reads the row (now in L2) and writes dL/dz with 16-byte
+// stores: logits read once from HBM, dlogits written once.
 #include "common.cuh"
 #include "prof.cuh"
 
@@ -55,16 +63,57 @@ __device__ __forceinline__ void load_vals<float>(const uint4 &u, float (&x)[8]) 
   x[4] = x[5] = x[6] = x[7] = -INFINITY;
 }
 
+// log sum_v exp(z_v) of one row, computed by the 32 lanes of a warp (every
+// lane returns it).  STREAM: evict-first loads (the row is not read again).
+template <typename T, bool STREAM>
+__device__ __forceinline__ float row_lse(const T *rowp, int vocab, int lane) {
+  constexpr int kPerVec = 16 / sizeof(T);
+  const int vecs = vocab / kPerVec;  // vocab * sizeof(T) % 16 == 0 checked on the host
+  const uint4 *row = reinterpret_cast<const uint4 *>(rowp);
+  float m = -INFINITY, s = 0.f;
+  for (int v0 = lane; v0 < vecs; v0 += 32 * kLoadsInFlight) {
+    uint4 u[kLoadsInFlight];
+#pragma unroll
+    for (int k = 0; k < kLoadsInFlight; ++k) {
+      const int v = v0 + k * 32;
+      if (v < vecs) u[k] = STREAM ? __ldcs(row + v) : __ldg(row + v);
+    }
+#pragma unroll
+    for (int k = 0; k < kLoadsInFlight; ++k) {
+      const int v = v0 + k * 32;
+      if (v < vecs) {
+        float x[8];
+        load_vals<T>(u[k], x);
+        float mx = x[0];
+#pragma unroll
+        for (int e = 1; e < 8; ++e) mx = fmaxf(mx, x[e]);
+        if (mx > m) {
+          s = (m == -INFINITY) ? 0.f : s * exp2f((m - mx) * kLog2e);
+          m = mx;
+        }
+        const float ml = m * kLog2e;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += exp2f(fmaf(x[e], kLog2e, -ml));
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+    merge(m, s, m2, s2);
+  }
+  return m + logf(s);
+}
+
 // grid = (blocks_per_shard, P).  Partials: part_sum[r * nb + blockIdx.x], part_cnt[...].
 template <typename T>
 __global__ void __launch_bounds__(kThreads) ce_partial_kernel(
     const T *__restrict__ logits, const int32_t *__restrict__ labels, long long per_shard,
     int vocab, int ignore_index, double *__restrict__ part_sum, long long *__restrict__ part_cnt,
     int *err) {
-  constexpr int kPerVec = 16 / sizeof(T);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.y, nb = gridDim.x;
-  const int vecs = vocab / kPerVec;  // vocab * sizeof(T) % 16 == 0 checked on the host
   double acc = 0.0;
   long long cnt = 0;
   for (long long tt = (long long)blockIdx.x * kWarps + warp; tt < per_shard;
@@ -76,45 +125,108 @@ __global__ void __launch_bounds__(kThreads) ce_partial_kernel(
       if (lane == 0) raise_error(err, ULY_ERR_LABEL);
       continue;
     }
-    const uint4 *row = reinterpret_cast<const uint4 *>(logits + t * (long long)vocab);
-    float m = -INFINITY, s = 0.f;
-    for (int v0 = lane; v0 < vecs; v0 += 32 * kLoadsInFlight) {
-      uint4 u[kLoadsInFlight];
-#pragma unroll
-      for (int k = 0; k < kLoadsInFlight; ++k) {
-        const int v = v0 + k * 32;
-        if (v < vecs) u[k] = __ldcs(row + v);
-      }
-#pragma unroll
-      for (int k = 0; k < kLoadsInFlight; ++k) {
-        const int v = v0 + k * 32;
-        if (v < vecs) {
-          float x[8];
-          load_vals<T>(u[k], x);
-          float mx = x[0];
-#pragma unroll
-          for (int e = 1; e < 8; ++e) mx = fmaxf(mx, x[e]);
-          if (mx > m) {
-            s = (m == -INFINITY) ? 0.f : s * exp2f((m - mx) * kLog2e);
-            m = mx;
-          }
-          const float ml = m * kLog2e;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) s += exp2f(fmaf(x[e], kLog2e, -ml));
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
-      const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
-      merge(m, s, m2, s2);
-    }
+    const float lse = row_lse<T, true>(logits + t * (long long)vocab, vocab, lane);
     if (lane == 0) {
       const float zy = static_cast<float>(logits[t * (long long)vocab + y]);
-      const float lse = m + logf(s);
       acc += (double)lse - (double)zy;
       cnt += 1;
+    }
+  }
+  __shared__ double sh_sum[kWarps];
+  __shared__ long long sh_cnt[kWarps];
+  if (lane == 0) { sh_sum[warp] = acc; sh_cnt[warp] = cnt; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0;
+    long long c = 0;
+    for (int w = 0; w < kWarps; ++w) { a += sh_sum[w]; c += sh_cnt[w]; }  // fixed order
+    part_sum[(long long)r * nb + blockIdx.x] = a;
+    part_cnt[(long long)r * nb + blockIdx.x] = c;
+  }
+}
+
+// Global count of valid labels (not the ignore index, inside [0, V)): one
+// CTA, fixed-order reduction; written to *count.
+__global__ void __launch_bounds__(1024) ce_count_kernel(const int32_t *__restrict__ labels, long long tokens,
+                                                        int vocab, int ignore_index, long long *count) {
+  long long c = 0;
+  for (long long t = threadIdx.x; t < tokens; t += blockDim.x) {
+    const int y = __ldg(labels + t);
+    c += (y != ignore_index && y >= 0 && y < vocab) ? 1 : 0;
+  }
+  __shared__ long long sh[1024];
+  sh[threadIdx.x] = c;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *count = sh[0];
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 pack_vals(const float (&x)[8]);
+template <>
+__device__ __forceinline__ uint4 pack_vals<__nv_bfloat16>(const float (&x)[8]) {
+  uint4 u;
+  uint32_t *w = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t *>(&h);
+  }
+  return u;
+}
+template <>
+__device__ __forceinline__ uint4 pack_vals<float>(const float (&x)[8]) {
+  return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+}
+
+// Loss partials as ce_partial_kernel, and dL/dz for every token of the shard.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) ce_fwd_bwd_kernel(
+    const T *__restrict__ logits, const int32_t *__restrict__ labels, long long per_shard, int vocab,
+    int ignore_index, const long long *__restrict__ count, T *__restrict__ dlogits,
+    double *__restrict__ part_sum, long long *__restrict__ part_cnt, int *err) {
+  constexpr int kPerVec = 16 / sizeof(T);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y, nb = gridDim.x;
+  const int vecs = vocab / kPerVec;
+  const long long C = *count;
+  const float invC = C > 0 ? (float)(1.0 / (double)C) : 0.f;
+  double acc = 0.0;
+  long long cnt = 0;
+  for (long long tt = (long long)blockIdx.x * kWarps + warp; tt < per_shard;
+       tt += (long long)nb * kWarps) {
+    const long long t = (long long)r * per_shard + tt;
+    const int y = __ldg(labels + t);
+    uint4 *drow = reinterpret_cast<uint4 *>(dlogits + t * (long long)vocab);
+    const bool counted = y != ignore_index && y >= 0 && y < vocab;
+    if (!counted) {
+      if (y != ignore_index && lane == 0) raise_error(err, ULY_ERR_LABEL);
+      for (int v = lane; v < vecs; v += 32) __stcs(drow + v, make_uint4(0, 0, 0, 0));
+      continue;
+    }
+    const T *rowp = logits + t * (long long)vocab;
+    const float lse = row_lse<T, false>(rowp, vocab, lane);
+    if (lane == 0) {
+      acc += (double)lse - (double)static_cast<float>(rowp[y]);
+      cnt += 1;
+    }
+    // dL/dz = (exp(z - lse) - [v == y]) / C; the row is read again from L2
+    const float lse2 = lse * kLog2e;
+    const uint4 *row = reinterpret_cast<const uint4 *>(rowp);
+    for (int v = lane; v < vecs; v += 32) {
+      float x[8];
+      load_vals<T>(__ldg(row + v), x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int col = v * kPerVec + e;
+        float gv = exp2f(fmaf(x[e], kLog2e, -lse2)) * invC;
+        if (col == y) gv -= invC;
+        x[e] = gv;
+      }
+      __stcs(drow + v, pack_vals<T>(x));
     }
   }
   __shared__ double sh_sum[kWarps];
@@ -208,6 +320,39 @@ uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, 
   prof::Scope s2(prof::K_LOSS_FINALIZE, stream);
   ce_finalize_kernel<<<1, 256, 0, stream>>>(psum, pcnt, P, nb, shard_sum, shard_count, loss);
   note_launches(2);
+  return last_launch_status();
+}
+
+// Fused forward + backward.  `ws`: the forward's partials followed by one
+// long long (the global count of valid labels).
+size_t loss_bwd_workspace_bytes(int P, long long per_shard) {
+  return ((loss_workspace_bytes(P, per_shard) + 15) & ~size_t(15)) + 16;
+}
+
+uly_status loss_bwd_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, const void *logits,
+                           const int32_t *labels, int32_t ignore_index, void *dlogits, float *shard_sum,
+                           int64_t *shard_count, float *loss, void *ws, cudaStream_t stream) {
+  const long long per = tokens / P;
+  const int nb = loss_blocks_per_shard(P, per);
+  double *psum = static_cast<double *>(ws);
+  long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb * P);
+  long long *count = reinterpret_cast<long long *>(static_cast<char *>(ws) +
+                                                   ((loss_workspace_bytes(P, per) + 15) & ~size_t(15)));
+  dim3 grid(nb, P);
+  prof::Scope s1(prof::K_LOSS_FWD_BWD, stream);
+  ce_count_kernel<<<1, 1024, 0, stream>>>(labels, tokens, vocab, ignore_index, count);
+  if (dtype == ULY_BF16)
+    ce_fwd_bwd_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(logits), labels, per, vocab, ignore_index, count,
+        static_cast<__nv_bfloat16 *>(dlogits), psum, pcnt, error_word());
+  else
+    ce_fwd_bwd_kernel<float><<<grid, kThreads, 0, stream>>>(
+        static_cast<const float *>(logits), labels, per, vocab, ignore_index, count,
+        static_cast<float *>(dlogits), psum, pcnt, error_word());
+  s1.end();
+  prof::Scope s2(prof::K_LOSS_FINALIZE, stream);
+  ce_finalize_kernel<<<1, 256, 0, stream>>>(psum, pcnt, P, nb, shard_sum, shard_count, loss);
+  note_launches(3);
   return last_launch_status();
 }
 

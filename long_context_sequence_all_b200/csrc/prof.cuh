@@ -23,6 +23,7 @@ enum Kernel {
   K_ATTN_DKDV_SM100,
   K_ATTN_DQ_SM100,
   K_ATTN_BWD_STATS,
+  K_LOSS_FWD_BWD,
   K_COUNT
 };
 

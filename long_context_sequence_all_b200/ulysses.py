@@ -25,7 +25,8 @@ STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE"
           8: "ULY_ERR_LABEL", 9: "ULY_ERR_TIMEOUT", 10: "ULY_ERR_WORKSPACE"}
 EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
-           "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_read_error", "ulysses_read_error_info",
+           "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
+           "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info",
            "ulysses_status_string", "ulysses_profile_enable", "ulysses_profile_read",
            "ulysses_kernel_count", "ulysses_kernel_name",
            "ulysses_launch_count"]
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
             L.ulysses_loss_aggregate.argtypes = [i32, i64, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
             L.ulysses_loss_aggregate_noalloc.argtypes = [i32, i64, i32, i32, vp, vp, i32, vp, vp, vp, vp]
             L.ulysses_loss_aggregate_noalloc.restype = ctypes.c_int
+            L.ulysses_loss_bwd_workspace_size.argtypes = [i32, i64, i32, ctypes.POINTER(sz)]
+            L.ulysses_loss_aggregate_bwd.argtypes = [i32, i64, i32, i32, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
             L.ulysses_read_error.argtypes = [ctypes.POINTER(i32)]
             L.ulysses_read_error_info.argtypes = [ctypes.POINTER(i32), i32]
             L.ulysses_status_string.argtypes = [ctypes.c_int]
@@ -84,7 +87,8 @@ def lib() -> ctypes.CDLL:
             L.ulysses_kernel_name.restype = ctypes.c_char_p
             for name in ("ulysses_attn_fwd", "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd",
                          "ulysses_loss_workspace_size", "ulysses_loss_aggregate", "ulysses_read_error",
-                         "ulysses_read_error_info"):
+                         "ulysses_read_error_info", "ulysses_loss_bwd_workspace_size",
+                         "ulysses_loss_aggregate_bwd"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -218,6 +222,35 @@ def ulysses_loss_aggregate(logits, labels, P, ignore_index=-100, shard_sum=None,
                                         _p(workspace), workspace.numel(), _stream(stream)),
            "ulysses_loss_aggregate")
     return shard_sum, shard_count, loss
+
+
+def ulysses_loss_bwd_workspace_size(P: int, tokens: int, vocab: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ulysses_loss_bwd_workspace_size(P, tokens, vocab, ctypes.byref(n)),
+           "ulysses_loss_bwd_workspace_size")
+    return n.value
+
+
+def ulysses_loss_aggregate_bwd(logits, labels, P, ignore_index=-100, dlogits=None, shard_sum=None,
+                               shard_count=None, loss=None, workspace=None, stream=None):
+    """The aggregated loss and dL/dlogits in one pass: returns (shard_sum, shard_count,
+    loss, dlogits); dlogits has the shape and dtype of logits."""
+    T, V = logits.shape
+    dev = logits.device
+    dlogits = torch.empty_like(logits) if dlogits is None else dlogits
+    if dlogits.shape != logits.shape or dlogits.dtype != logits.dtype:
+        raise ValueError("dlogits must match logits in shape and dtype")
+    shard_sum = torch.empty(P, dtype=torch.float32, device=dev) if shard_sum is None else shard_sum
+    shard_count = torch.empty(P, dtype=torch.int64, device=dev) if shard_count is None else shard_count
+    loss = torch.empty(1, dtype=torch.float32, device=dev) if loss is None else loss
+    need = ulysses_loss_bwd_workspace_size(P, T, V)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib().ulysses_loss_aggregate_bwd(P, T, V, _dtype_code(logits), _p(logits), _p(labels),
+                                            ignore_index, _p(dlogits), _p(shard_sum), _p(shard_count),
+                                            _p(loss), _p(workspace), workspace.numel(), _stream(stream)),
+           "ulysses_loss_aggregate_bwd")
+    return shard_sum, shard_count, loss, dlogits
 
 
 def ulysses_loss_aggregate_noalloc(logits, labels, P, ignore_index=-100, shard_sum=None,

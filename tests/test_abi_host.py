@@ -99,3 +99,15 @@ def test_library_has_no_cpu_fallback_symbols():
     """The product binding never imports the oracle."""
     src = open(os.path.join(ROOT, "long_context_sequence_all_b200", "ulysses.py")).read()
     assert "oracle" not in src.replace("no fallback", "")
+
+
+def test_smoke_shape_passes_host_validation(L):
+    """The shape smoke() runs on the GPU is one the library accepts (H, G
+    divisible by P, H by G), so the round-end smoke cannot fail on validation."""
+    import __graft_entry__ as ge
+    from long_context_sequence_all_b200 import ulysses as U
+    P, n, H, G, d = ge.SMOKE_SHAPE
+    n_ws = ctypes.c_size_t(0)
+    desc = U.make_desc(1, n, P, H, G, d, U.ULY_BF16, U.MASK_CAUSAL)
+    assert L.ulysses_attn_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(n_ws)) == 0
+    assert L.ulysses_loss_bwd_workspace_size(P, 256, 8192, ctypes.byref(n_ws)) == 0
