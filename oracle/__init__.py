@@ -48,6 +48,9 @@ def _load():
             i, l, dbl = ctypes.c_int, ctypes.c_long, ctypes.c_double
             lib.oracle_seq_to_head.argtypes = [i, i, i, i, l, P, P]
             lib.oracle_head_to_seq.argtypes = [i, i, i, i, l, P, P]
+            lib.oracle_kv_replicate_to_head.argtypes = [i, i, i, i, l, P, P]
+            lib.oracle_kv_reduce_to_seq.argtypes = [i, i, i, i, i, P, P]
+            lib.oracle_shift_labels.argtypes = [i, i, i, P, P, i, i, i, P]
             attn = [i, i, i, i, i, i, P, i, dbl]
             lib.oracle_attention_fwd.argtypes = attn + [P, P, P, P, P]
             lib.oracle_attention_bwd.argtypes = attn + [P, P, P, P, P, P, P]
@@ -75,9 +78,12 @@ def _f32(a):
 
 def _check_ulysses(n, P, H, G):
     """Divisibility the method needs: n % P (every rank holds n/P positions),
-    H % P and G % P (every rank owns whole heads), H % G (GQA groups)."""
-    if P <= 0 or n % P or H % P or G % P or H % G:
-        raise ValueError(f"need n%P == H%P == G%P == H%G == 0, got n={n} P={P} H={H} G={G}")
+    H % P (every rank owns whole query heads), H % G (GQA groups), and either
+    G % P (every rank owns whole KV heads) or P % G (fewer KV heads than
+    ranks: every rank receives a copy of the one KV head it uses)."""
+    if P <= 0 or n % P or H % P or H % G or (G % P and P % G):
+        raise ValueError(f"need n%P == H%P == H%G == 0 and G%P == 0 or P%G == 0, "
+                         f"got n={n} P={P} H={H} G={G}")
 
 
 def _cu(cu_seqlens):
@@ -107,6 +113,39 @@ def head_to_seq(x: np.ndarray, B: int, n: int, P: int, heads: int) -> np.ndarray
     out = np.empty(P * B * (n // P) * heads * d, dtype=x.dtype)
     _load().oracle_head_to_seq(B, n, P, heads, d * x.itemsize, _ptr(x), _ptr(out))
     return out.reshape(P, B, n // P, heads, d)
+
+
+def kv_replicate_to_head(x: np.ndarray, B: int, n: int, P: int, G: int) -> np.ndarray:
+    """KV heads fewer than ranks (P % G == 0): seq layout [P][B][n/P][G][d] ->
+    [P][B][1][n][d], rank r receiving KV head floor(r*G/P) (any dtype, byte copy)."""
+    x = np.ascontiguousarray(x)
+    d = x.size // (B * n * G)
+    out = np.empty(P * B * n * d, dtype=x.dtype)
+    _load().oracle_kv_replicate_to_head(B, n, P, G, d * x.itemsize, _ptr(x), _ptr(out))
+    return out.reshape(P, B, 1, n, d)
+
+
+def kv_reduce_to_seq(x: np.ndarray, B: int, n: int, P: int, G: int) -> np.ndarray:
+    """Gradients of the replicated KV heads, [P][B][1][n][d] -> seq layout
+    [P][B][n/P][G][d] (fp64): each KV head's gradient is the sum over its copies."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    d = x.size // (P * B * n)
+    out = np.empty((P, B, n // P, G, d), np.float64)
+    _load().oracle_kv_reduce_to_seq(B, n, P, G, d, _ptr(x), _ptr(out))
+    return out
+
+
+def shift_labels(ids: np.ndarray, P: int, cu_seqlens=None, valid_len=None, ignore_index=-100):
+    """Next-token labels of ids [B][n], shifted before sharding: label(t) =
+    ids[t+1] unless t+1 >= valid_len or t+1 starts a packed document, then
+    ignore_index.  Returns the seq layout [P][B][n/P] (int32)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    B, n = ids.shape
+    cu, nd = _cu(cu_seqlens)
+    vl = n if valid_len is None else int(valid_len)
+    out = np.empty((P, B, n // P), np.int32)
+    _load().oracle_shift_labels(B, n, P, _ptr(ids), _ptr(cu), nd, vl, ignore_index, _ptr(out))
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -94,6 +94,90 @@ void oracle_head_to_seq(int B, int n, int P, int heads, long row_bytes,
           }
 }
 
+/*
+ * First all-to-all of K and V when there are fewer KV heads than ranks
+ * (G < P, P % G == 0).  The pages require at least as many heads as ranks
+ * ("Ulysses 序列平行化", section "與 Ring Attention 的比較": num_heads >=
+ * sp_size); with
+ * grouped-query attention that bound holds for the H query heads but not for
+ * the G KV heads, and the plain reading is that each KV head is sent whole to
+ * every rank whose query heads use it.  Rank r2 owns query heads
+ * [r2*H/P, (r2+1)*H/P), all of which use KV head floor(r2*G/P); it receives
+ * that one KV head for all n positions.  dst: [P][B][1][n][row].
+ */
+void oracle_kv_replicate_to_head(int B, int n, int P, int G, long row_bytes,
+                                 const void *src, void *dst) {
+  const int s = n / P;
+  for (int r = 0; r < P; ++r)          /* sending rank   */
+    for (int r2 = 0; r2 < P; ++r2) {   /* receiving rank */
+      const int k = r2 * G / P;        /* the KV head rank r2's query heads use */
+      for (int b = 0; b < B; ++b)
+        for (int tt = 0; tt < s; ++tt) {
+          size_t src_row = (((size_t)r * B + b) * s + tt) * G + (size_t)k;
+          size_t dst_row = ((size_t)r2 * B + b) * n + (size_t)r * s + tt;
+          memcpy((char *)dst + dst_row * row_bytes,
+                 (const char *)src + src_row * row_bytes, (size_t)row_bytes);
+        }
+    }
+}
+
+/*
+ * Second all-to-all of dK and dV for replicated KV heads: the gradient of a
+ * KV head is the sum of the gradients its copies received on every rank that
+ * held one (the copies are the same variable).  src: [P][B][1][n][d] (rank
+ * r2's copy of KV head floor(r2*G/P)), dst: seq layout [P][B][n/P][G][d];
+ * fp64, summed over the copies in rank order.
+ */
+void oracle_kv_reduce_to_seq(int B, int n, int P, int G, int d, const double *src,
+                             double *dst) {
+  const int s = n / P;
+  memset(dst, 0, sizeof(double) * (size_t)B * n * G * d);
+  for (int r2 = 0; r2 < P; ++r2) {     /* rank holding a copy */
+    const int k = r2 * G / P;
+    for (int r = 0; r < P; ++r)        /* rank owning the positions */
+      for (int b = 0; b < B; ++b)
+        for (int tt = 0; tt < s; ++tt) {
+          const double *x = src + (((size_t)r2 * B + b) * n + (size_t)r * s + tt) * d;
+          double *y = dst + ((((size_t)r * B + b) * s + tt) * G + (size_t)k) * d;
+          for (int e = 0; e < d; ++e) y[e] += x[e];
+        }
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Label shift for next-token prediction, before the sequence is sharded.     */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * The label of position t is the token at t+1 (next-token prediction), and the
+ * shift has to happen on the whole sequence, before it is split over ranks:
+ * the last position of shard r needs the first token of shard r+1 (the
+ * SFT trainer's automatic label shift: "Ulysses 序列平行化", section
+ * "在 Hugging Face 生態系統中的整合"; padding to a multiple of sp_size and
+ * variable-length packed sequences: "Paralelismul de Secvență Ulysses",
+ * section "Integrarea cu Transformers Trainer și TRL SFTTrainer").  A position
+ * gets ignore_index when t+1 is past the valid tokens (t+1 >= valid_len: the
+ * last token and the padding that makes n a multiple of P) or when t+1 starts
+ * a new packed document (t+1 is one of cu_seqlens[1..num_docs]).
+ * ids: [B][n] in sequence order; labels: seq layout [P][B][n/P].
+ */
+void oracle_shift_labels(int B, int n, int P, const int *ids, const int *cu_seqlens,
+                         int num_docs, int valid_len, int ignore_index, int *labels) {
+  const int s = n / P;
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < n; ++t) {
+      int y = ignore_index;
+      if (t + 1 < valid_len) {
+        int starts_doc = 0;
+        for (int e = 1; e <= num_docs; ++e)
+          if (cu_seqlens[e] == t + 1) starts_doc = 1;
+        if (!starts_doc) y = ids[(size_t)b * n + t + 1];
+      }
+      const int r = t / s, tt = t % s;
+      labels[((size_t)r * B + b) * s + tt] = y;
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Step 4: scaled-dot-product attention of one head, row by row.             */
 /* ------------------------------------------------------------------------- */
@@ -347,11 +431,21 @@ static float *to_head_f(int B, int n, int P, int heads, int d, const float *x_se
   return y;
 }
 
+static float *to_head_rep_f(int B, int n, int P, int G, int d, const float *x_seq) {
+  float *y = (float *)malloc(sizeof(float) * (size_t)B * n * P * d);
+  oracle_kv_replicate_to_head(B, n, P, G, (long)d * (long)sizeof(float), x_seq, y);
+  return y;
+}
+
 /*
  * Forward: seq->head all-to-all of Q, K, V; every rank r runs attention on
  * its hl = H/P query heads (KV head of local head hh: hh / (H/G), local to the
  * rank because rank r also owns KV heads [r*G/P, (r+1)*G/P)); head->seq
  * all-to-all of O.  lse_head is left in head layout [P][B][H/P][n].
+ * With fewer KV heads than ranks (G < P, P % G == 0) every rank receives a
+ * copy of the one KV head its query heads use (oracle_kv_replicate_to_head)
+ * and, in the backward, the copies' gradients are summed on the way back
+ * (oracle_kv_reduce_to_seq).
  */
 void oracle_ulysses_fwd(int B, int n, int P, int H, int G, int d, int mask,
                         const int *cu_seqlens, int num_docs, double scale,
@@ -359,10 +453,11 @@ void oracle_ulysses_fwd(int B, int n, int P, int H, int G, int d, int mask,
                         double *o_seq, double *lse_head) {
   attn_cfg c = make_cfg(n, d, mask, cu_seqlens, num_docs, scale);
   int *doc = doc_index(&c);
-  const int hl = H / P, gl = G / P, group = H / G;
+  const int rep = G % P != 0;          /* G < P: one replicated KV head per rank */
+  const int hl = H / P, gl = rep ? 1 : G / P, group = hl / gl;
   float *qh = to_head_f(B, n, P, H, d, q_seq);
-  float *kh = to_head_f(B, n, P, G, d, k_seq);
-  float *vh = to_head_f(B, n, P, G, d, v_seq);
+  float *kh = rep ? to_head_rep_f(B, n, P, G, d, k_seq) : to_head_f(B, n, P, G, d, k_seq);
+  float *vh = rep ? to_head_rep_f(B, n, P, G, d, v_seq) : to_head_f(B, n, P, G, d, v_seq);
   double *oh = (double *)malloc(sizeof(double) * (size_t)B * n * H * d);
   for (int r = 0; r < P; ++r)
     for (int b = 0; b < B; ++b)
@@ -386,14 +481,15 @@ void oracle_ulysses_bwd(int B, int n, int P, int H, int G, int d, int mask,
                         const float *do_seq, double *dq_seq, double *dk_seq, double *dv_seq) {
   attn_cfg c = make_cfg(n, d, mask, cu_seqlens, num_docs, scale);
   int *doc = doc_index(&c);
-  const int hl = H / P, gl = G / P, group = H / G;
+  const int rep = G % P != 0;          /* G < P: one replicated KV head per rank */
+  const int hl = H / P, gl = rep ? 1 : G / P, group = hl / gl;
   float *qh = to_head_f(B, n, P, H, d, q_seq);
-  float *kh = to_head_f(B, n, P, G, d, k_seq);
-  float *vh = to_head_f(B, n, P, G, d, v_seq);
+  float *kh = rep ? to_head_rep_f(B, n, P, G, d, k_seq) : to_head_f(B, n, P, G, d, k_seq);
+  float *vh = rep ? to_head_rep_f(B, n, P, G, d, v_seq) : to_head_f(B, n, P, G, d, v_seq);
   float *doh = to_head_f(B, n, P, H, d, do_seq);
   double *dqh = (double *)malloc(sizeof(double) * (size_t)B * n * H * d);
-  double *dkh = (double *)malloc(sizeof(double) * (size_t)B * n * G * d);
-  double *dvh = (double *)malloc(sizeof(double) * (size_t)B * n * G * d);
+  double *dkh = (double *)malloc(sizeof(double) * (size_t)B * n * P * gl * d);
+  double *dvh = (double *)malloc(sizeof(double) * (size_t)B * n * P * gl * d);
   double *o = (double *)malloc(sizeof(double) * (size_t)n * d);
   double *lse = (double *)malloc(sizeof(double) * (size_t)hl * n);
   double *Dv = (double *)malloc(sizeof(double) * (size_t)hl * n);
@@ -436,8 +532,13 @@ void oracle_ulysses_bwd(int B, int n, int P, int H, int G, int d, int mask,
       }
     }
   oracle_head_to_seq(B, n, P, H, (long)d * (long)sizeof(double), dqh, dq_seq);
-  oracle_head_to_seq(B, n, P, G, (long)d * (long)sizeof(double), dkh, dk_seq);
-  oracle_head_to_seq(B, n, P, G, (long)d * (long)sizeof(double), dvh, dv_seq);
+  if (rep) {
+    oracle_kv_reduce_to_seq(B, n, P, G, d, dkh, dk_seq);
+    oracle_kv_reduce_to_seq(B, n, P, G, d, dvh, dv_seq);
+  } else {
+    oracle_head_to_seq(B, n, P, G, (long)d * (long)sizeof(double), dkh, dk_seq);
+    oracle_head_to_seq(B, n, P, G, (long)d * (long)sizeof(double), dvh, dv_seq);
+  }
   free(qh); free(kh); free(vh); free(doh); free(dqh); free(dkh); free(dvh);
   free(o); free(lse); free(Dv); free(doc);
 }

@@ -237,13 +237,129 @@ def test_ulysses_equals_full_attention(mask, B, n, P, H, G, d):
 
 
 def test_ulysses_rejects_indivisible_shapes():
-    """Every rank must own whole query and KV heads (H % P == G % P == 0)."""
-    q, k = _randn(1, 32, 4, 8), _randn(1, 32, 2, 8)
-    with pytest.raises(ValueError):          # G = 2 KV heads cannot split over P = 4
-        oracle.ulysses_fwd(_seq(q, 4), _seq(k, 4), _seq(k, 4), 4)
-    q6 = _randn(1, 32, 6, 8)
+    """Every rank must own whole query heads (H % P == 0), and the KV heads
+    either split over the ranks (G % P == 0) or are copied to them (P % G == 0)."""
+    k3 = _randn(1, 24, 3, 8)
+    with pytest.raises(ValueError):          # G = 3 KV heads over P = 4: neither divides
+        oracle.ulysses_fwd(_seq(_randn(1, 24, 12, 8), 4), _seq(k3, 4), _seq(k3, 4), 4)
+    q4 = _randn(1, 32, 4, 8)
     with pytest.raises(ValueError):          # H = 6 query heads cannot split over P = 4
-        oracle.ulysses_fwd(_seq(q6, 4), _seq(q, 4), _seq(q, 4), 4)
+        oracle.ulysses_fwd(_seq(_randn(1, 32, 6, 8), 4), _seq(q4, 4), _seq(q4, 4), 4)
+
+
+# ------------------------------------------------ KV heads fewer than ranks
+
+def test_kv_replicate_with_as_many_kv_heads_as_ranks_is_seq_to_head():
+    """With G == P each rank holds exactly one KV head either way, so the
+    copying all-to-all reduces to the plain one (pinned by its closed form)."""
+    B, n, P, d = 2, 16, 4, 3
+    x = np.arange(P * B * (n // P) * P * d, dtype=np.int32).reshape(P, B, n // P, P, d)
+    assert np.array_equal(oracle.kv_replicate_to_head(x, B, n, P, P),
+                          oracle.seq_to_head(x, B, n, P, P))
+
+
+@pytest.mark.parametrize("B,n,P,H,G", [(1, 16, 4, 8, 2), (2, 24, 8, 16, 2), (1, 8, 8, 8, 1),
+                                       (1, 12, 4, 4, 1), (2, 32, 8, 32, 4)])
+def test_kv_replicate_gives_each_rank_the_kv_head_of_its_query_heads(B, n, P, H, G):
+    """GQA semantics rather than the copy formula: for every rank r and each of
+    its query heads q = r*H/P + hh, the rank's KV copy at every position t is
+    the natural-layout K[t][floor(q / (H/G))]."""
+    d = 3
+    k_nat = np.arange(B * n * G * d, dtype=np.int32).reshape(B, n, G, d)
+    rep = oracle.kv_replicate_to_head(_seq(k_nat, P), B, n, P, G)
+    assert rep.shape == (P, B, 1, n, d)
+    hl, grp = H // P, H // G
+    for r in range(P):
+        for hh in range(hl):
+            assert np.array_equal(rep[r, :, 0], k_nat[:, :, (r * hl + hh) // grp])
+
+
+@pytest.mark.parametrize("P,G", [(4, 2), (8, 1), (8, 4), (4, 4)])
+def test_kv_reduce_of_copies_is_copy_count_times_x(P, G):
+    """The P/G copies of a KV head carry the same values, so summing them back
+    gives (P/G) x exactly (a power of two: no rounding in fp64)."""
+    B, n, d = 2, 24, 5
+    x = _randn(P, B, n // P, G, d).astype(np.float64)
+    rep = oracle.kv_replicate_to_head(x, B, n, P, G)
+    assert np.array_equal(oracle.kv_reduce_to_seq(rep, B, n, P, G), x * (P // G))
+    # a gradient that lives on one copy only comes back once, at its own head
+    one = np.zeros_like(rep)
+    one[P - 1] = rep[P - 1]
+    back = oracle.kv_reduce_to_seq(one, B, n, P, G)
+    kk = (P - 1) * G // P
+    assert np.array_equal(back[:, :, :, kk], x[:, :, :, kk])
+    assert not np.any(np.delete(back, kk, axis=3))
+
+
+@pytest.mark.parametrize("mask", [MASK_NONE, MASK_CAUSAL, MASK_DOC_CAUSAL])
+@pytest.mark.parametrize("B,n,P,H,G,d", [(1, 32, 4, 8, 2, 8), (2, 16, 8, 8, 1, 4), (1, 24, 4, 8, 1, 8)])
+def test_ulysses_with_kv_copies_equals_full_attention(mask, B, n, P, H, G, d):
+    """G < P: the decomposition with copied KV heads still reproduces plain GQA
+    attention -- the forward bitwise (same routine, same data), the backward
+    (whose KV gradients are now summed over the copies in another order) to
+    fp64 rounding."""
+    q, k, v, do = _randn(B, n, H, d), _randn(B, n, G, d), _randn(B, n, G, d), _randn(B, n, H, d)
+    cu = np.array([0, 5, 13, n], np.int32) if mask == MASK_DOC_CAUSAL else None
+    o, lse = oracle.attention_fwd(q, k, v, mask=mask, cu_seqlens=cu)
+    ou, lu = oracle.ulysses_fwd(_seq(q, P), _seq(k, P), _seq(v, P), P, mask=mask, cu_seqlens=cu)
+    assert np.array_equal(_nat(ou), o)
+    assert np.array_equal(lu.transpose(1, 0, 2, 3).reshape(B, H, n), lse)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, mask=mask, cu_seqlens=cu)
+    uq, uk, uv = oracle.ulysses_bwd(_seq(q, P), _seq(k, P), _seq(v, P), _seq(do, P), P,
+                                    mask=mask, cu_seqlens=cu)
+    assert np.array_equal(_nat(uq), dq)
+    for got, ref in ((uk, dk), (uv, dv)):
+        assert np.abs(_nat(got) - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+# ------------------------------------------------------------- label shift
+
+def test_shift_labels_single_sequence_is_the_causal_lm_shift():
+    """One document, no padding: label(t) = ids[t+1] and the last position is
+    ignored -- the shift torch code writes as F.pad(ids[:, 1:], (0, 1), value=-100)
+    -- laid out by shard (seq layout [P][B][n/P])."""
+    B, n, P = 2, 24, 4
+    ids = rng.integers(0, 1000, (B, n)).astype(np.int32)
+    lab = oracle.shift_labels(ids, P)
+    ref = F.pad(torch.from_numpy(ids)[:, 1:], (0, 1), value=-100).numpy()
+    assert np.array_equal(lab, ref.reshape(B, P, n // P).transpose(1, 0, 2))
+    # a one-document cu_seqlens changes nothing
+    assert np.array_equal(oracle.shift_labels(ids, P, cu_seqlens=[0, n]), lab)
+    # no valid token: everything ignored
+    assert np.all(oracle.shift_labels(ids, P, valid_len=0) == -100)
+
+
+def test_shifted_sharded_loss_equals_unsharded_causal_lm_loss():
+    """Why the shift comes before sharding: the token-weighted loss over the P
+    shards with the shifted labels equals the plain next-token loss of the whole
+    sequence (torch cross_entropy of logits[:, :-1] against ids[:, 1:]); with
+    packed documents and padding it equals the mean of every document's own
+    next-token loss, each document computed alone."""
+    B, n, P, V = 2, 32, 4, 11
+    ids = rng.integers(0, V, (B, n)).astype(np.int32)
+    logits = _randn(B, n, V)
+    z_seq = logits.reshape(B, P, n // P, V).transpose(1, 0, 2, 3).reshape(-1, V)
+    lab = oracle.shift_labels(ids, P)
+    S, C, L, bad = oracle.loss_aggregate(z_seq, lab.reshape(-1), P)
+    ref = F.cross_entropy(torch.tensor(logits[:, :-1], dtype=torch.float64).reshape(-1, V),
+                          torch.from_numpy(ids[:, 1:]).reshape(-1).long())
+    assert bad == 0 and C.sum() == B * (n - 1) and abs(L - ref.item()) < 1e-12
+    # packed documents [0,5) [5,19) [19,30) and two padding tokens [30,32)
+    cu, valid = [0, 5, 19, 30, 32], 30
+    lab = oracle.shift_labels(ids, P, cu_seqlens=cu, valid_len=valid)
+    S, C, L, bad = oracle.loss_aggregate(z_seq, lab.reshape(-1), P)
+    tot, cnt = 0.0, 0
+    for b in range(B):
+        for a, e in zip(cu[:-2], cu[1:-1]):
+            z = torch.tensor(logits[b, a:e - 1], dtype=torch.float64)
+            tot += F.cross_entropy(z, torch.from_numpy(ids[b, a + 1:e]).long(), reduction="sum").item()
+            cnt += e - a - 1
+    assert C.sum() == cnt and abs(L - tot / cnt) < 1e-12
+    # the label of a shard's last position is the next shard's first token
+    lab = oracle.shift_labels(ids, P)
+    s = n // P
+    for r in range(P - 1):
+        assert np.array_equal(lab[r, :, s - 1], ids[:, (r + 1) * s])
 
 
 # ------------------------------------------------------------------- backward
