@@ -377,6 +377,7 @@ def run_ours(args, rank, world, dev):
     tokens = inp["B"] * inp["n"]
     value = job_throughput(tokens, world, ms_max)
     peaks, peak_src = load_peaks()
+    side = side_kernels(inp, dev, args.steps, peaks)
     kernels = {}
     for name, (tot_ms, cnt) in prof.items():
         per_launch = tot_ms / cnt
@@ -437,6 +438,7 @@ def run_ours(args, rank, world, dev):
         "roofline": roof,
         "kernels": kernels,
         "loss_grad": loss_bwd,
+        "side_kernels": side,
         "gpu_launches": launches,
         "e2e": {"value": job_throughput(tokens, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": io.h2d, "d2h_bytes_per_step": io.d2h},
@@ -445,6 +447,58 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp, budget_s=args.cpu_budget)
     return line
+
+
+def side_kernels(inp, dev, steps: int, peaks) -> dict:
+    """Kernels outside the layer step, each timed on its own at the workload's
+    sizes (CUDA events on the launching stream, via the library's profiler):
+    the KV-head copies used when there are fewer KV heads than ranks (this K
+    split over 2G ranks, so every KV head goes to two ranks, and the summing
+    reverse of its gradient), and the label shift before sharding."""
+    from long_context_sequence_all_b200 import ulysses as U
+    B, n, G, d = inp["B"], inp["n"], inp["G"], inp["d"]
+    eb = inp["k"].element_size()
+    out = {}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        U.ulysses_profile_enable(True)
+        for _ in range(steps):
+            fn()
+        torch.cuda.synchronize()
+        prof = U.ulysses_profile_read()
+        U.ulysses_profile_enable(False)
+        if U.ulysses_read_error():
+            raise RuntimeError("device error word set by a side kernel")
+        return prof
+
+    def entry(prof, name, nbytes, note):
+        tot, cnt = prof[name]
+        gbs = nbytes / (tot / cnt / 1e3) / 1e9
+        return {"ms_per_launch": tot / cnt, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                "bytes_per_launch": nbytes, "note": note}
+
+    P2 = 2 * G
+    if n % P2 == 0:
+        k2 = to_natural(inp["k"]).reshape(B, P2, n // P2, G, d).transpose(0, 1).contiguous().to(dev)
+        rep = torch.empty((P2, B, 1, n, d), dtype=k2.dtype, device=dev)
+        back = torch.empty_like(k2)
+        prof = timed(lambda: (U.ulysses_kv_seq_to_head_replicated(k2, P2, out=rep),
+                              U.ulysses_kv_head_to_seq_reduce(rep, P2, G, out=back)))
+        small, big = B * n * G * d * eb, B * n * P2 * d * eb
+        note = f"K of this workload over P={P2} ranks (G={G}: two copies per KV head)"
+        out["kv_seq_to_head_rep"] = entry(prof, "kv_seq_to_head_rep", small + big, note)
+        out["kv_head_to_seq_sum"] = entry(prof, "kv_head_to_seq_sum", big + small, note)
+        del k2, rep, back
+    ids = torch.randint(0, 151936, (B, n), dtype=torch.int32, device=dev)
+    lab = torch.empty((inp["P"], B, n // inp["P"]), dtype=torch.int32, device=dev)
+    cu = inp["cu_seqlens"].to(dev) if inp["cu_seqlens"] is not None else None
+    prof = timed(lambda: U.ulysses_shift_labels(ids, inp["P"], cu_seqlens=cu, valid_len=inp["real_tokens"],
+                                                out=lab))
+    out["shift_labels"] = entry(prof, "shift_labels", 2.0 * B * n * 4,
+                                "int32 ids read once, labels written once")
+    return out
 
 
 def _l2_note(inp):

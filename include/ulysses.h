@@ -104,6 +104,61 @@ uly_status ulysses_head_to_seq(int32_t batch, int32_t seq_len, int32_t world, in
                                void *dst, void *stream);
 
 /*
+ * First all-to-all of K or V when there are fewer KV heads than ranks
+ * (G < P; "Ulysses 序列平行化", section "與 Ring Attention 的比較": the method
+ * needs at least as many heads as ranks, and grouped KV heads fall short of it).
+ * Rank r uses KV head floor(r*G/P) for all of its query heads, so that head is
+ * copied whole to each of its P/G ranks:
+ *   src: seq layout [P][B][n/P][G][head_dim]
+ *   dst: [P][B][1][n][head_dim], dst[r][b][0][t] = src[t/s][b][t%s][r*G/P]
+ * After it, ulysses_attn_fwd / _bwd run with n_kv_heads = P (one KV head per
+ * rank); their results equal plain GQA attention with G KV heads.  The element
+ * type is opaque (elem_bytes in {1,2,4,8}); the copy is bit-exact.  Requires
+ * n % P == 0, P % G == 0, head_dim * elem_bytes % 16 == 0 and a power-of-two
+ * number (<= 64) of 16-byte vectors per row.  dst must not overlap src.
+ */
+uly_status ulysses_kv_seq_to_head_replicated(int32_t batch, int32_t seq_len, int32_t world,
+                                             int32_t kv_heads, int32_t head_dim,
+                                             int32_t elem_bytes, const void *src, void *dst,
+                                             void *stream);
+
+/*
+ * Reverse of ulysses_kv_seq_to_head_replicated for gradients: the gradient of
+ * a KV head is the sum of the gradients its P/G copies received,
+ *   dst[r][b][tt][k] = sum_{j < P/G} src[k*P/G + j][b][0][r*s + tt],
+ * accumulated in fp32 in rank order and rounded once (RNE) to `dtype`
+ * (ULY_BF16 or ULY_F32).  src [P][B][1][n][d], dst seq layout [P][B][n/P][G][d].
+ * Same shape and alignment rules; dst must not overlap src.
+ */
+uly_status ulysses_kv_head_to_seq_reduce(int32_t batch, int32_t seq_len, int32_t world,
+                                         int32_t kv_heads, int32_t head_dim, int32_t dtype,
+                                         const void *src, void *dst, void *stream);
+
+/*
+ * Next-token labels, shifted on the whole sequence BEFORE it is sharded (the
+ * last position of shard r needs the first token of shard r+1; the SFT
+ * trainer's automatic label shift, "Ulysses 序列平行化", section
+ * "在 Hugging Face 生態系統中的整合"; padding and packed sequences,
+ * "Paralelismul de Secvență Ulysses", section "Integrarea cu Transformers
+ * Trainer și TRL SFTTrainer"):
+ *   labels[r][b][tt] (t = r*n/P + tt) = input_ids[b][t+1]  if t+1 < valid_len and
+ *                                       t+1 is not a document start,
+ *                                     = ignore_index       otherwise.
+ * input_ids: DEVICE int32 [B][n] in sequence order.  labels: DEVICE int32
+ * [P][B][n/P] (the layout ulysses_loss_aggregate reads as [P][tokens/P]).
+ * cu_seqlens: NULL (num_docs = 0) for one document per row, else DEVICE int32
+ * [num_docs+1] as in uly_attn_desc (cu[0] = 0, nondecreasing, cu[num_docs] = n;
+ * another array gives unspecified but in-bounds labels); document starts are
+ * cu[1..num_docs-1].  valid_len in [0, n]: positions >= valid_len are padding
+ * (padding to a multiple of P), and the token before them gets ignore_index.
+ * labels must not overlap input_ids or cu_seqlens.
+ */
+uly_status ulysses_shift_labels(int32_t batch, int32_t seq_len, int32_t world,
+                                const int32_t *input_ids, const int32_t *cu_seqlens,
+                                int32_t num_docs, int32_t valid_len, int32_t ignore_index,
+                                int32_t *labels, void *stream);
+
+/*
  * Local attention (step 4) of every logical rank, head layout in and out:
  * q, o [P][B][H/P][n][d]; k, v [P][B][G/P][n][d]; lse [P][B][H/P][n] (fp32).
  * O = softmax(scale * Q K^T + mask) V per query head, LSE its log-sum-exp.

@@ -51,6 +51,14 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *, const HeadGeom &, const M
                                 const void *, const void *, const void *, const void *,
                                 const float *, const void *, void *, void *, void *, float *,
                                 cudaStream_t);
+uly_status kv_rep_validate(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *,
+                           const void *);
+uly_status kv_replicate_launch(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *,
+                               void *, cudaStream_t);
+uly_status kv_reduce_launch(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *, void *,
+                            cudaStream_t);
+uly_status shift_labels_launch(int32_t, int32_t, int32_t, const int32_t *, const int32_t *, int32_t,
+                               int32_t, int32_t, int32_t *, cudaStream_t);
 size_t loss_workspace_bytes(int P, long long per_shard);
 size_t loss_bwd_workspace_bytes(int P, long long per_shard);
 uly_status loss_bwd_launch(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *, int32_t,
@@ -134,6 +142,45 @@ uly_status ulysses_head_to_seq(int32_t batch, int32_t seq_len, int32_t world, in
   if (st != ULY_OK) return st;
   return permute_launch(false, batch, seq_len, world, heads, head_dim, eb, src, dst,
                         static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_kv_seq_to_head_replicated(int32_t batch, int32_t seq_len, int32_t world,
+                                             int32_t kv_heads, int32_t head_dim, int32_t eb,
+                                             const void *src, void *dst, void *stream) {
+  uly_status st = kv_rep_validate(batch, seq_len, world, kv_heads, head_dim, eb, src, dst);
+  if (st != ULY_OK) return st;
+  return kv_replicate_launch(batch, seq_len, world, kv_heads, head_dim, eb, src, dst,
+                             static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_kv_head_to_seq_reduce(int32_t batch, int32_t seq_len, int32_t world,
+                                         int32_t kv_heads, int32_t head_dim, int32_t dtype,
+                                         const void *src, void *dst, void *stream) {
+  if (dtype != ULY_F32 && dtype != ULY_BF16) return ULY_ERR_DTYPE;
+  // the same rules as the forward copy with the roles of the buffers swapped
+  // (dst holds the G heads, src the P copies)
+  uly_status st = kv_rep_validate(batch, seq_len, world, kv_heads, head_dim,
+                                  dtype == ULY_BF16 ? 2 : 4, dst, src);
+  if (st != ULY_OK) return st;
+  return kv_reduce_launch(batch, seq_len, world, kv_heads, head_dim, dtype, src, dst,
+                          static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_shift_labels(int32_t batch, int32_t seq_len, int32_t world,
+                                const int32_t *input_ids, const int32_t *cu_seqlens,
+                                int32_t num_docs, int32_t valid_len, int32_t ignore_index,
+                                int32_t *labels, void *stream) {
+  if (!input_ids || !labels) return ULY_ERR_NULL;
+  if (batch <= 0 || seq_len <= 0 || world <= 0 || seq_len % world) return ULY_ERR_SHAPE;
+  if (valid_len < 0 || valid_len > seq_len) return ULY_ERR_SHAPE;
+  if (num_docs < 0 || (num_docs > 0 && !cu_seqlens)) return ULY_ERR_NULL;
+  if ((long long)batch * seq_len > (1LL << 40)) return ULY_ERR_SHAPE;
+  const size_t bytes = (size_t)batch * seq_len * sizeof(int32_t);
+  if (overlap(input_ids, bytes, labels, bytes)) return ULY_ERR_ALIAS;
+  if (num_docs > 0 && overlap(cu_seqlens, (size_t)(num_docs + 1) * sizeof(int32_t), labels, bytes))
+    return ULY_ERR_ALIAS;
+  return shift_labels_launch(batch, seq_len, world, input_ids, cu_seqlens, num_docs, valid_len,
+                             ignore_index, labels, static_cast<cudaStream_t>(stream));
 }
 
 uly_status ulysses_attn_fwd(const uly_attn_desc *d, const void *q, const void *k, const void *v,

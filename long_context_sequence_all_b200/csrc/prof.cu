@@ -40,7 +40,8 @@ const char *name(int k) {
   static const char *names[K_COUNT] = {
       "seq_to_head", "head_to_seq", "loss_partial", "loss_finalize", "attn_fwd_f32",
       "attn_dq_f32", "attn_dkdv_f32", "attn_bwd_dot", "attn_fwd_sm100", "attn_dkdv_sm100",
-      "attn_dq_sm100", "attn_bwd_stats", "loss_fwd_bwd"};
+      "attn_dq_sm100", "attn_bwd_stats", "loss_fwd_bwd", "kv_seq_to_head_rep",
+      "kv_head_to_seq_sum", "shift_labels"};
   return (k >= 0 && k < K_COUNT) ? names[k] : "unknown";
 }
 

@@ -24,6 +24,9 @@ enum Kernel {
   K_ATTN_DQ_SM100,
   K_ATTN_BWD_STATS,
   K_LOSS_FWD_BWD,
+  K_KV_REPLICATE,
+  K_KV_REDUCE,
+  K_SHIFT_LABELS,
   K_COUNT
 };
 

@@ -23,7 +23,8 @@ MASK_NONE, MASK_CAUSAL, MASK_DOC_CAUSAL = 0, 1, 2
 STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE",
           4: "ULY_ERR_ALIGN", 5: "ULY_ERR_ALIAS", 6: "ULY_ERR_UNSUPPORTED", 7: "ULY_ERR_CUDA",
           8: "ULY_ERR_LABEL", 9: "ULY_ERR_TIMEOUT", 10: "ULY_ERR_WORKSPACE"}
-EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd",
+EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head_replicated",
+           "ulysses_kv_head_to_seq_reduce", "ulysses_shift_labels", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
            "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
            "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info",
@@ -62,6 +63,12 @@ def lib() -> ctypes.CDLL:
             vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
             for name in ("ulysses_seq_to_head", "ulysses_head_to_seq"):
                 getattr(L, name).argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
+                getattr(L, name).restype = ctypes.c_int
+            L.ulysses_kv_seq_to_head_replicated.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
+            L.ulysses_kv_head_to_seq_reduce.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
+            L.ulysses_shift_labels.argtypes = [i32, i32, i32, vp, vp, i32, i32, i32, vp, vp]
+            for name in ("ulysses_kv_seq_to_head_replicated", "ulysses_kv_head_to_seq_reduce",
+                         "ulysses_shift_labels"):
                 getattr(L, name).restype = ctypes.c_int
             D = ctypes.POINTER(AttnDesc)
             L.ulysses_attn_fwd.argtypes = [D, vp, vp, vp, vp, vp, vp]
@@ -148,6 +155,54 @@ def ulysses_head_to_seq(x: torch.Tensor, P: int, out: torch.Tensor | None = None
         out = torch.empty((P, B, n // P, heads, d), dtype=x.dtype, device=x.device)
     _check(lib().ulysses_head_to_seq(B, n, P, heads, d, x.element_size(), _p(x), _p(out),
                                      _stream(stream)), "ulysses_head_to_seq")
+    return out
+
+
+def ulysses_kv_seq_to_head_replicated(x: torch.Tensor, P: int, out: torch.Tensor | None = None,
+                                      stream=None):
+    """G < P KV heads: [P][B][n/P][G][d] -> [P][B][1][n][d], rank r receiving
+    KV head floor(r*G/P) (bit-exact copy)."""
+    P_, B, s, G, d = x.shape
+    if P_ != P or G <= 0 or P % G:
+        raise UlyssesError(2, f"ulysses_kv_seq_to_head_replicated: shape {tuple(x.shape)} with P={P}")
+    n = P * s
+    if out is None:
+        out = torch.empty((P, B, 1, n, d), dtype=x.dtype, device=x.device)
+    _check(lib().ulysses_kv_seq_to_head_replicated(B, n, P, G, d, x.element_size(), _p(x), _p(out),
+                                                   _stream(stream)),
+           "ulysses_kv_seq_to_head_replicated")
+    return out
+
+
+def ulysses_kv_head_to_seq_reduce(x: torch.Tensor, P: int, G: int, out: torch.Tensor | None = None,
+                                  stream=None):
+    """Gradients of the KV copies, [P][B][1][n][d] -> seq layout [P][B][n/P][G][d],
+    each KV head's gradient summed over its P/G copies (fp32 sum, one rounding)."""
+    P_, B, one, n, d = x.shape
+    if P_ != P or one != 1 or G <= 0 or P % G or n % P:
+        raise UlyssesError(2, f"ulysses_kv_head_to_seq_reduce: shape {tuple(x.shape)} with P={P}, G={G}")
+    if out is None:
+        out = torch.empty((P, B, n // P, G, d), dtype=x.dtype, device=x.device)
+    _check(lib().ulysses_kv_head_to_seq_reduce(B, n, P, G, d, _dtype_code(x), _p(x), _p(out),
+                                               _stream(stream)),
+           "ulysses_kv_head_to_seq_reduce")
+    return out
+
+
+def ulysses_shift_labels(input_ids: torch.Tensor, P: int, cu_seqlens: torch.Tensor | None = None,
+                         valid_len: int | None = None, ignore_index: int = -100,
+                         out: torch.Tensor | None = None, stream=None):
+    """Next-token labels of input_ids [B][n] (int32), shifted before sharding:
+    returns the seq layout [P][B][n/P] (int32)."""
+    B, n = input_ids.shape
+    if input_ids.dtype != torch.int32 or n % P:
+        raise UlyssesError(2, f"ulysses_shift_labels: ids {tuple(input_ids.shape)} {input_ids.dtype} with P={P}")
+    nd = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((P, B, n // P), dtype=torch.int32, device=input_ids.device)
+    vl = n if valid_len is None else int(valid_len)
+    _check(lib().ulysses_shift_labels(B, n, P, _p(input_ids), _p(cu_seqlens), nd, vl, ignore_index,
+                                      _p(out), _stream(stream)), "ulysses_shift_labels")
     return out
 
 

@@ -58,6 +58,36 @@ def test_permute_validation(L):
     assert L.ulysses_seq_to_head(0, 1024, 4, 8, 64, 4, a, b, None) == 2
 
 
+def test_kv_copy_validation(L):
+    vp = ctypes.c_void_p
+    a, b = vp(1 << 20), vp(1 << 30)
+    rep, red = L.ulysses_kv_seq_to_head_replicated, L.ulysses_kv_head_to_seq_reduce
+    assert rep(1, 1024, 8, 2, 128, 2, None, b, None) == 1                 # NULL
+    assert rep(1, 1024, 8, 3, 128, 2, a, b, None) == 2                    # P % G
+    assert rep(1, 1020, 8, 2, 128, 2, a, b, None) == 2                    # n % P
+    assert rep(1, 1024, 8, 2, 128, 3, a, b, None) == 3                    # elem bytes
+    assert rep(1, 1024, 8, 2, 4, 2, a, b, None) == 4                      # row not 16 B
+    # the copies (dst, P rows per position) overlap a source placed inside them
+    assert rep(1, 1024, 8, 2, 128, 2, vp((1 << 20) + 1024 * 2 * 256), a, None) == 5
+    assert red(1, 1024, 8, 2, 128, 7, a, b, None) == 3                    # dtype
+    assert red(1, 1024, 8, 3, 128, 1, a, b, None) == 2
+    assert red(1, 1024, 8, 2, 128, 1, a, vp((1 << 20) + 1024 * 8 * 256 - 16), None) == 5
+    assert red(1, 1024, 8, 2, 128, 1, vp((1 << 20) + 8), b, None) == 4    # misaligned
+
+
+def test_shift_labels_validation(L):
+    vp = ctypes.c_void_p
+    ids, lab, cu = vp(1 << 20), vp(1 << 30), vp(1 << 24)
+    f = L.ulysses_shift_labels
+    assert f(1, 1024, 4, None, None, 0, 1024, -100, lab, None) == 1
+    assert f(1, 1023, 4, ids, None, 0, 1023, -100, lab, None) == 2        # n % P
+    assert f(1, 1024, 4, ids, None, 0, 1025, -100, lab, None) == 2        # valid_len > n
+    assert f(1, 1024, 4, ids, None, 0, -1, -100, lab, None) == 2
+    assert f(1, 1024, 4, ids, None, 3, 1024, -100, lab, None) == 1        # docs without cu
+    assert f(2, 1024, 4, ids, None, 0, 1024, -100, vp((1 << 20) + 4096), None) == 5
+    assert f(1, 1024, 4, ids, vp((1 << 30) + 64), 2, 1024, -100, lab, None) == 5  # cu inside labels
+
+
 def test_attn_desc_validation(L):
     from long_context_sequence_all_b200 import ulysses as U
     n = ctypes.c_size_t(0)
