@@ -5,8 +5,10 @@ baseline / reference arm may import this package.  The product path (the CUDA
 library and its binding) never imports, links or executes anything here.
 
 The arithmetic lives in ``ulysses_oracle.c`` (plain loops, fp64, OpenMP over
-independent rows); this module only builds it with gcc and marshals numpy
-arrays.  It shares no code with the CUDA path.  Every function is pinned by
+independent rows); this module builds it with gcc and marshals numpy arrays.
+The projections either side of the attention (a library fp64 matrix product
+as their one step) and the rotary position encoding are written here in
+numpy, fp64.  It shares no code with the CUDA path.  Every function is pinned by
 tests under ``tests/`` against closed forms, brute force, invariants, library
 routines and finite differences.
 """
@@ -301,3 +303,73 @@ def loss_grad(logits, labels, ignore_index=-100):
     g = np.empty((T, V), np.float64)
     C = _load().oracle_loss_grad(T, V, _ptr(z), _ptr(y), ignore_index, _ptr(g))
     return g, int(C)
+
+
+# --------------------------------------------------------------------------
+# Steps 2 and 6: QKV projection with rotary positions, output projection
+# --------------------------------------------------------------------------
+
+def rope(x, pos, base=1.0e6):
+    """Rotary position encoding of the last axis (d even), fp64, in the
+    rotate-half pairing: element e and e + d/2 form a pair rotated by the angle
+    pos * base^(-2e/d):
+        y[e]       = x[e] cos - x[e + d/2] sin
+        y[e + d/2] = x[e + d/2] cos + x[e] sin
+    x [..., d], pos broadcastable to x[..., 0]."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    theta = base ** (-2.0 * np.arange(half, dtype=np.float64) / d)
+    ang = np.asarray(pos, np.float64)[..., None] * theta
+    c, sn = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * sn, x2 * c + x1 * sn], axis=-1)
+
+
+def qkv_proj_rope(x_seq, w_qkv, P, H, G, d, base=1.0e6, positions=None):
+    """Ulysses steps 2-3 ("Paralelismul de Secvență Ulysses", section
+    "Mecanismul de funcționare Ulysses"): every rank projects its own tokens,
+    rotates Q and K by each token's position in the WHOLE sequence (rank r's
+    local token tt sits at t = r*n/P + tt: the shard's offset; ms-swift page,
+    section 6.2, names a RoPE that ignores this offset as a failure), and the
+    first all-to-all gives every rank all positions of its heads.
+      x_seq [P][B][s][hidden], w_qkv [(H+2G)*d][hidden] (rows: H query heads,
+      then G key heads, then G value heads, d rows each),
+      positions: None (t itself) or [B][n] (e.g. restarting per document).
+    Returns q [P][B][H/P][n][d], k and v [P][B][G/P][n][d] (fp64); with fewer
+    KV heads than ranks (P % G == 0) k and v are [P][B][1][n][d], every rank
+    holding a copy of the KV head its query heads use."""
+    x = np.asarray(x_seq, np.float64)
+    w = np.asarray(w_qkv, np.float64)
+    P_, B, s, hidden = x.shape
+    n = P * s
+    _check_ulysses(n, P, H, G)
+    if w.shape != ((H + 2 * G) * d, hidden):
+        raise ValueError(f"w_qkv shape {w.shape}, expected {((H + 2 * G) * d, hidden)}")
+    q_seq = np.empty((P, B, s, H, d))
+    k_seq = np.empty((P, B, s, G, d))
+    v_seq = np.empty((P, B, s, G, d))
+    for r in range(P):
+        y = (x[r].reshape(B * s, hidden) @ w.T).reshape(B, s, H + 2 * G, d)
+        t = r * s + np.arange(s)
+        pos = np.broadcast_to(t, (B, s)) if positions is None else np.asarray(positions)[:, t]
+        q_seq[r] = rope(y[:, :, :H], pos[:, :, None], base)
+        k_seq[r] = rope(y[:, :, H:H + G], pos[:, :, None], base)
+        v_seq[r] = y[:, :, H + G:]
+    kv = (lambda z: seq_to_head(z, B, n, P, G)) if G % P == 0 else \
+        (lambda z: kv_replicate_to_head(z, B, n, P, G))
+    return seq_to_head(q_seq, B, n, P, H), kv(k_seq), kv(v_seq)
+
+
+def o_proj(o_head, w_o, P):
+    """Ulysses steps 5-6: the second all-to-all returns every rank its own
+    positions for all heads, then each rank applies the output projection to
+    its tokens.  o_head [P][B][H/P][n][d], w_o [hidden][H*d] -> y seq layout
+    [P][B][n/P][hidden] (fp64)."""
+    o = np.asarray(o_head, np.float64)
+    P_, B, hl, n, d = o.shape
+    H = hl * P
+    o_seq = head_to_seq(o, B, n, P, H)                 # [P][B][s][H][d]
+    w = np.asarray(w_o, np.float64)
+    y = o_seq.reshape(P * B * (n // P), H * d) @ w.T
+    return y.reshape(P, B, n // P, w.shape[0])

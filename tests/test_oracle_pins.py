@@ -615,3 +615,93 @@ def test_pages_loss_parity_bound_is_met_by_sharding():
     ref = _ce_ref(z, y)
     for P in (1, 2, 4, 8, 16):
         assert abs(oracle.loss_aggregate(z, y, P)[2] - ref) < bound * 1e-6
+
+
+# ------------------------------------------- projections and rotary positions
+
+def test_rope_is_a_complex_rotation():
+    """Pairing element e with e + d/2 as the complex number x_e + i x_{e+d/2},
+    the encoding multiplies it by exp(i * pos * base^(-2e/d)) (numpy's complex
+    exponential, an independent formulation); position 0 is the identity and
+    the first pair turns by exactly pos radians."""
+    d, base = 16, 1.0e6
+    x = rng.standard_normal((5, d))
+    pos = np.array([0, 1, 7, 4096, 262143], np.float64)
+    z = (x[:, :d // 2] + 1j * x[:, d // 2:]) * np.exp(1j * pos[:, None] * base ** (-2.0 * np.arange(d // 2) / d))
+    y = oracle.rope(x, pos, base)
+    assert np.abs(y[:, :d // 2] - z.real).max() < 1e-12 and np.abs(y[:, d // 2:] - z.imag).max() < 1e-12
+    assert np.array_equal(y[0], x[0])
+    ang = np.arctan2(y[1, d // 2], y[1, 0]) - np.arctan2(x[1, d // 2], x[1, 0])
+    assert abs((ang + np.pi) % (2 * np.pi) - np.pi - 1.0) < 1e-12
+    # every pair keeps its length
+    assert np.allclose(np.hypot(y[:, :d // 2], y[:, d // 2:]), np.hypot(x[:, :d // 2], x[:, d // 2:]), atol=1e-12)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    """<rope(q, i), rope(k, j)> is a function of i - j: shifting both positions
+    by the same offset (a shard's offset, say) leaves every score unchanged."""
+    d = 32
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    for i, j, c in [(5, 2, 1000), (300, 301, 65536), (0, 0, 131072)]:
+        a = oracle.rope(q, i) @ oracle.rope(k, j)
+        b = oracle.rope(q, i + c) @ oracle.rope(k, j + c)
+        assert abs(a - b) < 1e-9 * max(1.0, abs(a))
+    assert abs(oracle.rope(q, 9) @ oracle.rope(k, 9) - q @ k) < 1e-12
+
+
+@pytest.mark.parametrize("P,B,H,G", [(4, 1, 8, 4), (2, 2, 4, 2), (4, 1, 8, 2)])
+def test_qkv_projection_sharded_equals_unsharded(P, B, H, G):
+    """Sharding must not change what attention sees: every rank rotates its
+    tokens by their positions in the whole sequence, so the P-rank projection
+    (in head layout) holds the single-rank result (to fp64 rounding: the
+    library product may block rows differently).  A rank that used its local
+    positions would fail this."""
+    d, hidden, n = 8, 24, 32
+    x_nat = rng.standard_normal((B, n, hidden))
+    w = rng.standard_normal(((H + 2 * G) * d, hidden)) / np.sqrt(hidden)
+    q1, k1, v1 = oracle.qkv_proj_rope(x_nat[None], w, 1, H, G, d)       # P = 1: [1][B][H][n][d]
+    qP, kP, vP = oracle.qkv_proj_rope(x_nat.reshape(B, P, n // P, hidden).transpose(1, 0, 2, 3), w, P, H, G, d)
+    nat = lambda z: z.transpose(1, 0, 2, 3, 4).reshape(B, -1, n, d)     # [B][heads][n][d]
+    same = lambda a, b: np.abs(a - b).max() < 1e-12
+    assert same(nat(qP), q1[0])
+    if G % P == 0:
+        assert same(nat(kP), k1[0]) and same(nat(vP), v1[0])
+    else:   # one copied KV head per rank: rank r holds KV head r*G/P
+        for r in range(P):
+            assert same(kP[r, :, 0], k1[0][:, r * G // P]) and same(vP[r, :, 0], v1[0][:, r * G // P])
+    # local positions (the failure the ms-swift page describes) would differ
+    pos_local = np.tile(np.arange(n) % (n // P), (B, 1))
+    qL, _, _ = oracle.qkv_proj_rope(x_nat.reshape(B, P, n // P, hidden).transpose(1, 0, 2, 3), w, P, H, G, d,
+                                    positions=pos_local)
+    assert not np.allclose(nat(qL)[:, :, n // P:], q1[0][:, :, n // P:])
+
+
+def test_qkv_projection_one_hot_reads_weight_columns():
+    """A token whose hidden state is the unit vector e_c projects to column c
+    of the weight matrix, split into H query heads, then G key heads, then G
+    value heads of d rows each (position 0: no rotation)."""
+    P, H, G, d, hidden, n = 2, 4, 2, 8, 16, 4
+    w = rng.standard_normal(((H + 2 * G) * d, hidden))
+    x = np.zeros((P, 1, n // P, hidden))
+    c = 5
+    x[0, 0, 0, c] = 1.0                 # token 0 of rank 0 (global position 0)
+    q, k, v = oracle.qkv_proj_rope(x, w, P, H, G, d)
+    col = w[:, c].reshape(H + 2 * G, d)
+    for h in range(H):
+        assert np.array_equal(q[h // (H // P), 0, h % (H // P), 0], col[h])
+    for g in range(G):
+        assert np.array_equal(k[g // (G // P), 0, g % (G // P), 0], col[H + g])
+        assert np.array_equal(v[g // (G // P), 0, g % (G // P), 0], col[H + G + g])
+    assert not np.any(q[:, :, :, 1:]) and not np.any(v[:, :, :, 1:])
+
+
+def test_output_projection_matches_torch_linear():
+    """Step 6 against torch.nn.functional.linear on the natural layout (the
+    head layout turned back by an independent numpy transpose)."""
+    P, B, H, d, n, hidden = 4, 2, 8, 8, 16, 12
+    o_head = rng.standard_normal((P, B, H // P, n, d))
+    w = rng.standard_normal((hidden, H * d))
+    y = oracle.o_proj(o_head, w, P)                                     # [P][B][s][hidden]
+    o_nat = o_head.transpose(1, 3, 0, 2, 4).reshape(B, n, H * d)        # heads r*H/P + hh in order
+    ref = F.linear(torch.from_numpy(o_nat), torch.from_numpy(w)).numpy()
+    assert np.abs(y.transpose(1, 0, 2, 3).reshape(B, n, hidden) - ref).max() < 1e-12
