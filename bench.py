@@ -491,6 +491,31 @@ def side_kernels(inp, dev, steps: int, peaks) -> dict:
         out["kv_seq_to_head_rep"] = entry(prof, "kv_seq_to_head_rep", small + big, note)
         out["kv_head_to_seq_sum"] = entry(prof, "kv_head_to_seq_sum", big + small, note)
         del k2, rep, back
+    # the projections either side of the attention (synthetic weights of the
+    # Qwen3-4B shapes: hidden 2560), each a tcgen05 GEMM with an all-to-all
+    # folded in; timed alone, so against the burst bf16 peak
+    P, H, hidden = inp["P"], inp["H"], 2560
+    if G % P == 0:
+        x = torch.randn((P, B, n // P, hidden), device=dev).to(torch.bfloat16)
+        w = (torch.randn(((H + 2 * G) * d, hidden), device=dev) / hidden ** 0.5).to(torch.bfloat16)
+        tab = U.ulysses_rope_table(n, d, 1.0e6, device=dev)
+        qb = torch.empty((P, B, H // P, n, d), dtype=torch.bfloat16, device=dev)
+        kb = torch.empty((P, B, G // P, n, d), dtype=torch.bfloat16, device=dev)
+        vb = torch.empty_like(kb)
+        prof = timed(lambda: U.ulysses_qkv_proj_rope(x, w, P, H, G, tab, q=qb, k=kb, v=vb))
+        wo = (torch.randn((hidden, H * d), device=dev) / (H * d) ** 0.5).to(torch.bfloat16)
+        yb = torch.empty((P, B, n // P, hidden), dtype=torch.bfloat16, device=dev)
+        prof2 = timed(lambda: U.ulysses_o_proj(qb, wo, P, y=yb))
+        for name, pr, fl, note in (
+                ("qkv_proj_sm100", prof, 2.0 * B * n * (H + 2 * G) * d * hidden,
+                 f"[Q K V] = X W^T, rotary positions, written in the head layout; hidden={hidden}"),
+                ("o_proj_sm100", prof2, 2.0 * B * n * hidden * H * d,
+                 f"Y = O W_o^T read from the head layout, written in the seq layout; hidden={hidden}")):
+            tot, cnt = pr[name]
+            tf = fl / (tot / cnt / 1e3) / 1e12
+            out[name] = {"ms_per_launch": tot / cnt, "tflops": tf, "frac_bf16": tf / peaks["bf16_tflops"],
+                         "flops_per_launch": fl, "note": note}
+        del x, w, tab, qb, kb, vb, wo, yb
     ids = torch.randint(0, 151936, (B, n), dtype=torch.int32, device=dev)
     lab = torch.empty((inp["P"], B, n // inp["P"]), dtype=torch.int32, device=dev)
     cu = inp["cu_seqlens"].to(dev) if inp["cu_seqlens"] is not None else None

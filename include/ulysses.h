@@ -159,6 +159,62 @@ uly_status ulysses_shift_labels(int32_t batch, int32_t seq_len, int32_t world,
                                 int32_t *labels, void *stream);
 
 /*
+ * Rotary position table for ulysses_qkv_proj_rope: for every position
+ * p < max_pos and pair e < head_dim/2, table[p][e] = (cos, sin) of the angle
+ * p * base^(-2e/head_dim), computed in double precision and rounded once to
+ * float.  table: DEVICE float [max_pos][head_dim/2][2], 16-byte aligned.
+ * base > 1 (Qwen3 uses 1e6).  Positions are those of the WHOLE sequence.
+ */
+uly_status ulysses_rope_table(int32_t max_pos, int32_t head_dim, double base, float *table,
+                              void *stream);
+
+/*
+ * Steps 2-3 ("Paralelismul de Secvență Ulysses", section "Mecanismul de
+ * funcționare Ulysses"): every rank projects its own tokens,
+ *   [Q K V](t) = x(t) W_qkv^T,
+ * rotates Q and K by the token's position in the whole sequence (rank r's
+ * local token tt is at t = r*n/P + tt; the ms-swift page, section 6.2, names a
+ * rotation that ignores the shard's offset as the cause of repeated tokens),
+ * and writes the results directly in the head layout (the first all-to-all
+ * happens in the same kernel).  bf16 in and out, fp32 accumulation, one
+ * rounding.  Rotation: rotate-half pairing, element e with e + head_dim/2:
+ *   y[e] = x[e] cos - x[e+d/2] sin,  y[e+d/2] = x[e+d/2] cos + x[e] sin,
+ * cos/sin from `rope_table` (ulysses_rope_table) at the token's position.
+ *   x:      DEVICE bf16 seq layout [P][B][n/P][hidden]
+ *   w_qkv:  DEVICE bf16 [(H + 2G) * head_dim][hidden] (nn.Linear weight: H query
+ *           heads, then G key heads, then G value heads, head_dim rows each)
+ *   positions: NULL (position = t, needs max_pos >= n) or DEVICE int32 [B][n]
+ *           in sequence order (e.g. restarting at every packed document); a
+ *           position outside [0, max_pos) sets ULY_ERR_SHAPE in the error word
+ *           and that row is rotated as position 0
+ *   q:      DEVICE bf16 [P][B][H/P][n][head_dim];  k, v: [P][B][G/P][n][head_dim]
+ * Needs n % P == H % P == G % P == H % G == 0, head_dim == 128, H + 2G even,
+ * hidden % 64 == 0 (else ULY_ERR_SHAPE / ULY_ERR_UNSUPPORTED; with fewer KV
+ * heads than ranks, project K/V in the seq layout and use
+ * ulysses_kv_seq_to_head_replicated).  Outputs must not overlap any input or
+ * each other.
+ */
+uly_status ulysses_qkv_proj_rope(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden,
+                                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                 const void *x, const void *w_qkv, const float *rope_table,
+                                 int32_t max_pos, const int32_t *positions, void *q, void *k,
+                                 void *v, void *stream);
+
+/*
+ * Steps 5-6: the second all-to-all and the output projection in one kernel:
+ * the attention output is read in the head layout and every rank's tokens
+ * are projected,  y(t) = [O_0(t) ... O_{H-1}(t)] W_o^T.
+ *   o:   DEVICE bf16 [P][B][H/P][n][head_dim]
+ *   w_o: DEVICE bf16 [hidden][H * head_dim]
+ *   y:   DEVICE bf16 seq layout [P][B][n/P][hidden]
+ * bf16 in and out, fp32 accumulation, one rounding.  Needs n % P == H % P == 0,
+ * head_dim == 128, hidden % 256 == 0.  y must not overlap o or w_o.
+ */
+uly_status ulysses_o_proj(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden,
+                          int32_t n_q_heads, int32_t head_dim, const void *o, const void *w_o,
+                          void *y, void *stream);
+
+/*
  * Local attention (step 4) of every logical rank, head layout in and out:
  * q, o [P][B][H/P][n][d]; k, v [P][B][G/P][n][d]; lse [P][B][H/P][n] (fp32).
  * O = softmax(scale * Q K^T + mask) V per query head, LSE its log-sum-exp.

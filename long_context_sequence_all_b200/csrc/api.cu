@@ -59,6 +59,11 @@ uly_status kv_reduce_launch(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t
                             cudaStream_t);
 uly_status shift_labels_launch(int32_t, int32_t, int32_t, const int32_t *, const int32_t *, int32_t,
                                int32_t, int32_t, int32_t *, cudaStream_t);
+uly_status rope_table_launch(int32_t, int32_t, double, float *, cudaStream_t);
+uly_status qkv_proj_launch(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *, const void *,
+                           const float *, int32_t, const int32_t *, void *, void *, void *, cudaStream_t);
+uly_status o_proj_launch(int32_t, int32_t, int32_t, int32_t, int32_t, const void *, const void *, void *,
+                         cudaStream_t);
 size_t loss_workspace_bytes(int P, long long per_shard);
 size_t loss_bwd_workspace_bytes(int P, long long per_shard);
 uly_status loss_bwd_launch(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *, int32_t,
@@ -181,6 +186,67 @@ uly_status ulysses_shift_labels(int32_t batch, int32_t seq_len, int32_t world,
     return ULY_ERR_ALIAS;
   return shift_labels_launch(batch, seq_len, world, input_ids, cu_seqlens, num_docs, valid_len,
                              ignore_index, labels, static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_rope_table(int32_t max_pos, int32_t head_dim, double base, float *table,
+                              void *stream) {
+  if (!table) return ULY_ERR_NULL;
+  if (max_pos <= 0 || head_dim <= 0 || head_dim % 2) return ULY_ERR_SHAPE;
+  if (!(base > 1.0) || !std::isfinite(base)) return ULY_ERR_SHAPE;
+  if ((long long)max_pos * head_dim > (1LL << 40)) return ULY_ERR_SHAPE;
+  if (!aligned16(table)) return ULY_ERR_ALIGN;
+  return rope_table_launch(max_pos, head_dim, base, table, static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_qkv_proj_rope(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden,
+                                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                 const void *x, const void *w_qkv, const float *rope_table,
+                                 int32_t max_pos, const int32_t *positions, void *q, void *k,
+                                 void *v, void *stream) {
+  if (!x || !w_qkv || !rope_table || !q || !k || !v) return ULY_ERR_NULL;
+  if (batch <= 0 || seq_len <= 0 || world <= 0 || hidden <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 ||
+      head_dim <= 0 || max_pos <= 0)
+    return ULY_ERR_SHAPE;
+  if (seq_len % world || n_q_heads % world || n_q_heads % n_kv_heads) return ULY_ERR_SHAPE;
+  if (n_kv_heads % world) return ULY_ERR_UNSUPPORTED;  // fewer KV heads than ranks: project, then copy
+  if (head_dim != 128 || (n_q_heads + 2 * n_kv_heads) % 2 || hidden % 64) return ULY_ERR_UNSUPPORTED;
+  if (!positions && max_pos < seq_len) return ULY_ERR_SHAPE;
+  const long long M = (long long)batch * seq_len;
+  if ((M + 127) / 128 * ((n_q_heads + 2 * n_kv_heads) / 2) > 0x7fffffffLL) return ULY_ERR_SHAPE;
+  if (!all_aligned({x, w_qkv, rope_table, q, k, v})) return ULY_ERR_ALIGN;
+  const size_t xb = (size_t)M * hidden * 2, wb = (size_t)(n_q_heads + 2 * n_kv_heads) * head_dim * hidden * 2;
+  const size_t qb = (size_t)M * n_q_heads * head_dim * 2, kb = (size_t)M * n_kv_heads * head_dim * 2;
+  const size_t rb = (size_t)max_pos * head_dim * 4, pb = positions ? (size_t)M * 4 : 0;
+  const void *outs[3] = {q, k, v};
+  const size_t osz[3] = {qb, kb, kb};
+  for (int i = 0; i < 3; ++i) {
+    if (overlap(outs[i], osz[i], x, xb) || overlap(outs[i], osz[i], w_qkv, wb) ||
+        overlap(outs[i], osz[i], rope_table, rb) || (positions && overlap(outs[i], osz[i], positions, pb)))
+      return ULY_ERR_ALIAS;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], osz[i], outs[j], osz[j])) return ULY_ERR_ALIAS;
+  }
+  return qkv_proj_launch(batch, seq_len, world, hidden, n_q_heads, n_kv_heads, x, w_qkv, rope_table,
+                         max_pos, positions, q, k, v, static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_o_proj(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden,
+                          int32_t n_q_heads, int32_t head_dim, const void *o, const void *w_o,
+                          void *y, void *stream) {
+  if (!o || !w_o || !y) return ULY_ERR_NULL;
+  if (batch <= 0 || seq_len <= 0 || world <= 0 || hidden <= 0 || n_q_heads <= 0 || head_dim <= 0)
+    return ULY_ERR_SHAPE;
+  if (seq_len % world || n_q_heads % world) return ULY_ERR_SHAPE;
+  if (head_dim != 128 || hidden % 256) return ULY_ERR_UNSUPPORTED;
+  const long long tiles = (long long)batch * ((seq_len + 127) / 128) * (hidden / 256);
+  if (tiles > 0x7fffffffLL || (long long)world * batch * (n_q_heads / world) > 0x7fffffffLL)
+    return ULY_ERR_SHAPE;
+  if (!all_aligned({o, w_o, y})) return ULY_ERR_ALIGN;
+  const size_t ob = (size_t)batch * seq_len * n_q_heads * head_dim * 2;
+  const size_t wb = (size_t)hidden * n_q_heads * head_dim * 2, yb = (size_t)batch * seq_len * hidden * 2;
+  if (overlap(y, yb, o, ob) || overlap(y, yb, w_o, wb)) return ULY_ERR_ALIAS;
+  return o_proj_launch(batch, seq_len, world, hidden, n_q_heads, o, w_o, y,
+                       static_cast<cudaStream_t>(stream));
 }
 
 uly_status ulysses_attn_fwd(const uly_attn_desc *d, const void *q, const void *k, const void *v,

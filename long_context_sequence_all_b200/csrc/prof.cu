@@ -41,7 +41,8 @@ const char *name(int k) {
       "seq_to_head", "head_to_seq", "loss_partial", "loss_finalize", "attn_fwd_f32",
       "attn_dq_f32", "attn_dkdv_f32", "attn_bwd_dot", "attn_fwd_sm100", "attn_dkdv_sm100",
       "attn_dq_sm100", "attn_bwd_stats", "loss_fwd_bwd", "kv_seq_to_head_rep",
-      "kv_head_to_seq_sum", "shift_labels"};
+      "kv_head_to_seq_sum", "shift_labels", "rope_table", "qkv_proj_sm100",
+      "o_proj_sm100"};
   return (k >= 0 && k < K_COUNT) ? names[k] : "unknown";
 }
 

@@ -27,6 +27,9 @@ enum Kernel {
   K_KV_REPLICATE,
   K_KV_REDUCE,
   K_SHIFT_LABELS,
+  K_ROPE_TABLE,
+  K_QKV_PROJ,
+  K_O_PROJ,
   K_COUNT
 };
 

@@ -1,0 +1,394 @@
+// The projections either side of Ulysses attention, on the 5th-generation
+// tensor cores ("Paralelismul de Secvență Ulysses", section "Mecanismul de
+// funcționare Ulysses", steps 2-3 and 5-6):
+//
+//  QKV: every rank projects its own tokens, [Q K V] = X W^T, rotates Q and K by
+//  each token's position in the whole sequence (rank r's local token tt sits at
+//  t = r*n/P + tt; the ms-swift page, section 6.2, lists a RoPE that ignores the
+//  shard's offset as a failure), and the first all-to-all is folded into the
+//  epilogue: every output row is written straight to its place in the head
+//  layout, so the projected Q/K/V never exist in the seq layout.
+//
+//  O-proj: the second all-to-all is folded into the operand load: a CTA's A
+//  tile (128 positions x 64 features of one head) is read by TMA directly from
+//  the head layout, and Y = O W_o^T is written in the seq layout.
+//
+// Both are C[M][N] = A[M][K] B[N][K]^T with bf16 operands and fp32
+// accumulation, tiles of 128 x 256 (two heads of 128 columns for QKV), K in
+// 64-column steps (one 128-byte swizzle span).  The kernel is persistent:
+// one CTA per SM walks the tiles (N fastest, so CTAs running at the same time
+// share their A rows in L2).
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer: A and B k-steps into a 4-stage ring (48 KB each)
+//   warp 1     TMEM allocator and MMA issuer: 4 MMAs (M=128 N=256 K=16) per
+//              stage into one of two 256-column accumulators
+//   warps 2-5  epilogue: one thread per accumulator row (TMEM lane) reads its
+//              row, applies the rotation (QKV), rounds to bf16 and stores;
+//              the other accumulator is filled by the next tile meanwhile.
+// Every wait is bounded (ULY_ERR_TIMEOUT); nothing can spin forever.
+#include "prof.cuh"
+#include "sm100.cuh"
+
+namespace uly {
+
+using namespace sm100;
+
+bool make_tmap_heads_bf16(CUtensorMap *map, const void *base, int d, int n, int heads, int box_rows);
+bool make_tmap_rows_bf16(CUtensorMap *map, const void *base, long long inner, long long rows, int box_inner,
+                         int box_rows);
+
+namespace {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kHD = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
+constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
+constexpr uint32_t kOffBar = kStages * kStageBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // barriers + alignment slack
+constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kBM, kBN, false, false);
+
+enum Mode { MODE_QKV = 0, MODE_OPROJ = 1 };
+
+struct ProjParams {
+  int mode;
+  int K;             // reduction length (hidden for QKV, H*d for the output projection)
+  int m_tiles, n_tiles;
+  int B, n, s, P;
+  int hl, gl, H, G;  // query / KV heads per rank and in total
+  long long M;       // QKV: rows of X (P*B*s)
+  int hidden;        // output projection: width of Y
+  int tiles_per_b;   // output projection: position tiles per batch row
+  const float4 *rope;        // [max_pos][32] float4 = (cos e, sin e, cos e+1, sin e+1)
+  int max_pos;
+  const int32_t *positions;  // nullable [B][n]
+  __nv_bfloat16 *q, *k, *v;  // QKV outputs, head layout
+  __nv_bfloat16 *y;          // output projection result, seq layout
+  int *err;
+};
+
+__device__ __forceinline__ void store_row_chunk(__nv_bfloat16 *dst, const float (&x)[32]) {
+  uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint4 w;
+    w.x = pack_bf16x2(x[8 * u + 0], x[8 * u + 1]);
+    w.y = pack_bf16x2(x[8 * u + 2], x[8 * u + 3]);
+    w.z = pack_bf16x2(x[8 * u + 4], x[8 * u + 5]);
+    w.w = pack_bf16x2(x[8 * u + 6], x[8 * u + 7]);
+    d4[u] = w;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    proj_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const ProjParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  enum { B_FULL = 0, B_EMPTY = kStages, B_ACCF = 2 * kStages, B_ACCE = B_ACCF + 2, B_DRAIN = B_ACCE + 2,
+         B_N = B_DRAIN + 1 };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = prm.m_tiles * prm.n_tiles;
+  const int KT = prm.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_ACCE || i == B_ACCE + 1) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      long long idx = 0;   // k-steps issued so far (ring position)
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        const int mt = tile / prm.n_tiles, nt = tile - mt * prm.n_tiles;
+        const int n0 = nt * kBN;
+        int b = 0, t0 = 0;
+        if (prm.mode == MODE_OPROJ) {
+          b = mt / prm.tiles_per_b;
+          t0 = (mt - b * prm.tiles_per_b) * kBM;
+        }
+        for (int kt = 0; kt < KT; ++kt, ++idx) {
+          const int stage = (int)(idx % kStages);
+          const long long use = idx / kStages;
+          if (use > 0 && !mbar_wait(bar(B_EMPTY + stage), (uint32_t)((use - 1) & 1), abort_flag, prm.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sA = sb + stage * kStageBytes, sB = sA + kABytes;
+          mbar_arrive_expect_tx(bar(B_FULL + stage), kStageBytes);
+          if (prm.mode == MODE_QKV) {
+            tma_load_2d(sA, &tmA, bar(B_FULL + stage), kt * kBK, mt * kBM);
+          } else {
+            // k-step kt covers features [64 (kt % 2), +64) of query head kt / 2,
+            // held by rank kt / 2 / hl as its local head (kt / 2) % hl
+            const int qh = kt >> 1, r2 = qh / prm.hl, hh = qh - r2 * prm.hl;
+            tma_load_3d(sA, &tmA, bar(B_FULL + stage), (kt & 1) * kBK, t0, (r2 * prm.B + b) * prm.hl + hh);
+          }
+          tma_load_2d(sB, &tmB, bar(B_FULL + stage), kt * kBK, n0);
+        }
+      }
+      if (!ok) {
+        // let the copies already in flight land before the CTA exits
+        for (long long j = (idx > kStages ? idx - kStages : 0); j < idx; ++j)
+          mbar_wait(bar(B_FULL + (int)(j % kStages)), (uint32_t)((j / kStages) & 1), nullptr, prm.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      long long idx = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        if (it >= 2) {
+          ok = mbar_wait(bar(B_ACCE + buf), (uint32_t)(((it >> 1) - 1) & 1), abort_flag, prm.err);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint32_t acc = tmem + buf * kBN;
+        for (int kt = 0; kt < KT; ++kt, ++idx) {
+          const int stage = (int)(idx % kStages);
+          const uint32_t sA = sb + stage * kStageBytes, sB = sA + kABytes;
+          const uint64_t da = sdesc_sw128(sA, 16, 1024), db = sdesc_sw128(sB, 16, 1024);
+          ok = mbar_wait(bar(B_FULL + stage), (uint32_t)((idx / kStages) & 1), abort_flag, prm.err);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16_ss(acc, sdesc_add(da, kk * 32), sdesc_add(db, kk * 32), kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(B_EMPTY + stage));
+        }
+        if (!ok) break;
+        tc_commit(bar(B_ACCF + buf));
+      }
+      if (!ok) {
+        // drain: wait for every MMA issued so far before TMEM is released
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int wq = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ACCF + buf), (uint32_t)((it >> 1) & 1), abort_flag, prm.err)))
+        break;
+      tc_fence_after();
+      const int mt = tile / prm.n_tiles, nt = tile - mt * prm.n_tiles;
+      const uint32_t acc = tmem + lane_off + buf * kBN;
+      if (prm.mode == MODE_QKV) {
+        const long long m = (long long)mt * kBM + row;
+        const bool valid = m < prm.M;
+        int b = 0, t = 0, pos = 0;
+        if (valid) {
+          const long long bs = (long long)prm.B * prm.s;
+          const int r = (int)(m / bs);
+          const long long rem = m - (long long)r * bs;
+          b = (int)(rem / prm.s);
+          const int tt = (int)(rem - (long long)b * prm.s);
+          t = r * prm.s + tt;
+          pos = prm.positions ? __ldg(prm.positions + (long long)b * prm.n + t) : t;
+          if (pos < 0 || pos >= prm.max_pos) {
+            raise_error(prm.err, ULY_ERR_SHAPE);
+            pos = 0;
+          }
+        }
+#pragma unroll 1
+        for (int hs = 0; hs < 2; ++hs) {
+          const int j = nt * 2 + hs;         // output head: H query, G key, G value heads
+          __nv_bfloat16 *base;
+          int heads_local, jj;
+          if (j < prm.H) { base = prm.q; heads_local = prm.hl; jj = j; }
+          else if (j < prm.H + prm.G) { base = prm.k; heads_local = prm.gl; jj = j - prm.H; }
+          else { base = prm.v; heads_local = prm.gl; jj = j - prm.H - prm.G; }
+          const bool rot = j < prm.H + prm.G;
+          const int r2 = jj / heads_local, hh = jj - r2 * heads_local;
+          __nv_bfloat16 *dst = base + ((((long long)r2 * prm.B + b) * heads_local + hh) * prm.n + t) * kHD;
+#pragma unroll 1
+          for (int c0 = 0; c0 < kHD / 2; c0 += 32) {
+            uint32_t a1[32], a2[32];
+            tmem_ld32(acc + hs * kHD + c0, a1);
+            tmem_ld32(acc + hs * kHD + kHD / 2 + c0, a2);
+            float y1[32], y2[32];
+            if (rot) {
+              const float4 *cs = prm.rope + (long long)pos * (kHD / 4) + c0 / 2;
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float4 w = __ldg(cs + e / 2);
+                const float x1a = __uint_as_float(a1[e]), x2a = __uint_as_float(a2[e]);
+                const float x1b = __uint_as_float(a1[e + 1]), x2b = __uint_as_float(a2[e + 1]);
+                y1[e] = x1a * w.x - x2a * w.y;
+                y2[e] = x2a * w.x + x1a * w.y;
+                y1[e + 1] = x1b * w.z - x2b * w.w;
+                y2[e + 1] = x2b * w.z + x1b * w.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                y1[e] = __uint_as_float(a1[e]);
+                y2[e] = __uint_as_float(a2[e]);
+              }
+            }
+            if (valid) {
+              store_row_chunk(dst + c0, y1);
+              store_row_chunk(dst + kHD / 2 + c0, y2);
+            }
+          }
+        }
+      } else {
+        const int b = mt / prm.tiles_per_b;
+        const int t = (mt - b * prm.tiles_per_b) * kBM + row;
+        const bool valid = t < prm.n;
+        const int r = valid ? t / prm.s : 0, tt = valid ? t - r * prm.s : 0;
+        __nv_bfloat16 *dst = prm.y + (((long long)r * prm.B + b) * prm.s + tt) * prm.hidden + nt * kBN;
+#pragma unroll 1
+        for (int c = 0; c < kBN; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(acc + c, a);
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(a[e]);
+          if (valid) store_row_chunk(dst + c, x);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_ACCE + buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// cos / sin of position p times base^(-2e/d), computed in double and rounded
+// once to float; laid out [p][e/2] as float4 (cos e, sin e, cos e+1, sin e+1).
+__global__ void rope_table_kernel(int max_pos, int half, double base, float *table) {
+  const long long total = (long long)max_pos * half;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int p = (int)(i / half), e = (int)(i - (long long)p * half);
+    const double theta = pow(base, -2.0 * e / (2.0 * half));
+    double sn, cs;
+    sincos((double)p * theta, &sn, &cs);
+    table[2 * i] = (float)cs;
+    table[2 * i + 1] = (float)sn;
+  }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 148;
+  }
+  return n;
+}
+
+uly_status launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const ProjParams &prm, int kernel_id,
+                       cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return ULY_ERR_CUDA;
+    attr_set = true;
+  }
+  const int ntiles = prm.m_tiles * prm.n_tiles;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  prof::Scope scope(kernel_id, stream);
+  proj_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, prm);
+  note_launches(1);
+  return last_launch_status();
+}
+
+}  // namespace
+
+uly_status rope_table_launch(int32_t max_pos, int32_t head_dim, double base, float *table, cudaStream_t stream) {
+  const long long total = (long long)max_pos * (head_dim / 2);
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148LL * 32) blocks = 148LL * 32;
+  prof::Scope scope(prof::K_ROPE_TABLE, stream);
+  rope_table_kernel<<<(unsigned)blocks, 256, 0, stream>>>(max_pos, head_dim / 2, base, table);
+  note_launches(1);
+  return last_launch_status();
+}
+
+uly_status qkv_proj_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int32_t H, int32_t G,
+                           const void *x, const void *w, const float *rope, int32_t max_pos,
+                           const int32_t *positions, void *q, void *k, void *v, cudaStream_t stream) {
+  const long long M = (long long)B * n;
+  const long long N = (long long)(H + 2 * G) * kHD;
+  CUtensorMap ta, tb;
+  if (!make_tmap_rows_bf16(&ta, x, hidden, M, kBK, kBM) || !make_tmap_rows_bf16(&tb, w, hidden, N, kBK, kBN))
+    return ULY_ERR_CUDA;
+  ProjParams prm = {};
+  prm.mode = MODE_QKV;
+  prm.K = hidden;
+  prm.m_tiles = (int)((M + kBM - 1) / kBM);
+  prm.n_tiles = (int)(N / kBN);
+  prm.B = B; prm.n = n; prm.s = n / P; prm.P = P;
+  prm.H = H; prm.G = G; prm.hl = H / P; prm.gl = G / P;
+  prm.M = M;
+  prm.rope = reinterpret_cast<const float4 *>(rope);
+  prm.max_pos = max_pos;
+  prm.positions = positions;
+  prm.q = static_cast<__nv_bfloat16 *>(q);
+  prm.k = static_cast<__nv_bfloat16 *>(k);
+  prm.v = static_cast<__nv_bfloat16 *>(v);
+  prm.err = error_word();
+  return launch_proj(ta, tb, prm, prof::K_QKV_PROJ, stream);
+}
+
+uly_status o_proj_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int32_t H, const void *o,
+                         const void *w, void *y, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!make_tmap_heads_bf16(&ta, o, kHD, n, P * B * (H / P), kBM) ||
+      !make_tmap_rows_bf16(&tb, w, (long long)H * kHD, hidden, kBK, kBN))
+    return ULY_ERR_CUDA;
+  ProjParams prm = {};
+  prm.mode = MODE_OPROJ;
+  prm.K = H * kHD;
+  prm.tiles_per_b = (n + kBM - 1) / kBM;
+  prm.m_tiles = B * prm.tiles_per_b;
+  prm.n_tiles = hidden / kBN;
+  prm.B = B; prm.n = n; prm.s = n / P; prm.P = P;
+  prm.H = H; prm.hl = H / P;
+  prm.hidden = hidden;
+  prm.y = static_cast<__nv_bfloat16 *>(y);
+  prm.err = error_word();
+  return launch_proj(ta, tb, prm, prof::K_O_PROJ, stream);
+}
+
+}  // namespace uly

@@ -24,7 +24,8 @@ STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE"
           4: "ULY_ERR_ALIGN", 5: "ULY_ERR_ALIAS", 6: "ULY_ERR_UNSUPPORTED", 7: "ULY_ERR_CUDA",
           8: "ULY_ERR_LABEL", 9: "ULY_ERR_TIMEOUT", 10: "ULY_ERR_WORKSPACE"}
 EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head_replicated",
-           "ulysses_kv_head_to_seq_reduce", "ulysses_shift_labels", "ulysses_attn_fwd",
+           "ulysses_kv_head_to_seq_reduce", "ulysses_shift_labels", "ulysses_rope_table",
+           "ulysses_qkv_proj_rope", "ulysses_o_proj", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
            "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
            "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info",
@@ -67,8 +68,13 @@ def lib() -> ctypes.CDLL:
             L.ulysses_kv_seq_to_head_replicated.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
             L.ulysses_kv_head_to_seq_reduce.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
             L.ulysses_shift_labels.argtypes = [i32, i32, i32, vp, vp, i32, i32, i32, vp, vp]
+            L.ulysses_rope_table.argtypes = [i32, i32, ctypes.c_double, vp, vp]
+            L.ulysses_qkv_proj_rope.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32, vp,
+                                                vp, vp, vp, vp]
+            L.ulysses_o_proj.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
             for name in ("ulysses_kv_seq_to_head_replicated", "ulysses_kv_head_to_seq_reduce",
-                         "ulysses_shift_labels"):
+                         "ulysses_shift_labels", "ulysses_rope_table", "ulysses_qkv_proj_rope",
+                         "ulysses_o_proj"):
                 getattr(L, name).restype = ctypes.c_int
             D = ctypes.POINTER(AttnDesc)
             L.ulysses_attn_fwd.argtypes = [D, vp, vp, vp, vp, vp, vp]
@@ -204,6 +210,50 @@ def ulysses_shift_labels(input_ids: torch.Tensor, P: int, cu_seqlens: torch.Tens
     _check(lib().ulysses_shift_labels(B, n, P, _p(input_ids), _p(cu_seqlens), nd, vl, ignore_index,
                                       _p(out), _stream(stream)), "ulysses_shift_labels")
     return out
+
+
+# --------------------------------------------------------------- projections
+
+def ulysses_rope_table(max_pos: int, head_dim: int = 128, base: float = 1.0e6, out=None, device=None,
+                       stream=None):
+    """(cos, sin) of p * base^(-2e/d) for p < max_pos, e < d/2: float32 [max_pos][d/2][2]."""
+    if out is None:
+        out = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device or "cuda")
+    _check(lib().ulysses_rope_table(max_pos, head_dim, float(base), _p(out), _stream(stream)),
+           "ulysses_rope_table")
+    return out
+
+
+def ulysses_qkv_proj_rope(x: torch.Tensor, w_qkv: torch.Tensor, P: int, H: int, G: int,
+                          rope_table: torch.Tensor, positions: torch.Tensor | None = None,
+                          q=None, k=None, v=None, stream=None):
+    """x seq layout [P][B][n/P][hidden] (bf16), w_qkv [(H+2G)*128][hidden] ->
+    q [P][B][H/P][n][128], k, v [P][B][G/P][n][128] (rotated Q, K; head layout)."""
+    P_, B, s, hidden = x.shape
+    n, d = P * s, 128
+    if P_ != P:
+        raise UlyssesError(2, f"ulysses_qkv_proj_rope: x {tuple(x.shape)} with P={P}")
+    dev = x.device
+    q = torch.empty((P, B, H // P, n, d), dtype=x.dtype, device=dev) if q is None else q
+    k = torch.empty((P, B, max(G // P, 1), n, d), dtype=x.dtype, device=dev) if k is None else k
+    v = torch.empty_like(k) if v is None else v
+    _check(lib().ulysses_qkv_proj_rope(B, n, P, hidden, H, G, d, _p(x), _p(w_qkv), _p(rope_table),
+                                       rope_table.shape[0], _p(positions), _p(q), _p(k), _p(v),
+                                       _stream(stream)), "ulysses_qkv_proj_rope")
+    return q, k, v
+
+
+def ulysses_o_proj(o: torch.Tensor, w_o: torch.Tensor, P: int, y=None, stream=None):
+    """o head layout [P][B][H/P][n][128] (bf16), w_o [hidden][H*128] -> y seq
+    layout [P][B][n/P][hidden]."""
+    P_, B, hl, n, d = o.shape
+    hidden = w_o.shape[0]
+    if P_ != P:
+        raise UlyssesError(2, f"ulysses_o_proj: o {tuple(o.shape)} with P={P}")
+    y = torch.empty((P, B, n // P, hidden), dtype=o.dtype, device=o.device) if y is None else y
+    _check(lib().ulysses_o_proj(B, n, P, hidden, hl * P, d, _p(o), _p(w_o), _p(y), _stream(stream)),
+           "ulysses_o_proj")
+    return y
 
 
 # ----------------------------------------------------------------- attention

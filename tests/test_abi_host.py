@@ -88,6 +88,34 @@ def test_shift_labels_validation(L):
     assert f(1, 1024, 4, ids, vp((1 << 30) + 64), 2, 1024, -100, lab, None) == 5  # cu inside labels
 
 
+def test_projection_validation(L):
+    vp = ctypes.c_void_p
+    x, w, tab, q, k, v = (vp(1 << (30 + i)) for i in range(6))
+    f = L.ulysses_qkv_proj_rope
+    args = lambda **kw: [kw.get("B", 1), kw.get("n", 8192), kw.get("P", 4), kw.get("hidden", 2560),
+                         kw.get("H", 32), kw.get("G", 8), kw.get("d", 128), x, w, tab,
+                         kw.get("max_pos", 8192), None, q, k, v, None]
+    assert f(*args(n=8190)) == 2                       # n % P
+    assert f(*args(G=2)) == 6                          # fewer KV heads than ranks: not fused
+    assert f(*args(d=64)) == 6
+    assert f(*args(hidden=2500)) == 6                  # hidden % 64
+    assert f(*args(max_pos=100)) == 2                  # table shorter than the sequence
+    a = args()
+    a[12] = vp((1 << 30) + 64)                         # q inside x
+    assert f(*a) == 5
+    a = args()
+    a[7] = None
+    assert f(*a) == 1
+    g = L.ulysses_o_proj
+    assert g(1, 8192, 4, 2500, 32, 128, x, w, q, None) == 6           # hidden % 256
+    assert g(1, 8190, 4, 2560, 32, 128, x, w, q, None) == 2
+    assert g(1, 8192, 4, 2560, 32, 128, x, w, vp((1 << 30) + 16), None) == 5
+    assert L.ulysses_rope_table(0, 128, 1e6, tab, None) == 2
+    assert L.ulysses_rope_table(8192, 127, 1e6, tab, None) == 2
+    assert L.ulysses_rope_table(8192, 128, 0.5, tab, None) == 2
+    assert L.ulysses_rope_table(8192, 128, 1e6, vp((1 << 30) + 4), None) == 4
+
+
 def test_attn_desc_validation(L):
     from long_context_sequence_all_b200 import ulysses as U
     n = ctypes.c_size_t(0)
