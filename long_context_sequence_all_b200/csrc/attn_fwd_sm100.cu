@@ -375,23 +375,6 @@ bool make_tmap_heads_bf16(CUtensorMap *map, const void *base, int d, int n, int 
   return r == CUDA_SUCCESS;
 }
 
-// 2-D bf16 map over a row-major [rows][inner] matrix with box_inner x
-// box_rows boxes (box_inner * 2 = 128 bytes: one 128-byte swizzle span);
-// elements past either edge read as zero.
-bool make_tmap_rows_bf16(CUtensorMap *map, const void *base, long long inner, long long rows,
-                         int box_inner, int box_rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
-  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const MaskInfo &mk,
                                 const void *q, const void *k, const void *v, void *o, float *lse,
                                 cudaStream_t stream) {
