@@ -27,6 +27,8 @@
 //              row, applies the rotation (QKV), rounds to bf16 and stores;
 //              the other accumulator is filled by the next tile meanwhile.
 // Every wait is bounded (ULY_ERR_TIMEOUT); nothing can spin forever.
+#include <atomic>
+
 #include "prof.cuh"
 #include "sm100.cuh"
 
@@ -338,27 +340,24 @@ __global__ void rope_table_kernel(int max_pos, int half, double base, float *tab
   }
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n = 148;
-  }
-  return n;
-}
-
 uly_status launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const ProjParams &prm, int kernel_id,
                        cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory opt-in is a per-device attribute: set it once on every
+  // device this process launches on
+  static std::atomic<uint64_t> attr_devices{0};
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return ULY_ERR_CUDA;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (!bit || !(attr_devices.load(std::memory_order_acquire) & bit)) {
     if (cudaFuncSetAttribute(proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
       return ULY_ERR_CUDA;
-    attr_set = true;
+    attr_devices.fetch_or(bit, std::memory_order_acq_rel);
   }
   const int ntiles = prm.m_tiles * prm.n_tiles;
-  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  const int grid = ntiles < sms ? ntiles : sms;
   prof::Scope scope(kernel_id, stream);
   proj_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, prm);
   note_launches(1);

@@ -201,7 +201,7 @@ def ulysses_shift_labels(input_ids: torch.Tensor, P: int, cu_seqlens: torch.Tens
     """Next-token labels of input_ids [B][n] (int32), shifted before sharding:
     returns the seq layout [P][B][n/P] (int32)."""
     B, n = input_ids.shape
-    if input_ids.dtype != torch.int32 or n % P:
+    if input_ids.dtype != torch.int32 or n % P or (cu_seqlens is not None and cu_seqlens.dtype != torch.int32):
         raise UlyssesError(2, f"ulysses_shift_labels: ids {tuple(input_ids.shape)} {input_ids.dtype} with P={P}")
     nd = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     if out is None:
@@ -231,8 +231,12 @@ def ulysses_qkv_proj_rope(x: torch.Tensor, w_qkv: torch.Tensor, P: int, H: int, 
     q [P][B][H/P][n][128], k, v [P][B][G/P][n][128] (rotated Q, K; head layout)."""
     P_, B, s, hidden = x.shape
     n, d = P * s, 128
-    if P_ != P:
-        raise UlyssesError(2, f"ulysses_qkv_proj_rope: x {tuple(x.shape)} with P={P}")
+    if P_ != P or tuple(w_qkv.shape) != ((H + 2 * G) * d, hidden):
+        raise UlyssesError(2, f"ulysses_qkv_proj_rope: x {tuple(x.shape)}, w {tuple(w_qkv.shape)} with P={P}")
+    if rope_table.dtype != torch.float32 or rope_table.dim() != 3 or tuple(rope_table.shape[1:]) != (d // 2, 2):
+        raise UlyssesError(2, f"ulysses_qkv_proj_rope: rope table {tuple(rope_table.shape)} {rope_table.dtype}")
+    if positions is not None and (positions.dtype != torch.int32 or tuple(positions.shape) != (B, n)):
+        raise UlyssesError(2, f"ulysses_qkv_proj_rope: positions {tuple(positions.shape)} {positions.dtype}")
     dev = x.device
     q = torch.empty((P, B, H // P, n, d), dtype=x.dtype, device=dev) if q is None else q
     k = torch.empty((P, B, max(G // P, 1), n, d), dtype=x.dtype, device=dev) if k is None else k
@@ -248,8 +252,8 @@ def ulysses_o_proj(o: torch.Tensor, w_o: torch.Tensor, P: int, y=None, stream=No
     layout [P][B][n/P][hidden]."""
     P_, B, hl, n, d = o.shape
     hidden = w_o.shape[0]
-    if P_ != P:
-        raise UlyssesError(2, f"ulysses_o_proj: o {tuple(o.shape)} with P={P}")
+    if P_ != P or tuple(w_o.shape) != (hidden, hl * P * d):
+        raise UlyssesError(2, f"ulysses_o_proj: o {tuple(o.shape)}, w_o {tuple(w_o.shape)} with P={P}")
     y = torch.empty((P, B, n // P, hidden), dtype=o.dtype, device=o.device) if y is None else y
     _check(lib().ulysses_o_proj(B, n, P, hidden, hl * P, d, _p(o), _p(w_o), _p(y), _stream(stream)),
            "ulysses_o_proj")
