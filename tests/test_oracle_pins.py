@@ -705,3 +705,45 @@ def test_output_projection_matches_torch_linear():
     o_nat = o_head.transpose(1, 3, 0, 2, 4).reshape(B, n, H * d)        # heads r*H/P + hh in order
     ref = F.linear(torch.from_numpy(o_nat), torch.from_numpy(w)).numpy()
     assert np.abs(y.transpose(1, 0, 2, 3).reshape(B, n, hidden) - ref).max() < 1e-12
+
+
+@pytest.mark.parametrize("P,H,G", [(4, 8, 4), (4, 8, 2), (2, 4, 2)])
+def test_whole_layer_sharded_equals_plain_layer(P, H, G):
+    """Steps 1-6 composed (shard, project and rotate at global positions,
+    first all-to-all -- copying KV heads when G < P --, per-rank attention,
+    second all-to-all, output projection) equal the plain single-device layer
+    written with torch float64 library calls: linear, the rotation as a complex
+    multiplication, scaled_dot_product_attention with GQA, linear."""
+    B, n, hidden, d = 1, 32, 24, 8
+    x = rng.standard_normal((B, n, hidden))
+    w = rng.standard_normal(((H + 2 * G) * d, hidden)) / np.sqrt(hidden)
+    wo = rng.standard_normal((hidden, H * d)) / np.sqrt(H * d)
+    x_seq = x.reshape(B, P, n // P, hidden).transpose(1, 0, 2, 3)
+    qh, kh, vh = oracle.qkv_proj_rope(x_seq, w, P, H, G, d)
+    if G % P == 0:
+        k_seq, v_seq = oracle.head_to_seq(kh, B, n, P, G), oracle.head_to_seq(vh, B, n, P, G)
+    else:   # recover the G heads from their copies (rank r holds head r*G/P)
+        k_seq = np.stack([kh[g * (P // G), :, 0] for g in range(G)], 2)       # [B][n][G][d]
+        v_seq = np.stack([vh[g * (P // G), :, 0] for g in range(G)], 2)
+        k_seq, v_seq = (z.reshape(B, P, n // P, G, d).transpose(1, 0, 2, 3, 4) for z in (k_seq, v_seq))
+    q_seq = oracle.head_to_seq(qh, B, n, P, H)
+    o_seq, _ = oracle.ulysses_fwd(q_seq.astype(np.float32), k_seq.astype(np.float32),
+                                  v_seq.astype(np.float32), P)
+    y = oracle.o_proj(oracle.seq_to_head(o_seq, B, n, P, H), wo, P)          # [P][B][s][hidden]
+    # plain layer in torch float64 (inputs rounded to fp32 where the oracle's attention reads fp32)
+    xt, wt, wot = (torch.from_numpy(a) for a in (x, w, wo))
+    proj = F.linear(xt, wt).reshape(B, n, H + 2 * G, d)
+    half = d // 2
+    ang = torch.arange(n, dtype=torch.float64)[:, None] * 1.0e6 ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)
+    rot = torch.polar(torch.ones_like(ang), ang)                                # e^{i angle}
+
+    def rope_t(z):
+        c = torch.complex(z[..., :half], z[..., half:]) * rot[None, :, None, :]
+        return torch.cat([c.real, c.imag], -1)
+    q, k, v = rope_t(proj[:, :, :H]), rope_t(proj[:, :, H:H + G]), proj[:, :, H + G:]
+    f32 = lambda z: z.float().double()
+    o = F.scaled_dot_product_attention(f32(q).transpose(1, 2), f32(k).transpose(1, 2), f32(v).transpose(1, 2),
+                                       is_causal=True, enable_gqa=True).transpose(1, 2).reshape(B, n, H * d)
+    ref = F.linear(o, wot).numpy()
+    got = y.transpose(1, 0, 2, 3).reshape(B, n, hidden)
+    assert np.abs(got - ref).max() < 1e-9
