@@ -132,6 +132,15 @@ class Layer:
                                           shard_sum=self.S, shard_count=self.C, loss=self.L,
                                           workspace=self.lbws)
 
+    def fwd_step(self):
+        """The forward half alone: seq->head(Q, K, V), attention forward, head->seq(O)."""
+        U, P = self.U, self.P
+        U.ulysses_seq_to_head(self.q, P, out=self.qh)
+        U.ulysses_seq_to_head(self.k, P, out=self.kh)
+        U.ulysses_seq_to_head(self.v, P, out=self.vh)
+        U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.oh, lse=self.lse)
+        U.ulysses_head_to_seq(self.oh, P, out=self.o)
+
     def step(self):
         U, P = self.U, self.P
         U.ulysses_seq_to_head(self.q, P, out=self.qh)
@@ -353,6 +362,24 @@ def run_ours(args, rank, world, dev):
     _barrier(world)
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
 
+    # the forward half alone (seq->head(Q,K,V), attention forward, head->seq(O)),
+    # this rank's device time; a failure here only records the error
+    fwd_only = None
+    try:
+        for _ in range(2):
+            layer.fwd_step()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            layer.fwd_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        fms = e0.elapsed_time(e1) / args.steps
+        fwd_only = {"ms_per_step": fms, "tokens_per_s": inp["B"] * inp["n"] / (fms / 1e3),
+                    "note": "seq->head(Q,K,V) + attention forward + head->seq(O); this rank alone"}
+    except Exception as exc:  # noqa: BLE001 -- a side figure never breaks the bench line
+        fwd_only = {"error": str(exc)[:200]}
+
     # the fused loss + gradient, timed on its own (it follows the layer's loss
     # in training and is not part of the layer step)
     loss_bwd = None
@@ -437,6 +464,7 @@ def run_ours(args, rank, world, dev):
         "permute_gbs": {k: kernels[k]["gbs"] for k in ("seq_to_head", "head_to_seq") if k in kernels},
         "roofline": roof,
         "kernels": kernels,
+        "forward_only": fwd_only,
         "loss_grad": loss_bwd,
         "side_kernels": side,
         "gpu_launches": launches,
