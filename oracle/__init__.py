@@ -373,3 +373,49 @@ def o_proj(o_head, w_o, P):
     w = np.asarray(w_o, np.float64)
     y = o_seq.reshape(P * B * (n // P), H * d) @ w.T
     return y.reshape(P, B, n // P, w.shape[0])
+
+
+def qkv_proj_rope_bwd(x_seq, w_qkv, dq_head, dk_head, dv_head, P, H, G, d, base=1.0e6, positions=None):
+    """Backward of qkv_proj_rope (the adjoint of steps 2-3): the gradients of
+    the rotated Q, K and of V go back through the all-to-all (head -> seq; the
+    copies of a KV head are summed when G < P), through the rotation (its
+    transpose: the same rotation by -pos), and through the projection:
+        dY(t) = [R(-pos) dQ(t) | R(-pos) dK(t) | dV(t)],
+        dX_r = dY_r W,   dW = sum over ranks of dY_r^T X_r.
+    Returns dx_seq [P][B][s][hidden] and dw [(H+2G)*d][hidden] (fp64)."""
+    x = np.asarray(x_seq, np.float64)
+    w = np.asarray(w_qkv, np.float64)
+    P_, B, s, hidden = x.shape
+    n = P * s
+    _check_ulysses(n, P, H, G)
+    dq = head_to_seq(np.asarray(dq_head, np.float64), B, n, P, H)              # [P][B][s][H][d]
+    if G % P == 0:
+        dk = head_to_seq(np.asarray(dk_head, np.float64), B, n, P, G)
+        dv = head_to_seq(np.asarray(dv_head, np.float64), B, n, P, G)
+    else:
+        dk = kv_reduce_to_seq(dk_head, B, n, P, G)
+        dv = kv_reduce_to_seq(dv_head, B, n, P, G)
+    dx = np.empty_like(x)
+    dw = np.zeros_like(w)
+    for r in range(P):
+        t = r * s + np.arange(s)
+        pos = np.broadcast_to(t, (B, s)) if positions is None else np.asarray(positions)[:, t]
+        dy = np.concatenate([rope(dq[r], -pos[:, :, None], base), rope(dk[r], -pos[:, :, None], base), dv[r]],
+                            axis=2).reshape(B * s, (H + 2 * G) * d)
+        dx[r] = (dy @ w).reshape(B, s, hidden)
+        dw += dy.T @ x[r].reshape(B * s, hidden)
+    return dx, dw
+
+
+def o_proj_bwd(o_head, w_o, dy_seq, P):
+    """Backward of o_proj (the adjoint of steps 5-6): dO_seq = dY W_o, back to
+    the head layout by the first all-to-all; dW_o = sum over ranks of
+    dY_r^T O_r.  Returns do_head [P][B][H/P][n][d] and dw_o [hidden][H*d] (fp64)."""
+    o = np.asarray(o_head, np.float64)
+    P_, B, hl, n, d = o.shape
+    H = hl * P
+    w = np.asarray(w_o, np.float64)
+    dy = np.asarray(dy_seq, np.float64).reshape(P * B * (n // P), w.shape[0])
+    o_seq = head_to_seq(o, B, n, P, H).reshape(P * B * (n // P), H * d)
+    do_seq = (dy @ w).reshape(P, B, n // P, H, d)
+    return seq_to_head(do_seq, B, n, P, H), dy.T @ o_seq

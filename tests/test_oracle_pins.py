@@ -747,3 +747,86 @@ def test_whole_layer_sharded_equals_plain_layer(P, H, G):
     ref = F.linear(o, wot).numpy()
     got = y.transpose(1, 0, 2, 3).reshape(B, n, hidden)
     assert np.abs(got - ref).max() < 1e-9
+
+
+def _torch_layer_proj(x_nat, w, H, G, d, P, pos, base=1.0e6):
+    """Forward of the QKV projection in torch float64, laid out in the head
+    layout with torch reshapes (independent of the oracle's index loops)."""
+    B, n, hidden = x_nat.shape
+    y = F.linear(x_nat, w).reshape(B, n, H + 2 * G, d)
+    half = d // 2
+    ang = pos[..., None] * base ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)   # [B][n][half]
+    rot = torch.polar(torch.ones_like(ang), ang)[:, :, None, :]
+
+    def rope_t(z):
+        c = torch.complex(z[..., :half], z[..., half:]) * rot
+        return torch.cat([c.real, c.imag], -1)
+    q, k, v = rope_t(y[:, :, :H]), rope_t(y[:, :, H:H + G]), y[:, :, H + G:]
+    head = lambda z, hx: z.reshape(B, n, P, hx // P, d).permute(2, 0, 3, 1, 4)   # [P][B][hx/P][n][d]
+    return head(q, H), head(k, G), head(v, G)
+
+
+def test_rotation_inverse_is_negative_angle():
+    x = rng.standard_normal((6, 16))
+    pos = np.array([0, 3, 100, 65535, 262143, 7])
+    assert np.abs(oracle.rope(oracle.rope(x, pos), -pos) - x).max() < 1e-10
+
+
+@pytest.mark.parametrize("P,B,H,G,docs", [(4, 1, 8, 4, False), (2, 2, 4, 2, True)])
+def test_qkv_projection_backward_matches_torch_autograd(P, B, H, G, docs):
+    d, hidden, n = 8, 20, 24
+    x = rng.standard_normal((B, n, hidden))
+    w = rng.standard_normal(((H + 2 * G) * d, hidden)) / np.sqrt(hidden)
+    pos = np.tile(np.concatenate([np.arange(10), np.arange(n - 10)]) if docs else np.arange(n), (B, 1))
+    xt = torch.tensor(x, requires_grad=True)
+    wt = torch.tensor(w, requires_grad=True)
+    q, k, v = _torch_layer_proj(xt, wt, H, G, d, P, torch.tensor(pos, dtype=torch.float64))
+    gq, gk, gv = (rng.standard_normal(tuple(z.shape)) for z in (q, k, v))
+    ((q * torch.tensor(gq)).sum() + (k * torch.tensor(gk)).sum() + (v * torch.tensor(gv)).sum()).backward()
+    x_seq = x.reshape(B, P, n // P, hidden).transpose(1, 0, 2, 3)
+    # the oracle's own forward agrees with the torch one (same layout)
+    oq, ok_, ov = oracle.qkv_proj_rope(x_seq, w, P, H, G, d, positions=pos)
+    assert np.abs(oq - q.detach().numpy()).max() < 1e-12 and np.abs(ov - v.detach().numpy()).max() < 1e-12
+    dx, dw = oracle.qkv_proj_rope_bwd(x_seq, w, gq, gk, gv, P, H, G, d, positions=pos)
+    assert np.abs(dx.transpose(1, 0, 2, 3).reshape(B, n, hidden) - xt.grad.numpy()).max() < 1e-11
+    assert np.abs(dw - wt.grad.numpy()).max() < 1e-11
+
+
+def test_qkv_projection_backward_with_kv_copies_finite_differences():
+    """G < P: the copies' gradients are summed before the projection's
+    backward; central differences of sum(Q*gq + K*gk + V*gv) in x and w."""
+    P, B, H, G, d, hidden, n = 4, 1, 8, 2, 8, 12, 16
+    x = np.round(rng.standard_normal((P, B, n // P, hidden)) * 64) / 64
+    w = np.round(rng.standard_normal(((H + 2 * G) * d, hidden)) * 64) / 64
+    q, k, v = oracle.qkv_proj_rope(x, w, P, H, G, d)
+    gq, gk, gv = (rng.standard_normal(z.shape) for z in (q, k, v))
+    dx, dw = oracle.qkv_proj_rope_bwd(x, w, gq, gk, gv, P, H, G, d)
+
+    def f(xx, ww):
+        a, b, c = oracle.qkv_proj_rope(xx, ww, P, H, G, d)
+        return float((a * gq).sum() + (b * gk).sum() + (c * gv).sum())
+    h = 2.0 ** -10
+    for arr, grad, which in ((x, dx, 0), (w, dw, 1)):
+        for _ in range(6):
+            ix = tuple(rng.integers(0, m) for m in arr.shape)
+            ap, am = arr.copy(), arr.copy()
+            ap[ix] += h
+            am[ix] -= h
+            fp = f(ap, w) if which == 0 else f(x, ap)
+            fm = f(am, w) if which == 0 else f(x, am)
+            assert abs((fp - fm) / (2 * h) - grad[ix]) < 1e-8 * max(1.0, abs(grad[ix]))
+
+
+def test_output_projection_backward_matches_torch_autograd():
+    P, B, H, d, n, hidden = 4, 2, 8, 8, 16, 12
+    o_head = rng.standard_normal((P, B, H // P, n, d))
+    w = rng.standard_normal((hidden, H * d))
+    gy = rng.standard_normal((P, B, n // P, hidden))
+    ot = torch.tensor(o_head, requires_grad=True)
+    wt = torch.tensor(w, requires_grad=True)
+    o_nat = ot.permute(1, 3, 0, 2, 4).reshape(B, n, H * d)
+    y = F.linear(o_nat, wt)                                               # [B][n][hidden]
+    (y * torch.tensor(gy.transpose(1, 0, 2, 3).reshape(B, n, hidden))).sum().backward()
+    do_head, dw = oracle.o_proj_bwd(o_head, w, gy, P)
+    assert np.abs(do_head - ot.grad.numpy()).max() < 1e-12
+    assert np.abs(dw - wt.grad.numpy()).max() < 1e-11
