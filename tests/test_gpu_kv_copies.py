@@ -197,3 +197,23 @@ def test_qwen8k_on_16_ranks_sampled():
                                         f32_inputs(kn[:, kvh]), f32_inputs(vn[:, kvh]), cols)
         _assert_summed_close(dkn[cols, kvh].double().numpy(), dk_ref, ek[cols, kvh], f"dK kv head {kvh}")
         _assert_summed_close(dvn[cols, kvh].double().numpy(), dv_ref, ev[cols, kvh], f"dV kv head {kvh}")
+
+
+def test_copies_at_the_benchmarked_size():
+    """The configuration the bench times: the 64K workload's K (G = 8) over
+    P = 16 ranks (two copies per KV head), iota payload (int16 pairs viewed as
+    bf16, every element distinct): copies bit-exact against the oracle, and
+    the summing reverse of the copies gives exactly 2 x (bf16: exact doubling)."""
+    P, G, n, d = 16, 8, 65536, 128
+    s = n // P
+    x = (torch.arange(P * s * G * d, dtype=torch.int64) % 16381 + 1).to(torch.int16).reshape(P, 1, s, G, d)
+    rep = U.ulysses_kv_seq_to_head_replicated(x.cuda().view(torch.bfloat16), P)
+    torch.cuda.synchronize()
+    assert np.array_equal(rep.view(torch.int16).cpu().numpy(), oracle.kv_replicate_to_head(x.numpy(), 1, n, P, G))
+    del rep
+    # doubling is exact in bf16 for finite values: sum of the two copies == 2 x
+    xb = torch.randn(P, 1, s, G, d, generator=torch.Generator().manual_seed(16)).to(torch.bfloat16)
+    back = U.ulysses_kv_head_to_seq_reduce(U.ulysses_kv_seq_to_head_replicated(xb.cuda(), P), P, G)
+    torch.cuda.synchronize()
+    assert torch.equal(back.cpu(), (xb.float() * 2).to(torch.bfloat16))
+    assert U.ulysses_read_error() == 0
