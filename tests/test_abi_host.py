@@ -169,3 +169,16 @@ def test_smoke_shape_passes_host_validation(L):
     desc = U.make_desc(1, n, P, H, G, d, U.ULY_BF16, U.MASK_CAUSAL)
     assert L.ulysses_attn_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(n_ws)) == 0
     assert L.ulysses_loss_bwd_workspace_size(P, 256, 8192, ctypes.byref(n_ws)) == 0
+
+
+def test_every_profiled_kernel_has_a_distinct_name(L):
+    """The per-kernel timing table names every kernel id (an id without a
+    name would make the profile unreadable)."""
+    names = [L.ulysses_kernel_name(k) for k in range(L.ulysses_kernel_count())]
+    assert all(n for n in names), names
+    names = [n.decode() for n in names]
+    assert len(set(names)) == len(names) and "unknown" not in names
+    for k in ("attn_fwd_sm100", "attn_dkdv_sm100", "attn_dq_sm100", "seq_to_head", "head_to_seq",
+              "loss_partial", "qkv_proj_sm100", "o_proj_sm100", "kv_seq_to_head_rep", "shift_labels"):
+        assert k in names
+    assert L.ulysses_kernel_name(L.ulysses_kernel_count()) == b"unknown"
