@@ -182,3 +182,27 @@ def test_every_profiled_kernel_has_a_distinct_name(L):
               "loss_partial", "qkv_proj_sm100", "o_proj_sm100", "kv_seq_to_head_rep", "shift_labels"):
         assert k in names
     assert L.ulysses_kernel_name(L.ulysses_kernel_count()) == b"unknown"
+
+
+def test_loss_gradient_validation(L):
+    vp = ctypes.c_void_p
+    T, V, P = 1024, 8192, 4
+    n = ctypes.c_size_t(0)
+    assert L.ulysses_loss_bwd_workspace_size(P, T, V, ctypes.byref(n)) == 0 and n.value > 0
+    need = n.value
+    z, y, dz = vp(1 << 32), vp(1 << 30), vp(1 << 34)           # logits 16 MiB, labels, dlogits
+    S, C, Lo, ws = vp(1 << 24), vp((1 << 24) + 4096), vp((1 << 24) + 8192), vp(1 << 26)
+    f = L.ulysses_loss_aggregate_bwd
+    ok = [P, T, V, 1, z, y, -100, dz, S, C, Lo, ws, need, None]
+    bad = list(ok); bad[7] = None
+    assert f(*bad) == 1                                          # no dlogits
+    bad = list(ok); bad[12] = need - 16
+    assert f(*bad) == 10                                         # workspace too small
+    bad = list(ok); bad[7] = vp((1 << 32) + 1024)
+    assert f(*bad) == 5                                          # dlogits inside the logits
+    bad = list(ok); bad[11] = vp((1 << 34) + 4096)
+    assert f(*bad) == 5                                          # workspace inside dlogits
+    bad = list(ok); bad[7] = vp((1 << 34) + 8)
+    assert f(*bad) == 4                                          # misaligned dlogits
+    bad = list(ok); bad[1] = T - 1
+    assert f(*bad) == 2                                          # tokens % P
