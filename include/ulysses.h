@@ -311,6 +311,13 @@ uly_status ulysses_loss_aggregate_noalloc(int32_t world, int64_t tokens, int32_t
                                           float *shard_sum, int64_t *shard_count, float *loss,
                                           void *stream);
 
+/* Device address of the current device's asynchronous error word (int32;
+ * bit s set <=> status s was raised by a kernel since it was last cleared),
+ * for callers that poll it themselves (e.g. with their own stream-ordered
+ * copy) instead of ulysses_read_error.  The word is owned by the library and
+ * lives as long as the process's context on that device. */
+uly_status ulysses_error_word(int32_t **dev_word);
+
 /* Asynchronous error word of the current device: reads it (synchronising the
  * device) into *word (bit s set <=> status s was raised) and clears it. */
 uly_status ulysses_read_error(int32_t *word);

@@ -390,6 +390,14 @@ uly_status ulysses_read_error_info(int32_t *info, int32_t n) {
   return ULY_OK;
 }
 
+uly_status ulysses_error_word(int32_t **dev_word) {
+  if (!dev_word) return ULY_ERR_NULL;
+  int *p = error_word();
+  if (!p) return ULY_ERR_CUDA;
+  *dev_word = p;
+  return ULY_OK;
+}
+
 uly_status ulysses_read_error(int32_t *word) {
   if (!word) return ULY_ERR_NULL;
   return ulysses_read_error_info(word, 1);

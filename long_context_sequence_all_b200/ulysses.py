@@ -28,7 +28,7 @@ EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head
            "ulysses_qkv_proj_rope", "ulysses_o_proj", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
            "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
-           "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info",
+           "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info", "ulysses_error_word",
            "ulysses_status_string", "ulysses_profile_enable", "ulysses_profile_read",
            "ulysses_kernel_count", "ulysses_kernel_name",
            "ulysses_launch_count"]
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.ulysses_loss_bwd_workspace_size.argtypes = [i32, i64, i32, ctypes.POINTER(sz)]
             L.ulysses_loss_aggregate_bwd.argtypes = [i32, i64, i32, i32, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
             L.ulysses_read_error.argtypes = [ctypes.POINTER(i32)]
+            L.ulysses_error_word.argtypes = [ctypes.POINTER(vp)]
+            L.ulysses_error_word.restype = ctypes.c_int
             L.ulysses_read_error_info.argtypes = [ctypes.POINTER(i32), i32]
             L.ulysses_status_string.argtypes = [ctypes.c_int]
             L.ulysses_status_string.restype = ctypes.c_char_p
@@ -385,6 +387,13 @@ def ulysses_read_error() -> int:
     w = ctypes.c_int32(0)
     _check(lib().ulysses_read_error(ctypes.byref(w)), "ulysses_read_error")
     return w.value
+
+
+def ulysses_error_word() -> int:
+    """Device address of the current device's asynchronous error word (int32)."""
+    p = ctypes.c_void_p(0)
+    _check(lib().ulysses_error_word(ctypes.byref(p)), "ulysses_error_word")
+    return int(p.value or 0)
 
 
 def ulysses_read_error_info() -> list:

@@ -206,3 +206,7 @@ def test_loss_gradient_validation(L):
     assert f(*bad) == 4                                          # misaligned dlogits
     bad = list(ok); bad[1] = T - 1
     assert f(*bad) == 2                                          # tokens % P
+
+
+def test_error_word_null_argument(L):
+    assert L.ulysses_error_word(None) == 1

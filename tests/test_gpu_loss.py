@@ -96,3 +96,28 @@ def test_loss_workload(name):
     documents with 20% ignored labels and an ignored pad tail)."""
     inp = make_inputs(name, with_grad_inputs=False)
     _check(inp["logits"], inp["labels"], inp["P"])
+
+
+def test_error_word_address_holds_the_async_errors():
+    """ulysses_error_word gives the device word that kernels OR their
+    data-dependent errors into: a bad label shows up there, and
+    ulysses_read_error reads and clears the same word."""
+    addr = U.ulysses_error_word()
+    assert addr and addr == U.ulysses_error_word()
+
+    class _Word:
+        __cuda_array_interface__ = {"shape": (1,), "typestr": "<i4", "data": (addr, False), "version": 3}
+    try:   # read the word at that address through torch's CUDA-array-interface import
+        word = torch.as_tensor(_Word(), device="cuda")
+    except (TypeError, RuntimeError, ValueError):
+        word = None
+    U.ulysses_read_error()
+    logits = torch.randn(8, 256, device="cuda").to(torch.bfloat16)
+    labels = torch.tensor([0, 1, 999, 3, 4, 5, 6, 7], dtype=torch.int32, device="cuda")
+    U.ulysses_loss_aggregate(logits, labels, 2)
+    torch.cuda.synchronize()
+    if word is not None:
+        assert int(word.item()) & (1 << 8)
+    assert U.ulysses_read_error() & (1 << 8)
+    if word is not None:
+        assert int(word.item()) == 0
