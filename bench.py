@@ -66,6 +66,16 @@ def causal_pairs(inp) -> float:
     return float(sum((b - a) * (b - a + 1) / 2.0 for a, b in zip(cu[:-1], cu[1:])))
 
 
+MASK_NAMES = {0: "full (no mask)", 1: "causal", 2: "doc-causal (packed documents)"}
+
+
+def workload_label(w, inp) -> str:
+    """The workload in words: shapes, input dtype, mask and the passes of one step."""
+    loss = f" + CE loss V={w.vocab}" if "logits" in inp else ""
+    return (f"{w.name}: Qwen3-4B-shaped Ulysses attention layer, B={w.B} n={inp['n']} P={w.P} H={w.H} "
+            f"G={w.G} d={w.d} bf16 {MASK_NAMES[inp['mask']]} fwd+bwd{loss}")
+
+
 def algorithmic_work(inp):
     """Algorithmic flops / bytes of each kernel per launch (see the design notes)."""
     B, H, G, d, n = inp["B"], inp["H"], inp["G"], inp["d"], inp["n"]
@@ -451,8 +461,7 @@ def run_ours(args, rank, world, dev):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(128) Q/K/V, N(0,1) dO and logits, uniform labels)",
-        "config": {"workload": f"{w.name}: Qwen3-4B-shaped Ulysses attention layer, B={w.B} n={inp['n']} "
-                               f"P={w.P} H={w.H} G={w.G} d={w.d} bf16 causal fwd+bwd + CE loss V={w.vocab}",
+        "config": {"workload": workload_label(w, inp),
                    "global_batch": inp["B"] * world, "seq_len": inp["n"],
                    "parallelism": f"P={w.P} logical Ulysses ranks per GPU; {world} independent replica(s)",
                    "l2": _l2_note(inp)},
@@ -701,8 +710,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded inputs as the GPU arm)",
-        "config": {"workload": f"{w.name}: Qwen3-4B-shaped Ulysses attention layer, B={w.B} n={inp['n']} "
-                               f"P={w.P} H={w.H} G={w.G} d={w.d} causal fwd+bwd + CE loss V={w.vocab}",
+        "config": {"workload": workload_label(w, inp),
                    "global_batch": inp["B"], "seq_len": inp["n"], "parallelism": "CPU oracle (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
                          "sample": desc},

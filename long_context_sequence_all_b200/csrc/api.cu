@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace uly {
 
@@ -104,6 +105,25 @@ uly_status check_desc(const uly_attn_desc *d, HeadGeom &g, MaskInfo &mk) {
   mk.cu = d->cu_seqlens;
   mk.num_docs = d->num_docs;
   return ULY_OK;
+}
+
+// One thread: cu_seqlens must start at 0, never decrease and end at n (the
+// pad tail is the last document).  Anything else is reported as
+// ULY_ERR_SHAPE in the error word; the attention kernels clamp document
+// bounds to the sequence, so a malformed table never sends them outside
+// their operands.
+__global__ void check_cu_seqlens_kernel(const int32_t *__restrict__ cu, int num_docs, int n, int *err) {
+  bool ok = __ldg(cu) == 0 && __ldg(cu + num_docs) == n;
+  for (int e = 0; ok && e < num_docs; ++e) ok = __ldg(cu + e) <= __ldg(cu + e + 1);
+  if (!ok) raise_error(err, ULY_ERR_SHAPE);
+}
+
+uly_status check_cu_seqlens(const uly_attn_desc *d, cudaStream_t s) {
+  if (d->mask != ULY_MASK_DOC_CAUSAL) return ULY_OK;
+  prof::Scope scope(prof::K_CHECK_CU, s);
+  check_cu_seqlens_kernel<<<1, 1, 0, s>>>(d->cu_seqlens, d->num_docs, d->seq_len, error_word());
+  note_launches(1);
+  return last_launch_status();
 }
 
 size_t elem_bytes(int dtype) { return dtype == ULY_BF16 ? 2 : 4; }
@@ -264,6 +284,7 @@ uly_status ulysses_attn_fwd(const uly_attn_desc *d, const void *q, const void *k
   }
   if (overlap(o, qb, lse, lb)) return ULY_ERR_ALIAS;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = check_cu_seqlens(d, s)) != ULY_OK) return st;
   if (d->dtype == ULY_F32) return attn_f32_fwd_launch(d, g, mk, q, k, v, o, lse, s);
   return attn_bf16_fwd_launch(d, g, mk, q, k, v, o, lse, s);
 }
@@ -308,6 +329,7 @@ uly_status ulysses_attn_bwd(const uly_attn_desc *d, const void *q, const void *k
       if (overlap(outs[a], outb[a], outs[b], outb[b])) return ULY_ERR_ALIAS;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = check_cu_seqlens(d, s)) != ULY_OK) return st;
   float *Dv = static_cast<float *>(workspace);
   if (d->dtype == ULY_F32)
     return attn_f32_bwd_launch(d, g, mk, q, k, v, o, lse, dout, dq, dk, dv, Dv, s);

@@ -705,15 +705,10 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
       !make_tmap_heads_bf16(&mK64, k, kHD, g.n, kvheads, 64) ||
       !make_tmap_heads_bf16(&mV64, v, kHD, g.n, kvheads, 64))
     return ULY_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_dkdv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kv::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             qk::kSmemBytes) != cudaSuccess)
-      return ULY_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> optin_kv{0}, optin_q{0};
+  if (!smem_optin(attn_dkdv_sm100_kernel, kv::kSmemBytes, optin_kv) ||
+      !smem_optin(attn_dq_sm100_kernel, qk::kSmemBytes, optin_q))
+    return ULY_ERR_CUDA;
   BwdParams prm;
   prm.q = static_cast<const __nv_bfloat16 *>(q);
   prm.dout = static_cast<const __nv_bfloat16 *>(dout);

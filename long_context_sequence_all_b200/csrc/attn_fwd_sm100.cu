@@ -384,13 +384,8 @@ uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
       !make_tmap_heads_bf16(&tk, k, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&tv, v, kHD, g.n, kvheads, 128))
     return ULY_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return ULY_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> optin_devices{0};
+  if (!smem_optin(attn_fwd_sm100_kernel, kSmemBytes, optin_devices)) return ULY_ERR_CUDA;
   FwdParams prm;
   prm.o = static_cast<__nv_bfloat16 *>(o);
   prm.lse = lse;

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "ulysses.h"
 
 namespace uly {
@@ -29,6 +31,21 @@ inline uly_status last_launch_status() {
   return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA;
 }
 
+// Opt `kernel` into `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to a device, so it is set once per device; `done`
+// holds one bit per device already set (atomic: host threads may race here).
+template <typename Kernel>
+inline bool smem_optin(Kernel kernel, int bytes, std::atomic<uint64_t> &done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool overlap(const void *a, size_t na, const void *b, size_t nb) {
@@ -38,21 +55,23 @@ inline bool overlap(const void *a, size_t na, const void *b, size_t nb) {
 
 // Position ranges of the three masks.  Row i may see keys [lo, hi].
 // doc-causal: the document containing i, found by binary search in cu_seqlens.
-__device__ __forceinline__ int doc_start_of(const int32_t *__restrict__ cu, int num_docs, int i) {
+// A well-formed cu_seqlens (cu[0] = 0, non-decreasing, cu[num_docs] = n) is
+// checked on the device by check_cu_seqlens_kernel; the bounds returned here
+// are clamped to [0, i] and [i + 1, n] so that a malformed one can only give a
+// wrong mask, never a tile outside the operands.
+__device__ __forceinline__ int doc_index_of(const int32_t *__restrict__ cu, int num_docs, int i) {
   int lo = 0, hi = num_docs - 1;  // find the largest e with cu[e] <= i
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
     if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
   }
-  return __ldg(cu + lo);
+  return lo;
 }
-__device__ __forceinline__ int doc_end_of(const int32_t *__restrict__ cu, int num_docs, int i) {
-  int lo = 0, hi = num_docs - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
-  }
-  return __ldg(cu + lo + 1);
+__device__ __forceinline__ int doc_start_of(const int32_t *__restrict__ cu, int num_docs, int i) {
+  return min(max(__ldg(cu + doc_index_of(cu, num_docs, i)), 0), i);
+}
+__device__ __forceinline__ int doc_end_of(const int32_t *__restrict__ cu, int num_docs, int i, int n) {
+  return min(max(__ldg(cu + doc_index_of(cu, num_docs, i) + 1), i + 1), n);
 }
 
 struct MaskInfo {
@@ -70,7 +89,7 @@ struct MaskInfo {
   __device__ __forceinline__ void col_range(int j, int &lo, int &hi) const {
     if (mask == ULY_MASK_NONE) { lo = 0; hi = n - 1; return; }
     lo = j;
-    hi = (mask == ULY_MASK_DOC_CAUSAL) ? doc_end_of(cu, num_docs, j) - 1 : n - 1;
+    hi = (mask == ULY_MASK_DOC_CAUSAL) ? doc_end_of(cu, num_docs, j, n) - 1 : n - 1;
   }
 };
 

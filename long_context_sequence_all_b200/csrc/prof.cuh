@@ -30,6 +30,7 @@ enum Kernel {
   K_ROPE_TABLE,
   K_QKV_PROJ,
   K_O_PROJ,
+  K_CHECK_CU,
   K_COUNT
 };
 

@@ -61,6 +61,7 @@ def _load():
             lib.oracle_ulysses_bwd.argtypes = uly + [P, P, P, P, P, P, P]
             lib.oracle_head_rows.argtypes = [i, i, i, P, i, dbl, P, P, P, P, P, i, P, P, P]
             lib.oracle_kv_cols.argtypes = [i, i, i, P, i, dbl, i, P, P, P, P, P, i, P, P]
+            lib.oracle_kv_cols_stats.argtypes = [i, i, i, P, i, dbl, i, P, P, P, P, P, P, P, i, P, P]
             lib.oracle_head_rows_step.argtypes = [i, i, i, P, i, dbl, P, P, P, P, P, i, P, P, P, P, P]
             lib.oracle_loss.argtypes = [i, l, i, P, P, i, P, P, P]
             lib.oracle_loss.restype = l
@@ -239,9 +240,13 @@ def head_rows(q, k, v, rows, dout=None, mask=MASK_CAUSAL, cu_seqlens=None, scale
     return (o, lse, dq) if dout is not None else (o, lse)
 
 
-def kv_cols(qs, douts, k, v, cols, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0):
+def kv_cols(qs, douts, k, v, cols, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0, stats=None):
     """One KV head k, v [n][d] and its query heads qs[e], douts[e] [n][d]:
-    exact dK, dV at the listed key columns, summed over the query heads."""
+    exact dK, dV at the listed key columns, summed over the query heads.
+
+    stats: None (the C routine computes LSE_i and D_i of every row that sees a
+    listed key, one row at a time), or a list of (lse [n], D [n]) per query
+    head covering at least those rows (e.g. from row_stats)."""
     qs = [_f32(x) for x in qs]
     douts = [_f32(x) for x in douts]
     k, v = _f32(k), _f32(v)
@@ -252,10 +257,91 @@ def kv_cols(qs, douts, k, v, cols, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0)
     dp = (ctypes.c_void_p * len(douts))(*[x.ctypes.data for x in douts])
     dk = np.empty((cols.size, d), np.float64)
     dv = np.empty((cols.size, d), np.float64)
-    _load().oracle_kv_cols(n, d, mask, _ptr(cu), nd, scale, len(qs),
-                           ctypes.cast(qp, ctypes.c_void_p), ctypes.cast(dp, ctypes.c_void_p),
-                           _ptr(k), _ptr(v), _ptr(cols), cols.size, _ptr(dk), _ptr(dv))
+    if stats is None:
+        _load().oracle_kv_cols(n, d, mask, _ptr(cu), nd, scale, len(qs),
+                               ctypes.cast(qp, ctypes.c_void_p), ctypes.cast(dp, ctypes.c_void_p),
+                               _ptr(k), _ptr(v), _ptr(cols), cols.size, _ptr(dk), _ptr(dv))
+        return dk, dv
+    if len(stats) != len(qs):
+        raise ValueError("one (lse, D) pair per query head")
+    ls = [np.ascontiguousarray(a, dtype=np.float64) for a, _ in stats]
+    Ds = [np.ascontiguousarray(b, dtype=np.float64) for _, b in stats]
+    if any(a.shape != (n,) for a in ls + Ds):
+        raise ValueError("lse and D must have n entries")
+    lp = (ctypes.c_void_p * len(ls))(*[x.ctypes.data for x in ls])
+    Dp = (ctypes.c_void_p * len(Ds))(*[x.ctypes.data for x in Ds])
+    _load().oracle_kv_cols_stats(n, d, mask, _ptr(cu), nd, scale, len(qs),
+                                 ctypes.cast(qp, ctypes.c_void_p), ctypes.cast(dp, ctypes.c_void_p),
+                                 _ptr(k), _ptr(v), ctypes.cast(lp, ctypes.c_void_p),
+                                 ctypes.cast(Dp, ctypes.c_void_p), _ptr(cols), cols.size, _ptr(dk), _ptr(dv))
     return dk, dv
+
+
+def rows_seeing(cols, n, mask=MASK_CAUSAL, cu_seqlens=None):
+    """[lo, hi): the smallest row range holding every query row that sees one
+    of the listed key columns (causal: j <= i; doc-causal: also the same
+    document; no mask: every row)."""
+    cols = np.asarray(cols)
+    if mask == MASK_NONE:
+        return 0, n
+    lo = int(cols.min())
+    if mask == MASK_CAUSAL:
+        return lo, n
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    last = int(cols.max())
+    e = int(np.searchsorted(cu, last, side="right")) - 1
+    return lo, int(min(n, cu[e + 1]))
+
+
+def row_stats(q, k, v, dout, lo, hi, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0, chunk=512):
+    """LSE_i and D_i = <dO_i, O_i> of the query rows [lo, hi) of one head
+    (q, dout [n][d]) with its KV head (k, v [n][d]), straight from the
+    definition in float64 with library matrix products (torch CPU), a chunk
+    of rows at a time (rows are independent):
+        s_ij = scale q_i.k_j over the visible keys j, m_i = max_j s_ij,
+        LSE_i = m_i + log sum_j exp(s_ij - m_i),
+        O_i = sum_j exp(s_ij - LSE_i) v_j,  D_i = <dO_i, O_i>.
+    Rows outside [lo, hi) get LSE = -inf, D = 0; a row that sees no key too."""
+    import torch
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    n, d = q.shape
+    sc = scale if scale > 0 else 1.0 / np.sqrt(d)
+    Q, K, V, dO = (torch.from_numpy(x).double() for x in (q, k, v, dout))
+    doc = None
+    if mask == MASK_DOC_CAUSAL:
+        cu = torch.from_numpy(np.asarray(cu_seqlens, dtype=np.int64))
+        doc = torch.searchsorted(cu, torch.arange(n, dtype=torch.int64), right=True) - 1
+    lse = np.full(n, -np.inf)
+    D = np.zeros(n)
+    for r0 in range(lo, hi, chunk):
+        r1 = min(hi, r0 + chunk)
+        k0, k1 = 0, n
+        if mask != MASK_NONE:
+            k1 = r1
+            if mask == MASK_DOC_CAUSAL:
+                k0 = int(cu[doc[r0]])
+        S = Q[r0:r1] @ K[k0:k1].T
+        S.mul_(sc)
+        if mask != MASK_NONE:
+            # keys before the chunk's first row are visible to all its rows
+            # (causal); the mask is needed from there on, and for documents
+            # from the chunk's first document start
+            c0 = r0 if mask == MASK_CAUSAL else k0
+            i = torch.arange(r0, r1).unsqueeze(1)
+            j = torch.arange(c0, k1).unsqueeze(0)
+            allowed = j <= i
+            if mask == MASK_DOC_CAUSAL:
+                allowed &= doc[c0:k1].unsqueeze(0) == doc[r0:r1].unsqueeze(1)
+            S[:, c0 - k0:].masked_fill_(~allowed, float("-inf"))
+        m = S.max(dim=1).values
+        seen = torch.isfinite(m)
+        ms = torch.where(seen, m, torch.zeros_like(m))
+        S.sub_(ms.unsqueeze(1)).exp_()          # S now holds exp(s_ij - m_i)
+        ls = S.sum(dim=1)
+        O = (S @ V[k0:k1]) / torch.where(seen, ls, torch.ones_like(ls)).unsqueeze(1)
+        lse[r0:r1] = torch.where(seen, ms + torch.log(ls), torch.full_like(m, float("-inf"))).numpy()
+        D[r0:r1] = torch.where(seen, (dO[r0:r1] * O).sum(dim=1), torch.zeros_like(m)).numpy()
+    return lse, D
 
 
 def head_rows_step(q, k, v, dout, rows, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0, dk=None, dv=None):

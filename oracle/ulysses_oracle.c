@@ -619,6 +619,23 @@ void oracle_kv_cols(int n, int d, int mask, const int *cu_seqlens, int num_docs,
   free(lse); free(Dv); free(need); free(doc);
 }
 
+/* The same key columns as oracle_kv_cols, with the per-row statistics
+ * lse[h][i] and D[h][i] of every row that sees a listed key supplied by the
+ * caller (computed from the definition elsewhere, e.g. with fp64 matrix
+ * products for a whole row range); only the column sums are formed here. */
+void oracle_kv_cols_stats(int n, int d, int mask, const int *cu_seqlens, int num_docs, double scale,
+                          int nq, const float *const *qs, const float *const *douts,
+                          const float *k, const float *v, const double *const *lse,
+                          const double *const *Dv, const int *cols, int ncols, double *dk, double *dv) {
+  attn_cfg c = make_cfg(n, d, mask, cu_seqlens, num_docs, scale);
+  int *doc = doc_index(&c);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int e = 0; e < ncols; ++e)
+    attn_col_bwd(&c, doc, cols[e], nq, qs, d, douts, d, k, d, v, d, lse, Dv,
+                 dk + (size_t)e * d, dv + (size_t)e * d);
+  free(doc);
+}
+
 /*
  * Everything one query row i of one head contributes to the layer: O_i,
  * lse_i, dQ_i, and its terms of dK_j = scale * sum_i dS_ij q_i and

@@ -18,3 +18,20 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """How many bf16 elements needed the rounding term of the bound (more than
+    the flat max-abs tolerance) over all element-wise checks of the run."""
+    try:
+        from helpers import ULP_ADMITTED
+    except ImportError:
+        return
+    if not ULP_ADMITTED:
+        return
+    total = sum(n for _, _, n in ULP_ADMITTED)
+    adm = [(w, a, n) for w, a, n in ULP_ADMITTED if a]
+    terminalreporter.write_line(
+        f"bf16 parity: {len(ULP_ADMITTED)} element-wise checks, {total} elements; "
+        f"{sum(a for _, a, _ in adm)} above the flat 2e-2 (admitted by the half-ulp term) in {len(adm)} checks"
+        + ("".join(f"; {w}: {a}/{n}" for w, a, n in adm[:8])))

@@ -35,22 +35,40 @@ def max_abs(a, b):
     return float(np.abs(a - b).max()) if a.size else 0.0
 
 
-BF16_ULP_REL = 2.0 ** -7   # one bf16 ulp is at most 2^-7 |x| (8 significant bits)
+# bf16 keeps 8 significant bits: rounding a value x to the nearest bf16 moves
+# it by at most 2^-8 |x| (half an ulp).
+BF16_HALF_ULP_REL = 2.0 ** -8
+# Accumulation allowance beside that rounding: the part of the stated 2e-2
+# that the half-ulp rounding leaves at |x| = 2.56, where the two terms meet
+# (2^-8 * 2.56 = 1e-2), so the bound below is continuous there.
+BF16_ACC_ABS = 1e-2
+
+# Every bf16 check records how many elements needed more than the flat
+# max-abs bound (admitted only by the rounding term); conftest prints them.
+ULP_ADMITTED = []
+
+
+def bf16_bound(ref, max_abs_tol=BF16_MAX_ABS):
+    """Element-wise bound max(2e-2, 2^-8 |ref| + 1e-2): the stated 2e-2, and
+    above |ref| = 2.56 (where a bf16 output cannot resolve 2e-2: rounding the
+    exact value alone may move it by 2^-8 |ref| > 1e-2) half an ulp of the
+    exact value plus the accumulation allowance."""
+    return np.maximum(max_abs_tol, BF16_HALF_ULP_REL * np.abs(ref) + BF16_ACC_ABS)
 
 
 def assert_bf16_close(got, ref, what="", max_abs_tol=BF16_MAX_ABS, rel_tol=BF16_REL_L2):
-    """Element-wise |got - ref| <= max(2e-2, one bf16 ulp of |ref|) and
-    relative L2 <= 1e-2.  The ulp term only matters for |ref| > 2.56, where a
-    bf16 output cannot resolve 2e-2 (the exact value rounded to bf16 may
-    already be 2^-8 |ref| away); below that the bound is the plain 2e-2."""
+    """Element-wise |got - ref| <= bf16_bound(ref) and relative L2 <= 1e-2."""
     g, r = to64(got), to64(ref)
     assert np.isfinite(g).all(), f"{what}: non-finite values"
     err = np.abs(g - r)
-    bound = np.maximum(max_abs_tol, BF16_ULP_REL * np.abs(r))
+    bound = bf16_bound(r, max_abs_tol)
     worst = float((err / bound).max()) if err.size else 0.0
     ma, rl = (float(err.max()) if err.size else 0.0), rel_l2(g, r)
+    admitted = int((err > max_abs_tol).sum())
+    ULP_ADMITTED.append((what, admitted, int(err.size)))
     assert worst <= 1.0 and rl <= rel_tol, \
-        f"{what}: max_abs={ma:.3e} (worst err/bound {worst:.2f}) rel_l2={rl:.3e}"
+        f"{what}: max_abs={ma:.3e} (worst err/bound {worst:.2f}, {admitted} of {err.size} above " \
+        f"{max_abs_tol:g}) rel_l2={rl:.3e}"
     return ma, rl
 
 

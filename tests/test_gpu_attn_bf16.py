@@ -202,6 +202,27 @@ def test_bwd_workload_sampled(name):
                                         mask=inp["mask"], cu_seqlens=cun)
         assert_bf16_close(dkn[cols, kvh], dk_ref, f"dK kv head {kvh}")
         assert_bf16_close(dvn[cols, kvh], dv_ref, f"dV kv head {kvh}")
+    # Key columns with the longest accumulations (the causal rows from the
+    # column on all see it): the first keys and shard starts at 64K (65,536
+    # rows x 4 query heads = 2,048 query tiles into one dK/dV tile), the last
+    # shard's start at 256K (32,768 rows x 4 heads).  The statistics of all
+    # those rows come from the oracle's fp64 matrix-product routine.
+    s = n // P
+    early = {"qwen64k": [0, 1, 127, 128, s - 1, s, 2 * s, 3 * s, n // 2],
+             "long256k": [n - s, n - s + 1, n - s + 127, n - s + 128]}.get(name)
+    if early:
+        kvh = G - 1
+        heads = range(kvh * group, (kvh + 1) * group)
+        cols = np.array(early, dtype=np.int32)
+        lo, hi = oracle.rows_seeing(cols, n, mask=inp["mask"], cu_seqlens=cun)
+        qs = [f32_inputs(qn[:, h]) for h in heads]
+        dos = [f32_inputs(don[:, h]) for h in heads]
+        kk, vv = f32_inputs(kn[:, kvh]), f32_inputs(vn[:, kvh])
+        stats = [oracle.row_stats(qh_, kk, vv, do_, lo, hi, mask=inp["mask"], cu_seqlens=cun)
+                 for qh_, do_ in zip(qs, dos)]
+        dk_ref, dv_ref = oracle.kv_cols(qs, dos, kk, vv, cols, mask=inp["mask"], cu_seqlens=cun, stats=stats)
+        assert_bf16_close(dkn[cols, kvh], dk_ref, f"dK kv head {kvh}, long accumulations")
+        assert_bf16_close(dvn[cols, kvh], dv_ref, f"dV kv head {kvh}, long accumulations")
     _gradient_invariants(inp, dk, dv)
 
 

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import (BF16_MAX_ABS, BF16_REL_L2, F32_MAX_ABS, assert_bf16_close, f32_inputs,
+from helpers import (BF16_MAX_ABS, BF16_REL_L2, F32_MAX_ABS, assert_bf16_close, bf16_bound, f32_inputs,
                      max_abs, rel_l2, sample_rows)
 from long_context_sequence_all_b200 import ulysses as U
 from long_context_sequence_all_b200.workloads import make_inputs, to_natural
@@ -71,16 +71,18 @@ def test_reduce_single_rounding_exact(P, B, n, G, dtype):
 
 @pytest.mark.parametrize("P,G,dtype", [(8, 2, torch.bfloat16), (16, 1, torch.bfloat16), (8, 1, torch.float32)])
 def test_reduce_random_within_fp32_sum_bound(P, G, dtype):
-    """N(0,1) data: |got - exact| <= one ulp of the element type at |exact| plus
-    the fp32 summation bound (P/G - 1) * 2^-24 * sum |x_j|."""
+    """N(0,1) data: |got - exact| <= the fp32 summation bound
+    e = (P/G - 1) * 2^-24 * sum |x_j| plus half an ulp of the element type at
+    |exact| + e (the one rounding of the fp32 sum)."""
     B, n, d = 1, 2048 + 8 * P, 128
     x = torch.randn(P, B, 1, n, d, generator=torch.Generator().manual_seed(5)).to(dtype)
     y = U.ulysses_kv_head_to_seq_reduce(x.cuda(), P, G)
     torch.cuda.synchronize()
     ref = oracle.kv_reduce_to_seq(x.double().numpy(), B, n, P, G)
     abs_sum = oracle.kv_reduce_to_seq(x.double().abs().numpy(), B, n, P, G)
-    ulp = (2.0 ** -7 if dtype == torch.bfloat16 else 2.0 ** -23) * np.abs(ref)
-    bound = ulp + (P // G - 1) * 2.0 ** -24 * abs_sum + 1e-30
+    acc = (P // G - 1) * 2.0 ** -24 * abs_sum
+    half_ulp = (2.0 ** -8 if dtype == torch.bfloat16 else 2.0 ** -24) * (np.abs(ref) + acc)
+    bound = half_ulp + acc + 1e-30
     err = np.abs(y.cpu().double().numpy() - ref)
     assert (err <= bound).all(), float((err / bound).max())
 
@@ -113,11 +115,11 @@ def _copy_rounding(parts, B, n, P, G):
 
 
 def _assert_summed_close(got, ref, extra, what):
-    """|got - ref| <= max(2e-2, one bf16 ulp of |ref|) + the partials' rounding,
-    element-wise; relative L2 <= 1e-2 unchanged."""
+    """|got - ref| <= bf16_bound(ref) + the partials' rounding, element-wise;
+    relative L2 <= 1e-2 unchanged."""
     g, r = np.asarray(got, np.float64), np.asarray(ref, np.float64)
     err = np.abs(g - r)
-    bound = np.maximum(BF16_MAX_ABS, 2.0 ** -7 * np.abs(r)) + extra
+    bound = bf16_bound(r) + extra
     worst = float((err / bound).max())
     assert worst <= 1.0 and rel_l2(g, r) <= BF16_REL_L2, f"{what}: worst err/bound {worst:.2f}"
 

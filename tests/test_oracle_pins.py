@@ -453,6 +453,52 @@ def test_sampled_rows_and_columns_match_full(mask):
 
 
 @pytest.mark.parametrize("mask", [MASK_CAUSAL, MASK_DOC_CAUSAL, MASK_NONE])
+def test_row_stats_match_full_forward(mask):
+    """The per-row statistics from fp64 matrix products (used for key columns
+    that every row sees at full size) equal the row-by-row oracle: LSE_i, and
+    D_i = <dO_i, O_i> with O from the oracle's forward; rows outside the range
+    get (-inf, 0).  Chunks of 7 rows make the row range cross chunk and
+    document boundaries."""
+    n, H, G, d = 70, 4, 2, 8
+    q, k, v, do = _randn(1, n, H, d), _randn(1, n, G, d), _randn(1, n, G, d), _randn(1, n, H, d)
+    cu = np.array([0, 9, 10, 41, n], np.int32) if mask == MASK_DOC_CAUSAL else None
+    o, lse = oracle.attention_fwd(q, k, v, mask=mask, cu_seqlens=cu)
+    for h in range(H):
+        g = h // (H // G)
+        lo, hi = 5, 66
+        ls, D = oracle.row_stats(q[0, :, h], k[0, :, g], v[0, :, g], do[0, :, h], lo, hi, mask=mask,
+                                 cu_seqlens=cu, chunk=7)
+        D_ref = (do[0, :, h].astype(np.float64) * o[0, :, h]).sum(1)
+        assert np.abs(ls[lo:hi] - lse[0, h, lo:hi]).max() < 1e-12
+        assert np.abs(D[lo:hi] - D_ref[lo:hi]).max() < 1e-12
+        assert np.all(ls[:lo] == -np.inf) and np.all(ls[hi:] == -np.inf)
+        assert np.all(D[:lo] == 0) and np.all(D[hi:] == 0)
+
+
+@pytest.mark.parametrize("mask", [MASK_CAUSAL, MASK_DOC_CAUSAL, MASK_NONE])
+def test_kv_cols_from_row_stats_match_full_backward(mask):
+    """dK, dV at key columns from supplied row statistics (row_stats over
+    rows_seeing(cols)) equal the full backward; rows_seeing is the smallest
+    range holding every row that sees a listed key (brute force)."""
+    n, H, G, d = 64, 4, 1, 8
+    q, k, v, do = _randn(1, n, H, d), _randn(1, n, G, d), _randn(1, n, G, d), _randn(1, n, H, d)
+    cu = np.array([0, 10, 40, n], np.int32) if mask == MASK_DOC_CAUSAL else None
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, mask=mask, cu_seqlens=cu)
+    for cols in (np.array([0, 1, 33]), np.array([12, 20]), np.array([45, 63])):
+        lo, hi = oracle.rows_seeing(cols, n, mask=mask, cu_seqlens=cu)
+        doc = None if cu is None else np.searchsorted(cu, np.arange(n), side="right") - 1
+        sees = [i for i in range(n) for j in cols
+                if mask == MASK_NONE or (j <= i and (doc is None or doc[i] == doc[j]))]
+        assert lo == min(sees) and hi == max(sees) + 1
+        stats = [oracle.row_stats(q[0, :, h], k[0, :, 0], v[0, :, 0], do[0, :, h], lo, hi, mask=mask,
+                                  cu_seqlens=cu, chunk=16) for h in range(H)]
+        ck, cv = oracle.kv_cols([q[0, :, h] for h in range(H)], [do[0, :, h] for h in range(H)],
+                                k[0, :, 0], v[0, :, 0], cols, mask=mask, cu_seqlens=cu, stats=stats)
+        assert np.abs(ck - dk[0, cols, 0]).max() < 1e-12
+        assert np.abs(cv - dv[0, cols, 0]).max() < 1e-12
+
+
+@pytest.mark.parametrize("mask", [MASK_CAUSAL, MASK_DOC_CAUSAL, MASK_NONE])
 def test_row_step_sums_to_full_backward(mask):
     """The per-row step (used to time the oracle on a row sample) summed over
     every row gives exactly the full forward and backward of the head."""
