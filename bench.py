@@ -82,19 +82,24 @@ def algorithmic_work(inp):
     pairs = causal_pairs(inp)
     qb = B * n * H * d * 2
     kvb = B * n * G * d * 2
+    n_pad = (n + 127) // 128 * 128
     w = {
         "attn_fwd_sm100": ("flops", 4.0 * B * H * d * pairs),
-        "attn_dkdv_sm100": ("flops", 8.0 * B * H * d * pairs),   # S, dP, dV, dK
-        "attn_dq_sm100": ("flops", 2.0 * B * H * d * pairs),     # dQ (S, dP recomputed)
-        # bf16: reads O, dO, LSE; writes D and LSE log2(e)
-        "attn_bwd_stats": ("bytes", 2.0 * qb + 3 * B * n * H * 4),
+        "attn_bwd_sm100": ("flops", 10.0 * B * H * d * pairs),   # S, dP, dV, dK, dQ in one pass
+        "attn_dkdv_sm100": ("flops", 8.0 * B * H * d * pairs),   # deterministic path: S, dP, dV, dK
+        "attn_dq_sm100": ("flops", 2.0 * B * H * d * pairs),     # deterministic path: dQ (S, dP recomputed)
+        # reads O, dO, LSE; writes D and LSE log2(e); zeroes the fp32 dQ accumulator
+        "attn_bwd_stats": ("bytes", 2.0 * qb + 3 * B * n * H * 4 + B * H * n_pad * d * 4.0),
+        # reads the fp32 dQ accumulator, writes dQ (bf16, seq layout)
+        "attn_dq_convert": ("bytes", B * H * n * d * 4.0 + qb),
     }
     if "logits" in inp:
         valid = int((inp["labels"] != -100).sum())
         w["loss_partial"] = ("bytes", valid * inp["vocab"] * 2.0 + inp["labels"].numel() * 4)
-    # permutations: one read + one write of every element, per step
+    # permutations: one read + one write of every element, per step (the
+    # head->seq direction is done by the attention kernels' epilogues)
     w["seq_to_head"] = ("bytes_step", 2.0 * (qb + 2 * kvb + qb))    # Q, K, V, dO
-    w["head_to_seq"] = ("bytes_step", 2.0 * (qb + qb + 2 * kvb))    # O, dQ, dK, dV
+    w["head_to_seq"] = ("bytes_step", 2.0 * (qb + qb + 2 * kvb))    # O, dQ, dK, dV (when run separately)
     return w, pairs
 
 
@@ -119,10 +124,11 @@ class Layer:
         self.kh = U.ulysses_seq_to_head(self.k, P)
         self.vh = U.ulysses_seq_to_head(self.v, P)
         self.doh = U.ulysses_seq_to_head(self.do, P)
-        self.oh, self.lse = U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu)
-        self.o = U.ulysses_head_to_seq(self.oh, P)
-        self.dqh, self.dkh, self.dvh = (torch.empty_like(x) for x in (self.qh, self.kh, self.vh))
-        desc = U._desc_from(self.qh, self.kh, self.mask, self.cu, 0.0)
+        # the layer's outputs O, dQ, dK, dV go straight to the seq layout (the
+        # second all-to-all in the attention kernels' epilogues)
+        self.o, self.lse = U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu,
+                                              out_seq_layout=True)
+        desc = U._desc_from(self.qh, self.kh, self.mask, self.cu, 0.0, out_seq_layout=True)
         self.ws = torch.empty(max(256, U.ulysses_attn_bwd_workspace_size(desc)), dtype=torch.uint8, device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(x) for x in (self.q, self.k, self.v))
         if self.logits is not None:
@@ -143,27 +149,26 @@ class Layer:
                                           workspace=self.lbws)
 
     def fwd_step(self):
-        """The forward half alone: seq->head(Q, K, V), attention forward, head->seq(O)."""
+        """The forward half alone: seq->head(Q, K, V), attention forward writing O
+        in the seq layout."""
         U, P = self.U, self.P
         U.ulysses_seq_to_head(self.q, P, out=self.qh)
         U.ulysses_seq_to_head(self.k, P, out=self.kh)
         U.ulysses_seq_to_head(self.v, P, out=self.vh)
-        U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.oh, lse=self.lse)
-        U.ulysses_head_to_seq(self.oh, P, out=self.o)
+        U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.o, lse=self.lse,
+                           out_seq_layout=True)
 
     def step(self):
         U, P = self.U, self.P
         U.ulysses_seq_to_head(self.q, P, out=self.qh)
         U.ulysses_seq_to_head(self.k, P, out=self.kh)
         U.ulysses_seq_to_head(self.v, P, out=self.vh)
-        U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.oh, lse=self.lse)
-        U.ulysses_head_to_seq(self.oh, P, out=self.o)
+        U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.o, lse=self.lse,
+                           out_seq_layout=True)
         U.ulysses_seq_to_head(self.do, P, out=self.doh)
-        U.ulysses_attn_bwd(self.qh, self.kh, self.vh, self.oh, self.lse, self.doh, mask=self.mask,
-                           cu_seqlens=self.cu, dq=self.dqh, dk=self.dkh, dv=self.dvh, workspace=self.ws)
-        U.ulysses_head_to_seq(self.dqh, P, out=self.dq)
-        U.ulysses_head_to_seq(self.dkh, P, out=self.dk)
-        U.ulysses_head_to_seq(self.dvh, P, out=self.dv)
+        U.ulysses_attn_bwd(self.qh, self.kh, self.vh, self.o, self.lse, self.doh, mask=self.mask,
+                           cu_seqlens=self.cu, dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws,
+                           out_seq_layout=True)
         if self.logits is not None:
             U.ulysses_loss_aggregate(self.logits, self.labels, P, shard_sum=self.S, shard_count=self.C,
                                      loss=self.L, workspace=self.lws)
@@ -289,6 +294,7 @@ def load_peaks():
 
 def kernel_source_hash(kernel: str) -> str:
     files = {"attn_fwd_sm100": "attn_fwd_sm100.cu", "attn_dkdv_sm100": "attn_bwd_sm100.cu",
+             "attn_bwd_sm100": "attn_bwd_fused_sm100.cu", "attn_dq_convert": "attn_bwd_fused_sm100.cu",
              "attn_dq_sm100": "attn_bwd_sm100.cu", "seq_to_head": "permute.cu", "head_to_seq": "permute.cu",
              "loss_partial": "loss.cu", "attn_bwd_stats": "attn_bwd_sm100.cu"}
     h = hashlib.sha256()
@@ -468,9 +474,11 @@ def run_ours(args, rank, world, dev):
         "attn_tflops": (fwd_fl * 3.5) / (attn_ms / 1e3) / 1e12,
         "attn_fwd_tflops": kernels.get("attn_fwd_sm100", {}).get("tflops"),
         "attn_bwd_tflops": (10.0 * inp["B"] * inp["H"] * inp["d"] * pairs) /
-                           (sum(kernels[k]["ms_per_step"] for k in ("attn_dkdv_sm100", "attn_dq_sm100",
-                                                                   "attn_bwd_stats") if k in kernels) / 1e3) / 1e12,
-        "permute_gbs": {k: kernels[k]["gbs"] for k in ("seq_to_head", "head_to_seq") if k in kernels},
+                           (sum(kernels[k]["ms_per_step"] for k in ("attn_bwd_sm100", "attn_dkdv_sm100",
+                                                                   "attn_dq_sm100", "attn_bwd_stats",
+                                                                   "attn_dq_convert") if k in kernels) / 1e3) / 1e12,
+        "permute_gbs": {"seq_to_head": kernels.get("seq_to_head", {}).get("gbs"),
+                        "head_to_seq": side.get("head_to_seq", {}).get("gbs")},
         "roofline": roof,
         "kernels": kernels,
         "forward_only": fwd_only,
@@ -516,6 +524,19 @@ def side_kernels(inp, dev, steps: int, peaks) -> dict:
         return {"ms_per_launch": tot / cnt, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                 "bytes_per_launch": nbytes, "note": note}
 
+    # the second all-to-all as its own kernel (the layer step folds it into the
+    # attention epilogues): O-sized head layout -> seq layout
+    P = inp["P"]
+    q_dev = inp["q"].to(dev)
+    qh = U.ulysses_seq_to_head(q_dev, P)
+    back = torch.empty_like(q_dev)
+    prof = timed(lambda: U.ulysses_head_to_seq(qh, P, out=back))
+    qbytes = q_dev.numel() * q_dev.element_size()
+    out["head_to_seq"] = entry(prof, "head_to_seq", 2.0 * qbytes,
+                               "O-sized tensor, head layout -> seq layout (one read, one write)")
+    if not torch.equal(back, q_dev):
+        raise RuntimeError("head_to_seq(seq_to_head(Q)) != Q")
+    del q_dev, qh, back
     P2 = 2 * G
     if n % P2 == 0:
         k2 = to_natural(inp["k"]).reshape(B, P2, n // P2, G, d).transpose(0, 1).contiguous().to(dev)

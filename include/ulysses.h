@@ -85,6 +85,18 @@ typedef struct {
                               * cu[num_docs] = n; shared by all batch rows        */
   int32_t num_docs;
   float softmax_scale;     /* 0 => 1/sqrt(head_dim)                               */
+  int32_t out_seq_layout;  /* 0: everything in the head layout.  1: the second
+                            * all-to-all (step 5) is done by the producing kernel:
+                            * o (fwd) and dq, dk, dv (bwd) are written straight into
+                            * the seq layout [P][B][n/P][heads][d], and the bwd
+                            * reads o in that layout too (as the fwd wrote it).
+                            * q, k, v, dout and lse stay in the head layout.      */
+  int32_t deterministic;   /* bf16 backward only.  0: one fused pass over the
+                            * (key tile, query tile) pairs; dQ is summed with fp32
+                            * adds in L2 and is not bitwise repeatable (dK, dV are).
+                            * 1: two passes, no atomics, bitwise repeatable (the dQ
+                            * pass recomputes the scores).  Needs a smaller
+                            * workspace.  Ignored by the f32 path (repeatable).   */
 } uly_attn_desc;
 
 /*
@@ -230,8 +242,15 @@ uly_status ulysses_attn_bwd_workspace_size(const uly_attn_desc *desc, size_t *by
 /*
  * Backward of the local attention (gradients of sum(O * dO)), head layout:
  * dout, dq like q; dk, dv like k (summed over the query heads of each KV
- * head); o and lse are the forward's outputs.  `workspace` must hold
- * ulysses_attn_bwd_workspace_size() bytes (caller owned, 256-byte aligned).
+ * head); o and lse are the forward's outputs.  With desc->out_seq_layout = 1,
+ * dq, dk, dv are written in the seq layout instead.  `workspace` must hold
+ * ulysses_attn_bwd_workspace_size() bytes (caller owned, 256-byte aligned,
+ * contents need not be initialised): per query row D_i = <dO_i, O_i> and
+ * LSE_i log2(e), and, for the fused bf16 backward (deterministic = 0), an fp32
+ * dQ accumulator of 512 bytes per query row (n rounded up to 128 per head).
+ * A malformed cu_seqlens (not starting at 0, decreasing, or not ending at n)
+ * sets ULY_ERR_SHAPE in the error word (fwd and bwd); its kernels stay inside
+ * their operands.
  */
 uly_status ulysses_attn_bwd(const uly_attn_desc *desc, const void *q, const void *k,
                             const void *v, const void *o, const float *lse, const void *dout,

@@ -21,7 +21,7 @@ LIB = os.path.join(HERE, "libulysses.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 SOURCES = ["api.cu", "prof.cu", "permute.cu", "loss.cu", "loss_noalloc.cu", "attn_f32.cu", "attn_fwd_sm100.cu",
-           "attn_bwd_sm100.cu", "proj_sm100.cu", "kv_copy.cu", "labels.cu"]
+           "attn_bwd_sm100.cu", "attn_bwd_fused_sm100.cu", "proj_sm100.cu", "kv_copy.cu", "labels.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-Wall", "-I", INCLUDE]
@@ -45,6 +45,7 @@ def _deps_mtime() -> float:
 REGISTER_SPLIT_KERNELS = {
     "attn_fwd_sm100.cu": [("attn_fwd_sm100_kernel", 168)],
     "attn_bwd_sm100.cu": [("attn_dkdv_sm100_kernel", 168), ("attn_dq_sm100_kernel", 168)],
+    "attn_bwd_fused_sm100.cu": [("attn_bwd_sm100_kernel", 128)],
 }
 
 

@@ -48,6 +48,7 @@ uly_status attn_f32_bwd_launch(const uly_attn_desc *, const HeadGeom &, const Ma
 uly_status attn_bf16_fwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
                                 const void *, const void *, const void *, void *, float *,
                                 cudaStream_t);
+size_t attn_bf16_bwd_workspace(const HeadGeom &, bool);
 uly_status attn_bf16_bwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
                                 const void *, const void *, const void *, const void *,
                                 const float *, const void *, void *, void *, void *, float *,
@@ -88,6 +89,8 @@ uly_status check_desc(const uly_attn_desc *d, HeadGeom &g, MaskInfo &mk) {
   if (d->mask < ULY_MASK_NONE || d->mask > ULY_MASK_DOC_CAUSAL) return ULY_ERR_UNSUPPORTED;
   if (d->mask == ULY_MASK_DOC_CAUSAL && (!d->cu_seqlens || d->num_docs < 1)) return ULY_ERR_NULL;
   if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return ULY_ERR_SHAPE;
+  if ((d->out_seq_layout != 0 && d->out_seq_layout != 1) || (d->deterministic != 0 && d->deterministic != 1))
+    return ULY_ERR_SHAPE;
   const long long heads_q = (long long)d->batch * d->n_q_heads;
   if (heads_q > 65535 || (d->seq_len + 63) / 64 > 65535) return ULY_ERR_SHAPE;  // grid limits
   if (d->dtype == ULY_F32 && d->head_dim != 64 && d->head_dim != 128) return ULY_ERR_UNSUPPORTED;
@@ -100,6 +103,7 @@ uly_status check_desc(const uly_attn_desc *d, HeadGeom &g, MaskInfo &mk) {
   g.gl = d->n_kv_heads / d->world;
   g.group = d->n_q_heads / d->n_kv_heads;
   g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)d->head_dim);
+  g.out_seq = d->out_seq_layout;
   mk.mask = d->mask;
   mk.n = d->seq_len;
   mk.cu = d->cu_seqlens;
@@ -296,9 +300,8 @@ uly_status ulysses_attn_bwd_workspace_size(const uly_attn_desc *d, size_t *bytes
   uly_status st = check_desc(d, g, mk);
   if (st != ULY_OK) return st;
   if (d->dtype == ULY_BF16) {
-    // D_i and LSE_i log2(e), query rows padded per head
-    const long long rows_pad = (long long)d->batch * d->n_q_heads * bwd_rows_padded(d->seq_len);
-    *bytes = 2 * sizeof(float) * (size_t)bwd_stats_stride(rows_pad);
+    // D_i and LSE_i log2(e), query rows padded per head (+ the fused pass's dQ accumulator)
+    *bytes = attn_bf16_bwd_workspace(g, d->deterministic != 0);
   } else {
     *bytes = align256(lse_bytes(d));  // D_i = <dO_i, O_i> for every query row
   }

@@ -67,21 +67,31 @@ struct BwdParams {
 
 // D_i = <dO_i, O_i> and LSE_i log2(e) of every query row (two rows per warp,
 // 16-byte loads), written to the padded per-head arrays; rows n..n_pad-1 get 0.
+// dq_acc (fused backward only, else null): the row's 128 fp32 dQ accumulators
+// are zeroed here, so the fused kernel finds them cleared.
+// O is read in the head layout, or in the seq layout when g.out_seq (the
+// layout the forward wrote it in); dO and LSE are in the head layout.
 __global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const __nv_bfloat16 *__restrict__ o,
                                                              const __nv_bfloat16 *__restrict__ dout,
                                                              const float *__restrict__ lse,
                                                              float *__restrict__ Dpad,
-                                                             float *__restrict__ L2pad, int n, int n_pad,
-                                                             long long rows_pad) {
+                                                             float *__restrict__ L2pad, float *__restrict__ dq_acc,
+                                                             HeadGeom g, int n_pad, long long rows_pad) {
+  const int n = g.n;
   const long long r = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
   const int l = threadIdx.x & 15;
+  if (dq_acc && r < rows_pad) {
+    float4 *z = reinterpret_cast<float4 *>(dq_acc + r * kHD) + 2 * l;
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const long long h = r / n_pad;
   const int i = (int)(r - h * n_pad);
   const bool valid = r < rows_pad && i < n;
   float acc = 0.f;
   if (valid) {
     const long long src = (h * n + i) * kHD;
-    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(o + src) + l);
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(o + g.q_out_row(h, i) * kHD) + l);
     const uint4 b = __ldg(reinterpret_cast<const uint4 *>(dout + src) + l);
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -381,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     __nv_bfloat16 *outp = (w == 0) ? prm.out0 : prm.out1;
     const float mul = (w == 0) ? 1.f : g.scale;
-    const long long orow = (long long)kvh * g.n + j;
+    const long long orow = (j < g.n) ? g.kv_out_row(kvh, j) : 0;
     if (ok && T > 0) {
       uint32_t rr[32];
 #pragma unroll
@@ -643,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_DS));
     }
     // epilogue: warpgroup w writes dQ columns [64w, 64w + 64)
+    const long long orow = valid ? g.q_out_row(qh, i) : 0;
     if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, abort_flag, prm.err));
     tc_fence_after();
     if (ok && NT > 0) {
@@ -651,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 2; ++c) {
         tmem_ld32(tmem + lane_off + kTdQ + 64 * w + 32 * c, rr);
         if (valid) {
-          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * w + 32 * c);
+          uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + orow * kHD + 64 * w + 32 * c);
           const float sc = g.scale;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -665,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else if (NT == 0 && valid) {
-      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + qrow * kHD + 64 * w);
+      uint4 *dptr = reinterpret_cast<uint4 *>(prm.out0 + orow * kHD + 64 * w);
       for (int u = 0; u < 8; ++u) dptr[u] = make_uint4(0, 0, 0, 0);
     }
   }
@@ -681,6 +692,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+uly_status attn_bf16_bwd_fused_launch(const HeadGeom &g, const MaskInfo &mk, const void *q, const void *k,
+                                      const void *v, const void *dout, void *dq, void *dk, void *dv,
+                                      const float *Dv, const float *L2, float *dq_acc, int n_pad,
+                                      cudaStream_t stream);
+
+// Workspace of the bf16 backward: D and LSE log2(e) (bwd_stats_stride floats
+// each), then, for the fused backward, the fp32 dQ accumulator
+// [query heads][n_pad][128] (256-byte aligned).
+size_t attn_bf16_bwd_workspace(const HeadGeom &g, bool deterministic) {
+  const long long rows_pad = (long long)g.P * g.B * g.hl * bwd_rows_padded(g.n);
+  const size_t stats = 2 * sizeof(float) * (size_t)bwd_stats_stride(rows_pad);
+  if (deterministic) return stats;
+  return ((stats + 255) & ~size_t(255)) + (size_t)rows_pad * kHD * sizeof(float);
+}
+
 uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const MaskInfo &mk,
                                 const void *q, const void *k, const void *v, const void *o,
                                 const float *lse, const void *dout, void *dq, void *dk, void *dv,
@@ -688,15 +714,23 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   const int qheads = g.P * g.B * g.hl, kvheads = g.P * g.B * g.gl;
   const int n_pad = bwd_rows_padded(g.n);
   const long long rows_pad = (long long)qheads * n_pad;
+  const bool fused = d->deterministic == 0;
   float *Dv = workspace;
   float *L2 = workspace + bwd_stats_stride(rows_pad);
+  float *dq_acc = nullptr;
+  if (fused) {
+    const size_t stats = 2 * sizeof(float) * (size_t)bwd_stats_stride(rows_pad);
+    dq_acc = reinterpret_cast<float *>(reinterpret_cast<char *>(workspace) + ((stats + 255) & ~size_t(255)));
+  }
   if (rows_pad > 0) {
     prof::Scope scope(prof::K_ATTN_BWD_STATS, stream);
     attn_bwd_stats_kernel<<<(unsigned)((rows_pad + 15) / 16), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, Dv, L2, g.n,
-        n_pad, rows_pad);
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, Dv, L2, dq_acc,
+        g, n_pad, rows_pad);
     note_launches(1);
   }
+  if (fused)
+    return attn_bf16_bwd_fused_launch(g, mk, q, k, v, dout, dq, dk, dv, Dv, L2, dq_acc, n_pad, stream);
   CUtensorMap mK128, mV128, mQ128, mO128, mK64, mV64;
   if (!make_tmap_heads_bf16(&mK128, k, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&mV128, v, kHD, g.n, kvheads, 128) ||

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32_kernel(
     }
   }
   if (valid) {
-    float *orow = o + ((long long)qh * g.n + i) * D + part * DQ;
+    float *orow = o + g.q_out_row(qh, i) * D + part * DQ;
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
     for (int x = 0; x < DQ; ++x) orow[x] = acc[x] * inv;
@@ -171,7 +171,9 @@ __global__ void __launch_bounds__(kThreads) attn_dq_f32_kernel(
   }
   if (valid) {
 #pragma unroll
-    for (int x = 0; x < DQ; ++x) dq[ro * D + part * DQ + x] = acc[x] * g.scale;
+    const long long out = g.q_out_row(qh, i);
+#pragma unroll
+    for (int x = 0; x < DQ; ++x) dq[out * D + part * DQ + x] = acc[x] * g.scale;
   }
 }
 
@@ -249,25 +251,29 @@ __global__ void __launch_bounds__(kThreads) attn_dkdv_f32_kernel(
     }
   }
   if (valid) {
+    const long long out = g.kv_out_row(kh, j);
 #pragma unroll
     for (int x = 0; x < DQ; ++x) {
-      dk[ko * D + part * DQ + x] = ak[x] * g.scale;
-      dvv[ko * D + part * DQ + x] = av[x];
+      dk[out * D + part * DQ + x] = ak[x] * g.scale;
+      dvv[out * D + part * DQ + x] = av[x];
     }
   }
 }
 
-// D_i = <dO_i, O_i> (fp32 path), one warp per row.
+// D_i = <dO_i, O_i> (fp32 path), one warp per row; dout in the head layout,
+// O in the head or (g.out_seq) the seq layout.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_bwd_dot_kernel(const T *__restrict__ o,
                                                            const T *__restrict__ dout,
-                                                           float *__restrict__ Dv, long long rows) {
+                                                           float *__restrict__ Dv, long long rows, HeadGeom g) {
   const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
+  const long long h = r / g.n;
+  const long long ro = g.q_out_row(h, (int)(r - h * g.n));
   float acc = 0.f;
   for (int x = lane; x < D; x += 32)
-    acc = fmaf(static_cast<float>(o[r * D + x]), static_cast<float>(dout[r * D + x]), acc);
+    acc = fmaf(static_cast<float>(o[ro * D + x]), static_cast<float>(dout[r * D + x]), acc);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) Dv[r] = acc;
@@ -294,16 +300,16 @@ uly_status attn_f32_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const 
 }
 
 uly_status attn_bwd_dot_launch(int dtype, int head_dim, const void *o, const void *dout, float *Dv,
-                               long long rows, cudaStream_t stream) {
+                               long long rows, const HeadGeom &g, cudaStream_t stream) {
   const unsigned blocks = (unsigned)((rows + 7) / 8);
   if (blocks == 0) return ULY_OK;
   prof::Scope scope(prof::K_ATTN_BWD_DOT, stream);
   if (dtype == ULY_F32 && head_dim == 64)
     attn_bwd_dot_kernel<float, 64><<<blocks, 256, 0, stream>>>(
-        static_cast<const float *>(o), static_cast<const float *>(dout), Dv, rows);
+        static_cast<const float *>(o), static_cast<const float *>(dout), Dv, rows, g);
   else if (dtype == ULY_F32 && head_dim == 128)
     attn_bwd_dot_kernel<float, 128><<<blocks, 256, 0, stream>>>(
-        static_cast<const float *>(o), static_cast<const float *>(dout), Dv, rows);
+        static_cast<const float *>(o), static_cast<const float *>(dout), Dv, rows, g);
   else
     return ULY_ERR_UNSUPPORTED;
   note_launches(1);
@@ -315,7 +321,7 @@ uly_status attn_f32_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const 
                                const float *lse, const void *dout, void *dq, void *dk, void *dv,
                                float *Dv, cudaStream_t stream) {
   const long long qrows = (long long)g.P * g.B * g.hl * g.n;
-  uly_status st = attn_bwd_dot_launch(ULY_F32, d->head_dim, o, dout, Dv, qrows, stream);
+  uly_status st = attn_bwd_dot_launch(ULY_F32, d->head_dim, o, dout, Dv, qrows, g, stream);
   if (st != ULY_OK) return st;
   const float *Q = static_cast<const float *>(q), *K = static_cast<const float *>(k),
               *V = static_cast<const float *>(v), *dO = static_cast<const float *>(dout);

@@ -309,7 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue
     if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + wg), 0, abort_flag, prm.err));
     tc_fence_after();
-    const long long orow = (long long)(qhead0 + wg) * g.n + i;
+    // O goes to the head layout, or straight to the seq layout (the second
+    // all-to-all in the epilogue); LSE stays in the head layout
+    const long long hrow = (long long)(qhead0 + wg) * g.n + i;
+    const long long orow = valid ? g.q_out_row(qhead0 + wg, i) : 0;
     const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
     if (ok && NT > 0) {
       uint32_t r[32];
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; u < kHD / 8; ++u) dst[u] = make_uint4(0, 0, 0, 0);
     }
     if (valid && (ok || NT == 0))
-      prm.lse[orow] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      prm.lse[hrow] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
   }
 
   tc_fence_before();

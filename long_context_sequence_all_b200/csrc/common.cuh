@@ -99,10 +99,32 @@ struct MaskInfo {
 __host__ __device__ inline int bwd_rows_padded(int n) { return (n + 127) / 128 * 128; }
 __host__ __device__ inline long long bwd_stats_stride(long long rows_pad) { return (rows_pad + 63) / 64 * 64; }
 
+// Row of the seq layout [P][B][n/P][heads][d] that holds row t of head hx of
+// the head layout [P][B][hl][n][d] (hx = (r*B + b)*hl + hh, heads = P*hl):
+// rank t / (n/P), position t % (n/P), global head r*hl + hh.  This is the
+// second all-to-all (step 5) for one row.
+__host__ __device__ inline long long seq_row_of(long long hx, int t, int B, int n, int P, int hl) {
+  const int s = n / P;
+  const long long bh = (long long)B * hl;
+  const long long r = hx / bh;
+  const long long rem = hx - r * bh;
+  const long long b = rem / hl, hh = rem - b * hl;
+  const int rt = t / s, tt = t - rt * s;
+  return (((long long)rt * B + b) * s + tt) * ((long long)P * hl) + r * hl + hh;
+}
+
 // Per-launch geometry of the head layout shared by the attention kernels.
 struct HeadGeom {
   int B, n, P, hl, gl, group;  // hl = H/P, gl = G/P, group = H/G
   float scale;                 // softmax scale
+  int out_seq;                 // 1: outputs go to the seq layout (uly_attn_desc.out_seq_layout)
+  // output row of query-head row (qh, t) and of KV-head row (kvh, t)
+  __host__ __device__ long long q_out_row(long long qh, int t) const {
+    return out_seq ? seq_row_of(qh, t, B, n, P, hl) : qh * n + t;
+  }
+  __host__ __device__ long long kv_out_row(long long kvh, int t) const {
+    return out_seq ? seq_row_of(kvh, t, B, n, P, gl) : kvh * n + t;
+  }
 };
 
 }  // namespace uly

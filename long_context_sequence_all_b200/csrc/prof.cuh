@@ -31,6 +31,8 @@ enum Kernel {
   K_QKV_PROJ,
   K_O_PROJ,
   K_CHECK_CU,
+  K_ATTN_BWD_SM100,
+  K_ATTN_DQ_CONVERT,
   K_COUNT
 };
 

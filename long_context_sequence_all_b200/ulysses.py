@@ -45,7 +45,8 @@ class AttnDesc(ctypes.Structure):
                 ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int32), ("mask", ctypes.c_int32),
                 ("cu_seqlens", ctypes.c_void_p), ("num_docs", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("out_seq_layout", ctypes.c_int32),
+                ("deterministic", ctypes.c_int32)]
 
 
 _lib = None
@@ -131,11 +132,12 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise UlyssesError(3, f"dtype {t.dtype}")
 
 
-def make_desc(B, n, P, H, G, d, dtype_code, mask, cu_seqlens=None, scale=0.0) -> AttnDesc:
+def make_desc(B, n, P, H, G, d, dtype_code, mask, cu_seqlens=None, scale=0.0, out_seq_layout=False,
+              deterministic=False) -> AttnDesc:
     nd = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     return AttnDesc(B, n, P, H, G, d, dtype_code, mask,
                     ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None,
-                    nd, float(scale))
+                    nd, float(scale), int(bool(out_seq_layout)), int(bool(deterministic)))
 
 
 # --------------------------------------------------------------- all-to-alls
@@ -264,19 +266,27 @@ def ulysses_o_proj(o: torch.Tensor, w_o: torch.Tensor, P: int, y=None, stream=No
 
 # ----------------------------------------------------------------- attention
 
-def _desc_from(q, k, mask, cu_seqlens, scale):
+def _desc_from(q, k, mask, cu_seqlens, scale, out_seq_layout=False, deterministic=False):
     P, B, hl, n, d = q.shape
     gl = k.shape[2]
-    return make_desc(B, n, P, hl * P, gl * P, d, _dtype_code(q), mask, cu_seqlens, scale)
+    return make_desc(B, n, P, hl * P, gl * P, d, _dtype_code(q), mask, cu_seqlens, scale,
+                     out_seq_layout, deterministic)
+
+
+def _seq_shape(x):
+    """Seq-layout shape [P][B][n/P][heads][d] of a head-layout tensor [P][B][heads/P][n][d]."""
+    P, B, hx, n, d = x.shape
+    return (P, B, n // P, hx * P, d)
 
 
 def ulysses_attn_fwd(q, k, v, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0, o=None, lse=None,
-                     stream=None):
-    """Head layout in/out: q [P][B][H/P][n][d], k, v [P][B][G/P][n][d] ->
-    o like q, lse float32 [P][B][H/P][n]."""
-    desc = _desc_from(q, k, mask, cu_seqlens, scale)
+                     out_seq_layout=False, stream=None):
+    """Head layout in: q [P][B][H/P][n][d], k, v [P][B][G/P][n][d] -> o like q
+    (or, with out_seq_layout, o in the seq layout [P][B][n/P][H][d]: the second
+    all-to-all done by the attention kernel), lse float32 [P][B][H/P][n]."""
+    desc = _desc_from(q, k, mask, cu_seqlens, scale, out_seq_layout)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(_seq_shape(q), dtype=q.dtype, device=q.device) if out_seq_layout else torch.empty_like(q)
     if lse is None:
         lse = torch.empty(q.shape[:4], dtype=torch.float32, device=q.device)
     _check(lib().ulysses_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse),
@@ -292,12 +302,17 @@ def ulysses_attn_bwd_workspace_size(desc: AttnDesc) -> int:
 
 
 def ulysses_attn_bwd(q, k, v, o, lse, dout, mask=MASK_CAUSAL, cu_seqlens=None, scale=0.0,
-                     dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """Gradients of sum(O * dO) in head layout: dq like q, dk/dv like k."""
-    desc = _desc_from(q, k, mask, cu_seqlens, scale)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+                     dq=None, dk=None, dv=None, workspace=None, out_seq_layout=False,
+                     deterministic=False, stream=None):
+    """Gradients of sum(O * dO), inputs in the head layout: dq like q, dk/dv
+    like k, or all three in the seq layout with out_seq_layout.
+    deterministic: the atomic-free two-pass backward (bitwise repeatable)."""
+    desc = _desc_from(q, k, mask, cu_seqlens, scale, out_seq_layout, deterministic)
+    mk = (lambda x: torch.empty(_seq_shape(x), dtype=x.dtype, device=x.device)) if out_seq_layout \
+        else torch.empty_like
+    dq = mk(q) if dq is None else dq
+    dk = mk(k) if dk is None else dk
+    dv = mk(v) if dv is None else dv
     need = ulysses_attn_bwd_workspace_size(desc)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)

@@ -140,6 +140,28 @@ def test_attn_desc_validation(L):
     assert L.ulysses_attn_bwd(ctypes.byref(d), *[vp(1 << (20 + i)) for i in range(9)], None, 0, None) == 10
 
 
+def test_attn_desc_flags_and_workspace_sizes(L):
+    """out_seq_layout and deterministic take 0 or 1.  The bf16 workspace holds
+    D and LSE log2(e) per query row (n rounded up to 128 per head); the fused
+    backward adds its fp32 dQ accumulator (512 bytes per padded query row)
+    after a 256-byte boundary."""
+    from long_context_sequence_all_b200 import ulysses as U
+    n = ctypes.c_size_t(0)
+    B, N, P, H, G = 1, 8000, 4, 32, 8
+    rows_pad = B * H * ((N + 127) // 128 * 128)
+    stats = 2 * 4 * ((rows_pad + 63) // 64 * 64)
+    det = U.make_desc(B, N, P, H, G, 128, U.ULY_BF16, 1, deterministic=True)
+    assert L.ulysses_attn_bwd_workspace_size(ctypes.byref(det), ctypes.byref(n)) == 0
+    assert n.value == stats
+    fused = U.make_desc(B, N, P, H, G, 128, U.ULY_BF16, 1, out_seq_layout=True)
+    assert L.ulysses_attn_bwd_workspace_size(ctypes.byref(fused), ctypes.byref(n)) == 0
+    assert n.value == (stats + 255) // 256 * 256 + rows_pad * 128 * 4
+    for field in ("out_seq_layout", "deterministic"):
+        bad = U.make_desc(B, N, P, H, G, 128, U.ULY_BF16, 1)
+        setattr(bad, field, 2)
+        assert L.ulysses_attn_bwd_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == 2
+
+
 def test_loss_validation(L):
     vp = ctypes.c_void_p
     n = ctypes.c_size_t(0)
