@@ -348,6 +348,20 @@ uly_status ulysses_read_error(int32_t *word);
  * The record is cleared. */
 uly_status ulysses_read_error_info(int32_t *info, int32_t n);
 
+/*
+ * Failure detection (no counterpart on the pages: the tcgen05 kernels wait on
+ * mbarriers, and every such wait is bounded).  Sets how many SM clock cycles a
+ * pipeline wait of the attention and projection kernels launched from now on
+ * may last before the kernel records ULY_ERR_TIMEOUT (and where, see
+ * ulysses_read_error_info), drains its copies and MMAs, frees its tensor
+ * memory and returns.  cycles = 0 restores the built-in limit (2e9 cycles,
+ * about a second); a shorter limit also makes the waits poll without
+ * suspending.  Meant for tests of that path: a limit of a few hundred cycles
+ * makes the first wait for a tile copy run out.  Process-wide, host only.
+ * Returns ULY_ERR_SHAPE for a negative value.
+ */
+uly_status ulysses_set_wait_limit(int64_t cycles);
+
 /* Human-readable name of a status. */
 const char *ulysses_status_string(uly_status status);
 

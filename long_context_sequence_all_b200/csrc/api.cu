@@ -21,6 +21,13 @@ int *g_err_ptr[64] = {nullptr};
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+namespace {
+constexpr long long kDefaultWaitLimit = 2000000000ll;   // sm100::kWaitLimitCycles
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+}  // namespace
+
+long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
+
 int *error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
@@ -420,6 +427,13 @@ uly_status ulysses_error_word(int32_t **dev_word) {
   int *p = error_word();
   if (!p) return ULY_ERR_CUDA;
   *dev_word = p;
+  return ULY_OK;
+}
+
+uly_status ulysses_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return ULY_ERR_SHAPE;
+  g_wait_limit.store(cycles == 0 || cycles > kDefaultWaitLimit ? kDefaultWaitLimit : cycles,
+                     std::memory_order_relaxed);
   return ULY_OK;
 }
 

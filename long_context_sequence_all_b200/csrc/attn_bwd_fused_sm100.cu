@@ -92,6 +92,7 @@ struct FusedParams {
   float scale_log2;
   int n_pad;
   int *err;
+  long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -164,32 +165,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
           const long long srow = (long long)(qh_base + e) * prm.n_pad + i0;
           const int sq = t % kQStages, uq = t / kQStages;
-          if (uq > 0 && !mbar_wait(bar(B_QE + sq), (uq - 1) & 1, abort_flag, prm.err)) break;
+          if (uq > 0 && !mbar_wait(bar(B_QE + sq), (uq - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
           mbar_arrive_expect_tx(bar(B_QF + sq), kTile + kBQ * 4);
           for (int c = 0; c < 2; ++c)
             tma_load_3d(sb + kOffQ + sq * kTile + c * 16384, &tmQ, bar(B_QF + sq), c * 64, i0, qh_base + e);
           bulk_load(sb + kOffLse + sq * kBQ * 4, prm.lse2 + srow, kBQ * 4, bar(B_QF + sq));
           issued_q = t + 1;
           const int so = t % kOStages, uo = t / kOStages;
-          if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err)) break;
+          if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
           mbar_arrive_expect_tx(bar(B_OF + so), kTile + kBQ * 4);
           for (int c = 0; c < 2; ++c)
             tma_load_3d(sb + kOffO + so * kTile + c * 16384, &tmO, bar(B_OF + so), c * 64, i0, qh_base + e);
           bulk_load(sb + kOffD + so * kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_OF + so));
           issued_o = t + 1;
         }
-        if (*abort_flag) {
-          // let the copies already in flight land before the CTA exits
-          for (int t = (issued_q > kQStages ? issued_q - kQStages : 0); t < issued_q; ++t)
-            mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, nullptr, prm.err);
-          for (int t = (issued_o > kOStages ? issued_o - kOStages : 0); t < issued_o; ++t)
-            mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, nullptr, prm.err);
-        }
+        // Every copy issued lands before the CTA can exit, also when a consumer
+        // gave up waiting for it (older stages were consumed, so landed,
+        // before they were refilled); on the normal path these return at once.
+        mbar_wait(bar(B_KV), 0, nullptr, prm.err);
+        for (int t = (issued_q > kQStages ? issued_q - kQStages : 0); t < issued_q; ++t)
+          mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, nullptr, prm.err);
+        for (int t = (issued_o > kOStages ? issued_o - kOStages : 0); t < issued_o; ++t)
+          mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, nullptr, prm.err);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA
       if (lane == 0 && T > 0) {
-        bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
+        bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err, prm.wait_limit);
         uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
         uint64_t dKt = sdesc_sw128(sb + kOffK, 16384, 1024);   // K^T (A of dQ^T): MN-major
         uint64_t dSb = sdesc_sw128(sb + kOffS, 16384, 1024);   // dS^T (B of dQ^T): MN-major
@@ -210,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(B_DPF));
         };
-        if (ok) ok = mbar_wait2(bar(B_QF), 0, bar(B_OF), 0, abort_flag, prm.err);
+        if (ok) ok = mbar_wait2(bar(B_QF), 0, bar(B_OF), 0, abort_flag, prm.err, prm.wait_limit);
         if (ok) {
           tc_fence_after();
           issue_s(sdesc_sw128(sb + kOffQ, 16, 1024));
@@ -234,8 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dOn = sdesc_sw128(sb + kOffO + so1 * kTile, 16, 1024);     // next dP^T: B = next dO
           // dV += P^T dO_t: A from TMEM (query columns [0,64) in the S^T
           // columns [0,32), [64,128) in [64,96))
-          ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + sq1), pq1, abort_flag, prm.err)
-                    : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
+          ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + sq1), pq1, abort_flag, prm.err, prm.wait_limit)
+                    : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the next tile's S^T over this tile's P^T (after the dV MMA in issue order)
           if (more) issue_s(dQn);
           // dS^T of the tile is in shared memory and the dP^T columns are read
-          ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err);
+          ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
           // dQ^T = K^T dS^T into the dP^T columns: M = head dims, N = queries,
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bar(B_DSE));
           if (more) {
             // the next dP^T reuses the dQ^T columns once the dQ warpgroup has read them
-            ok = mbar_wait2(bar(B_DQE), t & 1, bar(B_OF + so1), po1, abort_flag, prm.err);
+            ok = mbar_wait2(bar(B_DQE), t & 1, bar(B_OF + so1), po1, abort_flag, prm.err, prm.wait_limit);
             if (!ok) break;
             tc_fence_after();
             issue_dp(dOn);
@@ -277,10 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           sq = sq1; so = so1; pq = pq1; po = po1;
         }
         if (ok) tc_commit(bar(B_DONE));
-        if (!ok) {
-          tc_commit(bar(B_DRAIN));
-          mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
-        }
+        // every MMA issued has completed before TMEM can be released
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
       }
     }
   } else if (warp < 12) {
@@ -302,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *lsm = reinterpret_cast<const float *>(smem + kOffLse + sq * kBQ * 4) + 64 * w;
       const float *dsm = reinterpret_cast<const float *>(smem + kOffD + so * kBQ * 4) + 64 * w;
       // P^T over this warpgroup's first 32 columns of S^T
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err) &&
-                                       mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
+                                       mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
@@ -328,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_PS));
       // dS^T = P^T (dP^T - D) into shared memory
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + so), (t / kOStages) & 1, abort_flag, prm.err) &&
-                                       mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + so), (t / kOStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
+                                       mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       uint32_t dp[64];
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the previous tile's dQ^T and dK MMAs have read the buffer
       if (t > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSE), (t - 1) & 1, abort_flag, prm.err));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSE), (t - 1) & 1, abort_flag, prm.err, prm.wait_limit));
         if (!ok) break;
       }
 #pragma unroll
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_DS));
     }
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (scaled)
-    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err));
+    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err, prm.wait_limit));
     tc_fence_after();
     __nv_bfloat16 *outp = (w == 0) ? prm.dv : prm.dk;
     const float mul = (w == 0) ? 1.f : g.scale;
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < T; ++t) {
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ;
       float *dst = prm.dq_acc + ((long long)(qh_base + e) * prm.n_pad + i0) * kHD + dcol;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQF), t & 1, abort_flag, prm.err))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQF), t & 1, abort_flag, prm.err, prm.wait_limit))) break;
       tc_fence_after();
       uint32_t v[64];
       tmem_ld64(tX, v);
@@ -462,6 +463,7 @@ uly_status attn_bf16_bwd_fused_launch(const HeadGeom &g, const MaskInfo &mk, con
   prm.scale_log2 = g.scale * kLog2e;
   prm.n_pad = n_pad;
   prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
   {
     prof::Scope scope(prof::K_ATTN_BWD_SM100, stream);
     attn_bwd_sm100_kernel<<<dim3(kvheads, (g.n + kBN - 1) / kBN), kThreads, kSmemBytes, stream>>>(mK, mV, mQ, mO,

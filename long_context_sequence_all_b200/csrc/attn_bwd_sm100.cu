@@ -63,6 +63,7 @@ struct BwdParams {
   float scale_log2;
   int n_pad;          // n rounded up to a multiple of 128
   int *err;
+  long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
 };
 
 // D_i = <dO_i, O_i> and LSE_i log2(e) of every query row (two rows per warp,
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long srow = (long long)(qh_base + e) * prm.n_pad + i0;
         // Q tile and its LSE
         const int sq = t % kQStages, uq = t / kQStages;
-        if (uq > 0 && !mbar_wait(bar(B_QE + sq), (uq - 1) & 1, abort_flag, prm.err)) break;
+        if (uq > 0 && !mbar_wait(bar(B_QE + sq), (uq - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
         mbar_arrive_expect_tx(bar(B_QF + sq), kTile + kBQ * 4);
         for (int c = 0; c < 2; ++c)
           tma_load_3d(sb + kOffQ + sq * kTile + c * 16384, &tmQ, bar(B_QF + sq), c * 64, i0, qh_base + e);
@@ -226,23 +227,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued_q = t + 1;
         // dO tile and its D
         const int so = t % kOStages, uo = t / kOStages;
-        if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err)) break;
+        if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
         mbar_arrive_expect_tx(bar(B_OF + so), kTile + kBQ * 4);
         for (int c = 0; c < 2; ++c)
           tma_load_3d(sb + kOffO + so * kTile + c * 16384, &tmO, bar(B_OF + so), c * 64, i0, qh_base + e);
         bulk_load(sb + kOffD + so * kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_OF + so));
         issued_o = t + 1;
       }
-      if (*abort_flag) {
-        for (int t = (issued_q > kQStages ? issued_q - kQStages : 0); t < issued_q; ++t)
-          mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, nullptr, prm.err);
-        for (int t = (issued_o > kOStages ? issued_o - kOStages : 0); t < issued_o; ++t)
-          mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, nullptr, prm.err);
-      }
+      // every copy issued lands before the CTA can exit (see the forward)
+      mbar_wait(bar(B_KV), 0, nullptr, prm.err);
+      for (int t = (issued_q > kQStages ? issued_q - kQStages : 0); t < issued_q; ++t)
+        mbar_wait(bar(B_QF + t % kQStages), (t / kQStages) & 1, nullptr, prm.err);
+      for (int t = (issued_o > kOStages ? issued_o - kOStages : 0); t < issued_o; ++t)
+        mbar_wait(bar(B_OF + t % kOStages), (t / kOStages) & 1, nullptr, prm.err);
     }
   } else if (warp == 1) {
     if (lane == 0 && T > 0) {
-      bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err);
+      bool ok = mbar_wait(bar(B_KV), 0, abort_flag, prm.err, prm.wait_limit);
       const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024), dV = sdesc_sw128(sb + kOffV, 16, 1024);
       // S^T = K Q^T into the S^T columns; dP^T = V dO^T into the dP^T columns
       auto issue_s = [&](uint64_t dQ) {
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(B_DPF));
       };
-      if (ok) ok = mbar_wait2(bar(B_QF), 0, bar(B_OF), 0, abort_flag, prm.err);
+      if (ok) ok = mbar_wait2(bar(B_QF), 0, bar(B_OF), 0, abort_flag, prm.err, prm.wait_limit);
       if (ok) {
         tc_fence_after();
         issue_s(sdesc_sw128(sb + kOffQ, 16, 1024));
@@ -284,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dOn = sdesc_sw128(sb + kOffO + so1 * kTile, 16, 1024);     // next dP^T: B = next dO
         // dV += P^T dO_t: A from TMEM (query columns [0,64) in the S^T
         // columns [0,32), [64,128) in [64,96))
-        ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + sq1), pq1, abort_flag, prm.err)
-                  : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err);
+        ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + sq1), pq1, abort_flag, prm.err, prm.wait_limit)
+                  : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err, prm.wait_limit);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the next tile's S^T over this tile's P^T (after the dV MMA in issue order)
         if (more) issue_s(dQn);
         // dK += dS^T Q_t: A from TMEM (dS^T over the dP^T columns)
-        ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err);
+        ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err, prm.wait_limit);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(bar(B_QE + sq));
         tc_commit(bar(B_OE + so));
         if (more) {
-          ok = mbar_wait(bar(B_OF + so1), po1, abort_flag, prm.err);
+          ok = mbar_wait(bar(B_OF + so1), po1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
           issue_dp(dOn);
@@ -319,10 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         sq = sq1; so = so1; pq = pq1; po = po1;
       }
       if (ok) tc_commit(bar(B_DONE));
-      if (!ok) {
-        tc_commit(bar(B_DRAIN));
-        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
-      }
+      // every MMA issued has completed before TMEM can be released
+      tc_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
     }
   }
   } else {
@@ -342,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *lsm = reinterpret_cast<const float *>(smem + kOffLse + sq * kBQ * 4) + 64 * w;
       const float *dsm = reinterpret_cast<const float *>(smem + kOffD + so * kBQ * 4) + 64 * w;
       // phase a/b: P^T over this warpgroup's first 32 columns of S^T
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err) &&
-                                       mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
+                                       mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
@@ -368,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_PS));
       // phase c: dS^T over this warpgroup's first 32 columns of dP^T
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + so), (t / kOStages) & 1, abort_flag, prm.err) &&
-                                       mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + so), (t / kOStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
+                                       mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       uint32_t dp[64];
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_DS));
     }
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (scaled)
-    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err));
+    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort_flag, prm.err, prm.wait_limit));
     tc_fence_after();
     __nv_bfloat16 *outp = (w == 0) ? prm.out0 : prm.out1;
     const float mul = (w == 0) ? 1.f : g.scale;
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int issued = 0;
         for (int j = 0; j < NT; ++j) {
           const int s = j % kStages, use = j / kStages;
-          if (use > 0 && !mbar_wait(bar(B_KE + s), (use - 1) & 1, abort_flag, prm.err)) break;
+          if (use > 0 && !mbar_wait(bar(B_KE + s), (use - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
           const uint32_t st = sb + kOffKV + s * 2 * kTile;
           const int row0 = (jt0 + j) * kBK;
           mbar_arrive_expect_tx(bar(B_KF + s), 2 * kTile);
@@ -511,13 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           issued = j + 1;
         }
-        if (*abort_flag)
-          for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-            mbar_wait(bar(B_KF + j % kStages), (j / kStages) & 1, nullptr, prm.err);
+        // every copy issued lands before the CTA can exit
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(bar(B_KF + j % kStages), (j / kStages) & 1, nullptr, prm.err);
       }
     } else if (warp == 1) {
       if (lane == 0 && NT > 0) {
-        bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err);
+        bool ok = mbar_wait(bar(B_QO), 0, abort_flag, prm.err, prm.wait_limit);
         tc_fence_after();
         // S = Q K_j^T (A = Q from TMEM), dP = dO V_j^T (A = dO from TMEM); B tiles K-major
         auto issue_s = [&](uint64_t dK) {
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         kIdescN128, kk > 0);
           tc_commit(bar(B_DPF));
         };
-        if (ok) ok = mbar_wait(bar(B_KF), 0, abort_flag, prm.err);
+        if (ok) ok = mbar_wait(bar(B_KF), 0, abort_flag, prm.err, prm.wait_limit);
         if (ok) {
           tc_fence_after();
           issue_s(sdesc_sw128(sb + kOffKV, 16, 1024));
@@ -553,14 +553,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dKm = sdesc_sw128(st, 16384, 1024);   // dQ: B = K tile, MN-major over d
           // both warpgroups hold S_j in registers, and the next K/V stage has
           // landed: the next tile's S (one wait point for both)
-          ok = more ? mbar_wait2(bar(B_SR), j & 1, bar(B_KF + s1), ps1, abort_flag, prm.err)
-                    : mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err);
+          ok = more ? mbar_wait2(bar(B_SR), j & 1, bar(B_KF + s1), ps1, abort_flag, prm.err, prm.wait_limit)
+                    : mbar_wait(bar(B_SR), j & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
           if (more) issue_s(dKn);
           // dQ += dS K_j: A = dS from TMEM (key columns [0,64) in the dP
           // columns [0,32), [64,128) in [64,96))
-          ok = mbar_wait(bar(B_DS), j & 1, abort_flag, prm.err);
+          ok = mbar_wait(bar(B_DS), j & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -575,10 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ps = ps1;
         }
         if (ok) tc_commit(bar(B_DQ));
-        if (!ok) {
-          tc_commit(bar(B_DRAIN));
-          mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
-        }
+        // every MMA issued has completed before TMEM can be released
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
       }
     }
   } else {
@@ -616,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < NT; ++j) {
       // phase a: P
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF), j & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF), j & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       uint32_t r[64];
@@ -635,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         r[c] = __float_as_uint(pv);
       }
       // phase b: dS over this warpgroup's first 32 columns of dP
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), j & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), j & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       uint32_t dp[64];
@@ -654,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // epilogue: warpgroup w writes dQ columns [64w, 64w + 64)
     const long long orow = valid ? g.q_out_row(qh, i) : 0;
-    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, abort_flag, prm.err));
+    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, abort_flag, prm.err, prm.wait_limit));
     tc_fence_after();
     if (ok && NT > 0) {
       uint32_t rr[32];
@@ -753,6 +752,7 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.mk = mk;
   prm.scale_log2 = g.scale * kLog2e;
   prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
   prm.out0 = static_cast<__nv_bfloat16 *>(dv);
   prm.out1 = static_cast<__nv_bfloat16 *>(dk);
   dim3 gkv(kvheads, (g.n + kv::kBN - 1) / kv::kBN);

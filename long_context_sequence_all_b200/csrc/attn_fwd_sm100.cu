@@ -63,6 +63,7 @@ struct FwdParams {
   MaskInfo mk;
   float scale_log2;  // softmax scale * log2(e)
   int *err;          // device error word
+  long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int idx = 0; idx < 2 * NT; ++idx) {
         const int slot = idx % kSlots, use = idx / kSlots;
-        if (use > 0 && !mbar_wait(bar(B_KVE + slot), (use - 1) & 1, abort_flag, prm.err)) break;
+        if (use > 0 && !mbar_wait(bar(B_KVE + slot), (use - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
         mbar_arrive_expect_tx(bar(B_KVF + slot), kTileBytes);
         const CUtensorMap *map = (idx & 1) ? &tmV : &tmK;
         const int row0 = (jt0 + idx / 2) * kBN;
@@ -140,17 +141,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sb + kOffKV + slot * kTileBytes + c * 16384, map, bar(B_KVF + slot), c * 64, row0, kvhead);
         issued = idx + 1;
       }
-      if (*abort_flag) {
-        // let the copies already in flight land before the CTA exits
-        for (int idx = (issued > kSlots ? issued - kSlots : 0); idx < issued; ++idx) {
-          mbar_wait(bar(B_KVF + idx % kSlots), (idx / kSlots) & 1, nullptr, prm.err);
-        }
-      }
+      // Every copy issued lands before the CTA can exit, also when a consumer
+      // gave up waiting for it (older ring entries were consumed, so landed,
+      // before their slot was refilled); on the normal path these return at once.
+      mbar_wait(bar(B_Q), 0, nullptr, prm.err);
+      for (int idx = (issued > kSlots ? issued - kSlots : 0); idx < issued; ++idx)
+        mbar_wait(bar(B_KVF + idx % kSlots), (idx / kSlots) & 1, nullptr, prm.err);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0 && NT > 0) {
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err);
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err, prm.wait_limit);
       tc_fence_after();
       // descriptors of the fixed operands; per-k-step offsets are constants
       const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
@@ -177,13 +178,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; ok && it < NT; ++it) {
         const uint64_t dk = sdesc_sw128(sb + kOffKV + slotK * kTileBytes, 16, 1024);
         const uint64_t dv = sdesc_sw128(sb + kOffKV + slotV * kTileBytes, 16384, 1024);   // V: MN-major
-        ok = (it > 0) ? mbar_wait2(bar(B_KVF + slotK), parK, bar(B_KVF + slotV), parV, abort_flag, prm.err)
-                      : mbar_wait(bar(B_KVF + slotK), parK, abort_flag, prm.err);
+        ok = (it > 0) ? mbar_wait2(bar(B_KVF + slotK), parK, bar(B_KVF + slotV), parV, abort_flag, prm.err, prm.wait_limit)
+                      : mbar_wait(bar(B_KVF + slotK), parK, abort_flag, prm.err, prm.wait_limit);
         if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < 2 && ok; ++t) {
           if (it > 0) {
-            ok = mbar_wait(bar(B_PF + t), (it - 1) & 1, abort_flag, prm.err);
+            ok = mbar_wait(bar(B_PF + t), (it - 1) & 1, abort_flag, prm.err, prm.wait_limit);
             if (!ok) break;
             tc_fence_after();
             issue_pv(t, dv, it == 1);
@@ -202,10 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         // the last tile's V (ring index 2 NT - 1: where slotV has rolled to)
         const uint64_t dv = sdesc_sw128(sb + kOffKV + slotV * kTileBytes, 16384, 1024);
-        ok = mbar_wait(bar(B_KVF + slotV), parV, abort_flag, prm.err);
+        ok = mbar_wait(bar(B_KVF + slotV), parV, abort_flag, prm.err, prm.wait_limit);
         tc_fence_after();
         for (int t = 0; t < 2 && ok; ++t) {
-          ok = mbar_wait(bar(B_PF + t), (NT - 1) & 1, abort_flag, prm.err);
+          ok = mbar_wait(bar(B_PF + t), (NT - 1) & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
           issue_pv(t, dv, NT == 1);
@@ -213,11 +214,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) tc_commit(bar(B_KVE + slotV));
       }
-      if (!ok) {
-        // drain: wait for every MMA issued so far before TMEM is released
-        tc_commit(bar(B_DRAIN));
-        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
-      }
+      // drain: every MMA issued has completed before TMEM can be released
+      tc_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
     }
   }
   } else {
@@ -236,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int it = 0; it < NT; ++it) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + wg), it & 1, abort_flag, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + wg), it & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       const int n0 = (jt0 + it) * kBN;
@@ -307,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PF + wg));
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + wg), 0, abort_flag, prm.err));
+    if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + wg), 0, abort_flag, prm.err, prm.wait_limit));
     tc_fence_after();
     // O goes to the head layout, or straight to the seq layout (the second
     // all-to-all in the epilogue); LSE stays in the head layout
@@ -396,6 +395,7 @@ uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.mk = mk;
   prm.scale_log2 = g.scale * kLog2e;
   prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
   dim3 grid(g.P * g.B * (g.hl / 2), (g.n + kBM - 1) / kBM);
   prof::Scope scope(prof::K_ATTN_FWD_SM100, stream);
   attn_fwd_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);

@@ -26,6 +26,11 @@ int *error_word();
 // Host-side launch bookkeeping (counts every kernel launched by the library).
 void note_launches(int n);
 
+// Cycles a pipeline wait of the tcgen05 kernels may last before it reports
+// ULY_ERR_TIMEOUT: the built-in limit, or a shorter one a test set with
+// ulysses_set_wait_limit (read by the launchers into the kernel parameters).
+long long wait_limit_cycles();
+
 inline uly_status last_launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA;

@@ -101,6 +101,7 @@ struct ProjParams {
   __nv_bfloat16 *q, *k, *v;  // QKV outputs, head layout
   __nv_bfloat16 *y;          // output projection result, seq layout
   int *err;
+  long long wait_limit;      // cycles a pipeline wait may last (wait_limit_cycles())
 };
 
 __device__ __forceinline__ void store_row_chunk(__nv_bfloat16 *dst, const float (&x)[32]) {
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < KT; ++kt, ++idx) {
           const int stage = (int)(idx % kStages);
           const long long use = idx / kStages;
-          if (use > 0 && !mbar_wait(bar(B_EMPTY + stage), (uint32_t)((use - 1) & 1), abort_flag, prm.err)) {
+          if (use > 0 && !mbar_wait(bar(B_EMPTY + stage), (uint32_t)((use - 1) & 1), abort_flag, prm.err, prm.wait_limit)) {
             ok = false;
             break;
           }
@@ -182,11 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sB, &tmB, bar(B_FULL + stage), kt * kBK, n0);
         }
       }
-      if (!ok) {
-        // let the copies already in flight land before the CTA exits
-        for (long long j = (idx > kStages ? idx - kStages : 0); j < idx; ++j)
-          mbar_wait(bar(B_FULL + (int)(j % kStages)), (uint32_t)((j / kStages) & 1), nullptr, prm.err);
-      }
+      // every copy issued lands before the CTA can exit, also when the MMA
+      // thread gave up waiting for it; on the normal path these return at once
+      for (long long j = (idx > kStages ? idx - kStages : 0); j < idx; ++j)
+        mbar_wait(bar(B_FULL + (int)(j % kStages)), (uint32_t)((j / kStages) & 1), nullptr, prm.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
         const int buf = it & 1;
         if (it >= 2) {
-          ok = mbar_wait(bar(B_ACCE + buf), (uint32_t)(((it >> 1) - 1) & 1), abort_flag, prm.err);
+          ok = mbar_wait(bar(B_ACCE + buf), (uint32_t)(((it >> 1) - 1) & 1), abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
         }
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int stage = (int)(idx % kStages);
           const uint32_t sA = sb + stage * kStageBytes, sB = sA + kABytes;
           const uint64_t da = sdesc_sw128(sA, 16, 1024), db = sdesc_sw128(sB, 16, 1024);
-          ok = mbar_wait(bar(B_FULL + stage), (uint32_t)((idx / kStages) & 1), abort_flag, prm.err);
+          ok = mbar_wait(bar(B_FULL + stage), (uint32_t)((idx / kStages) & 1), abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -217,11 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_commit(bar(B_ACCF + buf));
       }
-      if (!ok) {
-        // drain: wait for every MMA issued so far before TMEM is released
-        tc_commit(bar(B_DRAIN));
-        mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
-      }
+      // drain: every MMA issued has completed before TMEM can be released
+      tc_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, nullptr, prm.err);
     }
   } else {
     // ------------------------------------------------------------- epilogue
@@ -231,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const int buf = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ACCF + buf), (uint32_t)((it >> 1) & 1), abort_flag, prm.err)))
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ACCF + buf), (uint32_t)((it >> 1) & 1), abort_flag, prm.err, prm.wait_limit)))
         break;
       tc_fence_after();
       const int mt = tile / prm.n_tiles, nt = tile - mt * prm.n_tiles;
@@ -399,6 +397,7 @@ uly_status qkv_proj_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int3
   prm.k = static_cast<__nv_bfloat16 *>(k);
   prm.v = static_cast<__nv_bfloat16 *>(v);
   prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
   return launch_proj(ta, tb, prm, prof::K_QKV_PROJ, stream);
 }
 
@@ -419,6 +418,7 @@ uly_status o_proj_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int32_
   prm.hidden = hidden;
   prm.y = static_cast<__nv_bfloat16 *>(y);
   prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
   return launch_proj(ta, tb, prm, prof::K_O_PROJ, stream);
 }
 

@@ -75,17 +75,22 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // runs out (see kWaitLimitCycles / kPeerAbortCycles) or when *abort is already set;
 // then *abort is set so the CTA's other roles stop too.  abort == nullptr:
 // a drain wait that only honours the limits.  err: the device error word.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          int *err) {
+// limit: cycles before giving up.  Below kWaitLimitCycles (a limit a test set
+// with ulysses_set_wait_limit, passed in the kernel's parameters) the wait
+// polls without suspending and checks the clock every time, so a wait that is
+// not already complete runs out after about `limit` cycles.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *err,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_test_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const bool short_limit = limit < kWaitLimitCycles;
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 0) {
+    if (short_limit ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (short_limit || (it & 127u) == 0) {
       if (abort && *abort) return false;
       const long long dt = clock64() - t0;
       bool give_up = false;
-      if (dt > kWaitLimitCycles) {
+      if (dt > limit) {
         raise_error(err, ULY_ERR_TIMEOUT);
         if (err && atomicCAS(err + 1, 0, 1) == 0) {
           // first timeout of this device: where it happened
@@ -115,12 +120,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // both have completed (the common case in the MMA-issuing thread) their
 // latencies overlap.
 __device__ __forceinline__ bool mbar_wait2(uint32_t bar_a, uint32_t parity_a, uint32_t bar_b,
-                                           uint32_t parity_b, volatile int *abort, int *err) {
+                                           uint32_t parity_b, volatile int *abort, int *err,
+                                           long long limit = kWaitLimitCycles) {
   const bool a = mbar_test_wait(bar_a, parity_a);
   const bool b = mbar_test_wait(bar_b, parity_b);
   if (a && b) return true;
-  if (!a && !mbar_wait(bar_a, parity_a, abort, err)) return false;
-  return b || mbar_wait(bar_b, parity_b, abort, err);
+  if (!a && !mbar_wait(bar_a, parity_a, abort, err, limit)) return false;
+  return b || mbar_wait(bar_b, parity_b, abort, err, limit);
 }
 
 // ---------------------------------------------------------------------- TMA

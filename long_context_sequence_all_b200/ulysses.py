@@ -29,6 +29,7 @@ EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
            "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
            "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info", "ulysses_error_word",
+           "ulysses_set_wait_limit",
            "ulysses_status_string", "ulysses_profile_enable", "ulysses_profile_read",
            "ulysses_kernel_count", "ulysses_kernel_name",
            "ulysses_launch_count"]
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
             L.ulysses_error_word.argtypes = [ctypes.POINTER(vp)]
             L.ulysses_error_word.restype = ctypes.c_int
             L.ulysses_read_error_info.argtypes = [ctypes.POINTER(i32), i32]
+            L.ulysses_set_wait_limit.argtypes = [i64]
+            L.ulysses_set_wait_limit.restype = ctypes.c_int
             L.ulysses_status_string.argtypes = [ctypes.c_int]
             L.ulysses_status_string.restype = ctypes.c_char_p
             L.ulysses_launch_count.restype = ctypes.c_uint64
@@ -416,6 +419,12 @@ def ulysses_read_error_info() -> list:
     buf = (ctypes.c_int32 * 16)()
     _check(lib().ulysses_read_error_info(buf, 16), "ulysses_read_error_info")
     return list(buf)
+
+
+def ulysses_set_wait_limit(cycles: int = 0):
+    """Cycles a pipeline wait of the tcgen05 kernels may last before it reports
+    ULY_ERR_TIMEOUT (0: the built-in limit).  For tests of the timeout path."""
+    _check(lib().ulysses_set_wait_limit(int(cycles)), "ulysses_set_wait_limit")
 
 
 def ulysses_status_string(status: int) -> str:
