@@ -149,20 +149,16 @@ class Layer:
                                           workspace=self.lbws)
 
     def fwd_step(self):
-        """The forward half alone: seq->head(Q, K, V), attention forward writing O
-        in the seq layout."""
+        """The forward half alone: seq->head(Q, K, V) in one launch, attention
+        forward writing O in the seq layout."""
         U, P = self.U, self.P
-        U.ulysses_seq_to_head(self.q, P, out=self.qh)
-        U.ulysses_seq_to_head(self.k, P, out=self.kh)
-        U.ulysses_seq_to_head(self.v, P, out=self.vh)
+        U.ulysses_seq_to_head_batch([self.q, self.k, self.v], P, outs=[self.qh, self.kh, self.vh])
         U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.o, lse=self.lse,
                            out_seq_layout=True)
 
     def step(self):
         U, P = self.U, self.P
-        U.ulysses_seq_to_head(self.q, P, out=self.qh)
-        U.ulysses_seq_to_head(self.k, P, out=self.kh)
-        U.ulysses_seq_to_head(self.v, P, out=self.vh)
+        U.ulysses_seq_to_head_batch([self.q, self.k, self.v], P, outs=[self.qh, self.kh, self.vh])
         U.ulysses_attn_fwd(self.qh, self.kh, self.vh, mask=self.mask, cu_seqlens=self.cu, o=self.o, lse=self.lse,
                            out_seq_layout=True)
         U.ulysses_seq_to_head(self.do, P, out=self.doh)

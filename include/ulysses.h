@@ -109,6 +109,30 @@ uly_status ulysses_seq_to_head(int32_t batch, int32_t seq_len, int32_t world, in
                                int32_t head_dim, int32_t elem_bytes, const void *src,
                                void *dst, void *stream);
 
+/* One tensor of a batched all-to-all (the source and destination of one
+ * permutation and its number of heads). */
+typedef struct {
+  const void *src;
+  void *dst;
+  int32_t heads;
+} uly_permute_item;
+
+/*
+ * The first (seq -> head) or second (head -> seq) all-to-all of `count`
+ * tensors at once (1 <= count <= 4, e.g. Q, K and V), all with the same
+ * batch, seq_len, world, head_dim and elem_bytes and each with its own number
+ * of heads; `items` is a HOST array the call reads before it returns.  Every
+ * tensor follows the rules of ulysses_seq_to_head; no destination may overlap
+ * any source or destination of the call.  Bit-exact copies, one launch when
+ * the shapes allow (up to 256 heads per tensor, rows of at most 1 KB).
+ */
+uly_status ulysses_seq_to_head_batch(int32_t batch, int32_t seq_len, int32_t world, int32_t head_dim,
+                                     int32_t elem_bytes, int32_t count, const uly_permute_item *items,
+                                     void *stream);
+uly_status ulysses_head_to_seq_batch(int32_t batch, int32_t seq_len, int32_t world, int32_t head_dim,
+                                     int32_t elem_bytes, int32_t count, const uly_permute_item *items,
+                                     void *stream);
+
 /* Second all-to-all (step 5): head layout -> seq layout; exact inverse of
  * ulysses_seq_to_head, same arguments and rules. */
 uly_status ulysses_head_to_seq(int32_t batch, int32_t seq_len, int32_t world, int32_t heads,

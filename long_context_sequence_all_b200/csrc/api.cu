@@ -45,6 +45,8 @@ uly_status permute_validate(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t
                             const void *);
 uly_status permute_launch(bool, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *,
                           void *, cudaStream_t);
+uly_status permute_batch_launch(bool, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
+                                const uly_permute_item *, cudaStream_t);
 uly_status attn_f32_fwd_launch(const uly_attn_desc *, const HeadGeom &, const MaskInfo &,
                                const void *, const void *, const void *, void *, float *,
                                cudaStream_t);
@@ -178,6 +180,36 @@ uly_status ulysses_head_to_seq(int32_t batch, int32_t seq_len, int32_t world, in
   if (st != ULY_OK) return st;
   return permute_launch(false, batch, seq_len, world, heads, head_dim, eb, src, dst,
                         static_cast<cudaStream_t>(stream));
+}
+
+static uly_status permute_batch(bool to_head, int32_t batch, int32_t seq_len, int32_t world, int32_t head_dim,
+                                int32_t eb, int32_t count, const uly_permute_item *items, void *stream) {
+  if (!items) return ULY_ERR_NULL;
+  if (count < 1 || count > 4) return ULY_ERR_SHAPE;
+  size_t bytes[4];
+  for (int i = 0; i < count; ++i) {
+    uly_status st = permute_validate(batch, seq_len, world, items[i].heads, head_dim, eb, items[i].src,
+                                     items[i].dst);
+    if (st != ULY_OK) return st;
+    bytes[i] = (size_t)batch * seq_len * items[i].heads * head_dim * eb;
+  }
+  for (int i = 0; i < count; ++i)
+    for (int j = 0; j < count; ++j)
+      if (i != j && (overlap(items[i].dst, bytes[i], items[j].dst, bytes[j]) ||
+                     overlap(items[i].dst, bytes[i], items[j].src, bytes[j])))
+        return ULY_ERR_ALIAS;
+  return permute_batch_launch(to_head, batch, seq_len, world, head_dim, eb, count, items,
+                              static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_seq_to_head_batch(int32_t batch, int32_t seq_len, int32_t world, int32_t head_dim,
+                                     int32_t eb, int32_t count, const uly_permute_item *items, void *stream) {
+  return permute_batch(true, batch, seq_len, world, head_dim, eb, count, items, stream);
+}
+
+uly_status ulysses_head_to_seq_batch(int32_t batch, int32_t seq_len, int32_t world, int32_t head_dim,
+                                     int32_t eb, int32_t count, const uly_permute_item *items, void *stream) {
+  return permute_batch(false, batch, seq_len, world, head_dim, eb, count, items, stream);
 }
 
 uly_status ulysses_kv_seq_to_head_replicated(int32_t batch, int32_t seq_len, int32_t world,

@@ -33,6 +33,8 @@ enum Kernel {
   K_CHECK_CU,
   K_ATTN_BWD_SM100,
   K_ATTN_DQ_CONVERT,
+  K_SEQ_TO_HEAD_VEC,
+  K_HEAD_TO_SEQ_VEC,
   K_COUNT
 };
 

@@ -23,7 +23,8 @@ MASK_NONE, MASK_CAUSAL, MASK_DOC_CAUSAL = 0, 1, 2
 STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE",
           4: "ULY_ERR_ALIGN", 5: "ULY_ERR_ALIAS", 6: "ULY_ERR_UNSUPPORTED", 7: "ULY_ERR_CUDA",
           8: "ULY_ERR_LABEL", 9: "ULY_ERR_TIMEOUT", 10: "ULY_ERR_WORKSPACE"}
-EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head_replicated",
+EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_seq_to_head_batch", "ulysses_head_to_seq_batch",
+           "ulysses_kv_seq_to_head_replicated",
            "ulysses_kv_head_to_seq_reduce", "ulysses_shift_labels", "ulysses_rope_table",
            "ulysses_qkv_proj_rope", "ulysses_o_proj", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
@@ -50,6 +51,10 @@ class AttnDesc(ctypes.Structure):
                 ("deterministic", ctypes.c_int32)]
 
 
+class PermuteItem(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("heads", ctypes.c_int32)]
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -66,6 +71,9 @@ def lib() -> ctypes.CDLL:
             vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
             for name in ("ulysses_seq_to_head", "ulysses_head_to_seq"):
                 getattr(L, name).argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
+                getattr(L, name).restype = ctypes.c_int
+            for name in ("ulysses_seq_to_head_batch", "ulysses_head_to_seq_batch"):
+                getattr(L, name).argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(PermuteItem), vp]
                 getattr(L, name).restype = ctypes.c_int
             L.ulysses_kv_seq_to_head_replicated.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
             L.ulysses_kv_head_to_seq_reduce.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp]
@@ -169,6 +177,43 @@ def ulysses_head_to_seq(x: torch.Tensor, P: int, out: torch.Tensor | None = None
     _check(lib().ulysses_head_to_seq(B, n, P, heads, d, x.element_size(), _p(x), _p(out),
                                      _stream(stream)), "ulysses_head_to_seq")
     return out
+
+
+def _batch(to_head: bool, xs, P: int, outs=None, stream=None):
+    if not 1 <= len(xs) <= 4:
+        raise UlyssesError(2, "batched all-to-all: 1 to 4 tensors")
+    x0 = xs[0]
+    if to_head:
+        _, B, s, _, d = x0.shape
+        n = P * s
+        heads = [x.shape[3] for x in xs]
+        shape = lambda x: (P, B, x.shape[3] // P, n, d)
+    else:
+        _, B, _, n, d = x0.shape
+        heads = [x.shape[2] * P for x in xs]
+        shape = lambda x: (P, B, n // P, x.shape[2] * P, d)
+    for x in xs:
+        if x.dtype != x0.dtype or x.shape[0] != P or x.shape[1] != B or x.shape[-1] != d:
+            raise UlyssesError(2, f"batched all-to-all: shapes {[tuple(y.shape) for y in xs]} with P={P}")
+    if outs is None:
+        outs = [torch.empty(shape(x), dtype=x.dtype, device=x.device) for x in xs]
+    arr = (PermuteItem * len(xs))(*[PermuteItem(x.data_ptr(), o.data_ptr(), h) for x, o, h in zip(xs, outs, heads)])
+    fn = lib().ulysses_seq_to_head_batch if to_head else lib().ulysses_head_to_seq_batch
+    _check(fn(B, n, P, d, x0.element_size(), len(xs), arr, _stream(stream)),
+           "ulysses_seq_to_head_batch" if to_head else "ulysses_head_to_seq_batch")
+    return outs
+
+
+def ulysses_seq_to_head_batch(xs, P: int, outs=None, stream=None):
+    """The first all-to-all of up to four tensors in one call (e.g. Q, K, V):
+    each [P][B][n/P][heads_i][d] -> [P][B][heads_i/P][n][d]."""
+    return _batch(True, xs, P, outs, stream)
+
+
+def ulysses_head_to_seq_batch(xs, P: int, outs=None, stream=None):
+    """The second all-to-all of up to four tensors in one call:
+    each [P][B][heads_i/P][n][d] -> [P][B][n/P][heads_i][d]."""
+    return _batch(False, xs, P, outs, stream)
 
 
 def ulysses_kv_seq_to_head_replicated(x: torch.Tensor, P: int, out: torch.Tensor | None = None,
