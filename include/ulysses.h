@@ -250,6 +250,44 @@ uly_status ulysses_o_proj(int32_t batch, int32_t seq_len, int32_t world, int32_t
                           int32_t n_q_heads, int32_t head_dim, const void *o, const void *w_o,
                           void *y, void *stream);
 
+/* Bytes of device workspace ulysses_qkv_proj_rope_bwd needs: the projection's
+ * output gradient dY, bf16 [B*n][(H + 2G) * head_dim]. */
+uly_status ulysses_qkv_proj_rope_bwd_workspace_size(int32_t batch, int32_t seq_len, int32_t n_q_heads,
+                                                   int32_t n_kv_heads, int32_t head_dim, size_t *bytes);
+
+/*
+ * Backward of steps 2-3 (the adjoint of ulysses_qkv_proj_rope):
+ *   dY(t) = [R(-pos) dQ(t) | R(-pos) dK(t) | dV(t)]   (the gradients back
+ *           through the folded all-to-all and through the rotation, whose
+ *           transpose is the rotation by -pos), written to `workspace`;
+ *   dX = dY W_qkv          (bf16, seq layout [P][B][n/P][hidden]);
+ *   dW = sum over all tokens of dY^T X   (fp32 [(H+2G)*head_dim][hidden]).
+ * dq [P][B][H/P][n][d], dk, dv [P][B][G/P][n][d] (bf16 head layout); x, w_qkv,
+ * rope_table, max_pos, positions as for the forward.  Needs G % P == 0 (with
+ * fewer KV heads than ranks, sum the copies' gradients first), head_dim ==
+ * 128, H + 2G even, hidden % 256 == 0.  Tensor-core GEMMs with fp32
+ * accumulation; the pre-pass is HBM-bound.  Outputs must not overlap inputs.
+ */
+uly_status ulysses_qkv_proj_rope_bwd(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, const void *x,
+                                     const void *w_qkv, const float *rope_table, int32_t max_pos,
+                                     const int32_t *positions, const void *dq, const void *dk, const void *dv,
+                                     void *dx, float *dw, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Backward of steps 5-6 (the adjoint of ulysses_o_proj):
+ *   dO = dY W_o   written straight into the head layout [P][B][H/P][n][d]
+ *                 (bf16; the first all-to-all in the GEMM's epilogue);
+ *   dW_o = sum over all tokens of dY^T O   (fp32 [hidden][H * head_dim]).
+ * o_seq: the attention output in the seq layout [P][B][n/P][H][d] (as
+ * ulysses_attn_fwd writes it with out_seq_layout = 1); w_o [hidden][H*d];
+ * dy: the layer output's gradient, seq layout [P][B][n/P][hidden] (bf16).
+ * Needs head_dim == 128, H even, hidden % 256 == 0.
+ */
+uly_status ulysses_o_proj_bwd(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden, int32_t n_q_heads,
+                              int32_t head_dim, const void *o_seq, const void *w_o, const void *dy, void *do_head,
+                              float *dw_o, void *stream);
+
 /*
  * Local attention (step 4) of every logical rank, head layout in and out:
  * q, o [P][B][H/P][n][d]; k, v [P][B][G/P][n][d]; lse [P][B][H/P][n] (fp32).

@@ -75,6 +75,11 @@ uly_status qkv_proj_launch(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
                            const float *, int32_t, const int32_t *, void *, void *, void *, cudaStream_t);
 uly_status o_proj_launch(int32_t, int32_t, int32_t, int32_t, int32_t, const void *, const void *, void *,
                          cudaStream_t);
+uly_status qkv_proj_bwd_launch(int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, const void *, const void *,
+                               const float *, int32_t, const int32_t *, const void *, const void *, const void *,
+                               void *, float *, void *, cudaStream_t);
+uly_status o_proj_bwd_launch(int32_t, int32_t, int32_t, int32_t, int32_t, const void *, const void *, const void *,
+                             void *, float *, cudaStream_t);
 size_t loss_workspace_bytes(int P, long long per_shard);
 size_t loss_bwd_workspace_bytes(int P, long long per_shard);
 uly_status loss_bwd_launch(int32_t, int64_t, int32_t, int32_t, const void *, const int32_t *, int32_t,
@@ -310,6 +315,73 @@ uly_status ulysses_o_proj(int32_t batch, int32_t seq_len, int32_t world, int32_t
   if (overlap(y, yb, o, ob) || overlap(y, yb, w_o, wb)) return ULY_ERR_ALIAS;
   return o_proj_launch(batch, seq_len, world, hidden, n_q_heads, o, w_o, y,
                        static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_qkv_proj_rope_bwd_workspace_size(int32_t batch, int32_t seq_len, int32_t n_q_heads,
+                                                   int32_t n_kv_heads, int32_t head_dim, size_t *bytes) {
+  if (!bytes) return ULY_ERR_NULL;
+  if (batch <= 0 || seq_len <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0) return ULY_ERR_SHAPE;
+  *bytes = align256((size_t)batch * seq_len * (n_q_heads + 2 * n_kv_heads) * head_dim * 2);
+  return ULY_OK;
+}
+
+uly_status ulysses_qkv_proj_rope_bwd(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, const void *x,
+                                     const void *w_qkv, const float *rope_table, int32_t max_pos,
+                                     const int32_t *positions, const void *dq, const void *dk, const void *dv,
+                                     void *dx, float *dw, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!x || !w_qkv || !rope_table || !dq || !dk || !dv || !dx || !dw) return ULY_ERR_NULL;
+  if (batch <= 0 || seq_len <= 0 || world <= 0 || hidden <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 ||
+      head_dim <= 0 || max_pos <= 0)
+    return ULY_ERR_SHAPE;
+  if (seq_len % world || n_q_heads % world || n_q_heads % n_kv_heads) return ULY_ERR_SHAPE;
+  if (n_kv_heads % world) return ULY_ERR_UNSUPPORTED;  // fewer KV heads than ranks: sum the copies first
+  if (head_dim != 128 || (n_q_heads + 2 * n_kv_heads) % 2 || hidden % 256) return ULY_ERR_UNSUPPORTED;
+  if (!positions && max_pos < seq_len) return ULY_ERR_SHAPE;
+  const long long M = (long long)batch * seq_len;
+  const long long N = (long long)(n_q_heads + 2 * n_kv_heads) * head_dim;
+  if (M > 0x7fffffffLL || (M + 127) / 128 * (hidden / 256) > 0x7fffffffLL) return ULY_ERR_SHAPE;
+  size_t need = 0;
+  ulysses_qkv_proj_rope_bwd_workspace_size(batch, seq_len, n_q_heads, n_kv_heads, head_dim, &need);
+  if (!workspace || workspace_bytes < need) return ULY_ERR_WORKSPACE;
+  if (!all_aligned({x, w_qkv, rope_table, dq, dk, dv, dx, dw, workspace})) return ULY_ERR_ALIGN;
+  const size_t xb = (size_t)M * hidden * 2, wb = (size_t)N * hidden * 2, qb = (size_t)M * n_q_heads * head_dim * 2,
+               kb = (size_t)M * n_kv_heads * head_dim * 2, rb = (size_t)max_pos * head_dim * 4,
+               pb = positions ? (size_t)M * 4 : 0;
+  const void *ins[7] = {x, w_qkv, rope_table, positions, dq, dk, dv};
+  const size_t inb[7] = {xb, wb, rb, pb, qb, kb, kb};
+  void *outs[3] = {dx, dw, workspace};
+  const size_t outb[3] = {xb, (size_t)N * hidden * 4, need};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 7; ++b)
+      if (ins[b] && overlap(outs[a], outb[a], ins[b], inb[b])) return ULY_ERR_ALIAS;
+    for (int b = a + 1; b < 3; ++b)
+      if (overlap(outs[a], outb[a], outs[b], outb[b])) return ULY_ERR_ALIAS;
+  }
+  return qkv_proj_bwd_launch(batch, seq_len, world, hidden, n_q_heads, n_kv_heads, x, w_qkv, rope_table, max_pos,
+                             positions, dq, dk, dv, dx, dw, workspace, static_cast<cudaStream_t>(stream));
+}
+
+uly_status ulysses_o_proj_bwd(int32_t batch, int32_t seq_len, int32_t world, int32_t hidden, int32_t n_q_heads,
+                              int32_t head_dim, const void *o_seq, const void *w_o, const void *dy, void *do_head,
+                              float *dw_o, void *stream) {
+  if (!o_seq || !w_o || !dy || !do_head || !dw_o) return ULY_ERR_NULL;
+  if (batch <= 0 || seq_len <= 0 || world <= 0 || hidden <= 0 || n_q_heads <= 0 || head_dim <= 0)
+    return ULY_ERR_SHAPE;
+  if (seq_len % world || n_q_heads % world) return ULY_ERR_SHAPE;
+  if (head_dim != 128 || hidden % 256 || n_q_heads % 2) return ULY_ERR_UNSUPPORTED;
+  const long long M = (long long)batch * seq_len;
+  if (M > 0x7fffffffLL) return ULY_ERR_SHAPE;
+  if (!all_aligned({o_seq, w_o, dy, do_head, dw_o})) return ULY_ERR_ALIGN;
+  const size_t ob = (size_t)M * n_q_heads * head_dim * 2, wb = (size_t)hidden * n_q_heads * head_dim * 2,
+               yb = (size_t)M * hidden * 2, dwb = (size_t)hidden * n_q_heads * head_dim * 4;
+  const void *ins[3] = {o_seq, w_o, dy};
+  const size_t inb[3] = {ob, wb, yb};
+  for (int b = 0; b < 3; ++b)
+    if (overlap(do_head, ob, ins[b], inb[b]) || overlap(dw_o, dwb, ins[b], inb[b])) return ULY_ERR_ALIAS;
+  if (overlap(do_head, ob, dw_o, dwb)) return ULY_ERR_ALIAS;
+  return o_proj_bwd_launch(batch, seq_len, world, hidden, n_q_heads, o_seq, w_o, dy, do_head, dw_o,
+                           static_cast<cudaStream_t>(stream));
 }
 
 uly_status ulysses_attn_fwd(const uly_attn_desc *d, const void *q, const void *k, const void *v,

@@ -43,7 +43,8 @@ const char *name(int k) {
       "attn_dq_sm100", "attn_bwd_stats", "loss_fwd_bwd", "kv_seq_to_head_rep",
       "kv_head_to_seq_sum", "shift_labels", "rope_table", "qkv_proj_sm100",
       "o_proj_sm100", "check_cu_seqlens", "attn_bwd_sm100", "attn_dq_convert",
-      "seq_to_head_vec", "head_to_seq_vec"};
+      "seq_to_head_vec", "head_to_seq_vec", "qkv_dy", "qkv_proj_dx_sm100", "qkv_proj_dw_sm100",
+      "o_proj_do_sm100", "o_proj_dw_sm100"};
   return (k >= 0 && k < K_COUNT) ? names[k] : "unknown";
 }
 

@@ -35,6 +35,11 @@ enum Kernel {
   K_ATTN_DQ_CONVERT,
   K_SEQ_TO_HEAD_VEC,
   K_HEAD_TO_SEQ_VEC,
+  K_QKV_DY,
+  K_QKV_DX,
+  K_QKV_DW,
+  K_O_PROJ_DO,
+  K_O_PROJ_DWO,
   K_COUNT
 };
 

@@ -83,8 +83,21 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
 constexpr uint32_t kOffBar = kStages * kStageBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // barriers + alignment slack
 constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kBM, kBN, false, false);
+constexpr uint32_t kIdescKM = sm100::idesc_bf16_f32(kBM, kBN, false, true);   // B MN-major
+constexpr uint32_t kIdescMK = sm100::idesc_bf16_f32(kBM, kBN, true, false);   // A MN-major
+constexpr uint32_t kIdescMM = sm100::idesc_bf16_f32(kBM, kBN, true, true);
 
-enum Mode { MODE_QKV = 0, MODE_OPROJ = 1 };
+// QKV / OPROJ: the forward projections.  The backward ones (the adjoints of
+// steps 2-3 and 5-6) reuse the same pipeline with other operand layouts and
+// epilogues:
+//   DX:    dX[M][hidden]  = dY[M][Nqkv] W[Nqkv][hidden]      A K-major, B MN-major, bf16 rows
+//   DW:    dW[Nqkv][hidden] = dY^T X  (sum over all tokens)   A, B MN-major, fp32 rows
+//   DO:    dO = dY_o[M][hidden] W_o[hidden][H*d] -> head layout  A K-major, B MN-major
+//   DWO:   dW_o[hidden][H*d] = dY_o^T O_seq                   A, B MN-major, fp32 rows
+// An MN-major operand (its M or N index contiguous in memory, K along rows)
+// arrives as 64-row TMA boxes of 64 contiguous elements, one per 64 columns
+// of the tile: the same 16 KB (A) and 32 KB (B) per stage.
+enum Mode { MODE_QKV = 0, MODE_OPROJ = 1, MODE_DX = 2, MODE_DW = 3, MODE_DO = 4, MODE_DWO = 5 };
 
 struct ProjParams {
   int mode;
@@ -100,6 +113,11 @@ struct ProjParams {
   const int32_t *positions;  // nullable [B][n]
   __nv_bfloat16 *q, *k, *v;  // QKV outputs, head layout
   __nv_bfloat16 *y;          // output projection result, seq layout
+  int a_mn, b_mn;            // operand A / B is MN-major (2-D map with 64 x 64 boxes)
+  long long ldc;             // DX / DW / DWO: row stride of C in elements
+  __nv_bfloat16 *c16;        // DX: bf16 C
+  float *c32;                // DW / DWO: fp32 C
+  long long M_rows;          // DX / DW / DWO: rows of C (rows past it are not stored)
   int *err;
   long long wait_limit;      // cycles a pipeline wait may last (wait_limit_cycles())
 };
@@ -132,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = prm.m_tiles * prm.n_tiles;
-  const int KT = prm.K / kBK;
+  const int KT = (prm.K + kBK - 1) / kBK;   // a ragged last k-step reads zeros past K
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_ACCE || i == B_ACCE + 1) ? 128 : 1);
@@ -172,15 +190,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t sA = sb + stage * kStageBytes, sB = sA + kABytes;
           mbar_arrive_expect_tx(bar(B_FULL + stage), kStageBytes);
-          if (prm.mode == MODE_QKV) {
-            tma_load_2d(sA, &tmA, bar(B_FULL + stage), kt * kBK, mt * kBM);
-          } else {
+          if (prm.mode == MODE_OPROJ) {
             // k-step kt covers features [64 (kt % 2), +64) of query head kt / 2,
             // held by rank kt / 2 / hl as its local head (kt / 2) % hl
             const int qh = kt >> 1, r2 = qh / prm.hl, hh = qh - r2 * prm.hl;
             tma_load_3d(sA, &tmA, bar(B_FULL + stage), (kt & 1) * kBK, t0, (r2 * prm.B + b) * prm.hl + hh);
+          } else if (prm.a_mn) {
+            for (int c = 0; c < kBM / 64; ++c)
+              tma_load_2d(sA + c * 8192, &tmA, bar(B_FULL + stage), mt * kBM + 64 * c, kt * kBK);
+          } else {
+            tma_load_2d(sA, &tmA, bar(B_FULL + stage), kt * kBK, mt * kBM);
           }
-          tma_load_2d(sB, &tmB, bar(B_FULL + stage), kt * kBK, n0);
+          if (prm.b_mn) {
+            for (int c = 0; c < kBN / 64; ++c)
+              tma_load_2d(sB + c * 8192, &tmB, bar(B_FULL + stage), n0 + 64 * c, kt * kBK);
+          } else {
+            tma_load_2d(sB, &tmB, bar(B_FULL + stage), kt * kBK, n0);
+          }
         }
       }
       // every copy issued lands before the CTA can exit, also when the MMA
@@ -205,13 +231,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < KT; ++kt, ++idx) {
           const int stage = (int)(idx % kStages);
           const uint32_t sA = sb + stage * kStageBytes, sB = sA + kABytes;
-          const uint64_t da = sdesc_sw128(sA, 16, 1024), db = sdesc_sw128(sB, 16, 1024);
+          // K-major: 16 K-elements are 32 bytes along a row; MN-major: 16 K-rows
+          // are 2048 bytes, the 64-element MN chunks 8 KB apart (LBO)
+          const uint64_t da = prm.a_mn ? sdesc_sw128(sA, 8192, 1024) : sdesc_sw128(sA, 16, 1024);
+          const uint64_t db = prm.b_mn ? sdesc_sw128(sB, 8192, 1024) : sdesc_sw128(sB, 16, 1024);
+          const uint32_t astep = prm.a_mn ? 2048 : 32, bstep = prm.b_mn ? 2048 : 32;
+          const uint32_t idesc = prm.a_mn ? (prm.b_mn ? kIdescMM : kIdescMK) : (prm.b_mn ? kIdescKM : kIdesc);
           ok = mbar_wait(bar(B_FULL + stage), (uint32_t)((idx / kStages) & 1), abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ss(acc, sdesc_add(da, kk * 32), sdesc_add(db, kk * 32), kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ss(acc, sdesc_add(da, kk * astep), sdesc_add(db, kk * bstep), idesc,
+                        (kt > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(B_EMPTY + stage));
         }
         if (!ok) break;
@@ -234,7 +266,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int mt = tile / prm.n_tiles, nt = tile - mt * prm.n_tiles;
       const uint32_t acc = tmem + lane_off + buf * kBN;
-      if (prm.mode == MODE_QKV) {
+      if (prm.mode == MODE_DX || prm.mode == MODE_DW || prm.mode == MODE_DWO) {
+        // plain row-major C: bf16 (dX) or fp32 (the weight gradients)
+        const long long m = (long long)mt * kBM + row;
+        const bool valid = m < prm.M_rows;
+        const long long c0 = m * prm.ldc + (long long)nt * kBN;
+#pragma unroll 1
+        for (int c = 0; c < kBN; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(acc + c, a);
+          if (valid) {
+            if (prm.mode == MODE_DX) {
+              float x[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(a[e]);
+              store_row_chunk(prm.c16 + c0 + c, x);
+            } else {
+              float4 *d4 = reinterpret_cast<float4 *>(prm.c32 + c0 + c);
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                d4[u] = make_float4(__uint_as_float(a[4 * u]), __uint_as_float(a[4 * u + 1]),
+                                    __uint_as_float(a[4 * u + 2]), __uint_as_float(a[4 * u + 3]));
+            }
+          }
+        }
+      } else if (prm.mode == MODE_QKV || prm.mode == MODE_DO) {
         const long long m = (long long)mt * kBM + row;
         const bool valid = m < prm.M;
         int b = 0, t = 0, pos = 0;
@@ -245,10 +301,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           b = (int)(rem / prm.s);
           const int tt = (int)(rem - (long long)b * prm.s);
           t = r * prm.s + tt;
-          pos = prm.positions ? __ldg(prm.positions + (long long)b * prm.n + t) : t;
-          if (pos < 0 || pos >= prm.max_pos) {
-            raise_error(prm.err, ULY_ERR_SHAPE);
-            pos = 0;
+          if (prm.mode == MODE_QKV) {
+            pos = prm.positions ? __ldg(prm.positions + (long long)b * prm.n + t) : t;
+            if (pos < 0 || pos >= prm.max_pos) {
+              raise_error(prm.err, ULY_ERR_SHAPE);
+              pos = 0;
+            }
           }
         }
 #pragma unroll 1
@@ -256,10 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j = nt * 2 + hs;         // output head: H query, G key, G value heads
           __nv_bfloat16 *base;
           int heads_local, jj;
+          // QKV: H query, G key, G value heads (Q and K rotated); DO: the H
+          // query heads of dO, not rotated
           if (j < prm.H) { base = prm.q; heads_local = prm.hl; jj = j; }
           else if (j < prm.H + prm.G) { base = prm.k; heads_local = prm.gl; jj = j - prm.H; }
           else { base = prm.v; heads_local = prm.gl; jj = j - prm.H - prm.G; }
-          const bool rot = j < prm.H + prm.G;
+          const bool rot = prm.mode == MODE_QKV && j < prm.H + prm.G;
           const int r2 = jj / heads_local, hh = jj - r2 * heads_local;
           __nv_bfloat16 *dst = base + ((((long long)r2 * prm.B + b) * heads_local + hh) * prm.n + t) * kHD;
 #pragma unroll 1
@@ -338,6 +398,63 @@ __global__ void rope_table_kernel(int max_pos, int half, double base, float *tab
   }
 }
 
+// dY of the QKV projection's backward, seq layout [M][(H + 2G) * 128] with
+// M = P*B*s tokens (m = (r*B + b)*s + tt, position t = r*s + tt): output head
+// j's gradient row comes from the head layout (the inverse of the folded
+// all-to-all) and, for query and key heads, is rotated back by -pos (the
+// transpose of the rotation: d1 = g1 cos + g2 sin, d2 = g2 cos - g1 sin for
+// the pair (e, e + 64)).  16 threads per row, 4 pairs each; HBM-bound.
+__global__ void __launch_bounds__(256) qkv_dy_kernel(const __nv_bfloat16 *__restrict__ dq,
+                                                     const __nv_bfloat16 *__restrict__ dk,
+                                                     const __nv_bfloat16 *__restrict__ dv,
+                                                     const float4 *__restrict__ rope, int max_pos,
+                                                     const int32_t *__restrict__ positions,
+                                                     __nv_bfloat16 *__restrict__ dy, int B, int n, int s, int H,
+                                                     int G, int hl, int gl, long long rows, int *err) {
+  const int l = threadIdx.x & 15;
+  const int J = H + 2 * G;
+  for (long long R = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4; R < rows;
+       R += ((long long)gridDim.x * blockDim.x) >> 4) {
+    const long long m = R / J;
+    const int j = (int)(R - m * J);
+    const long long bs = (long long)B * s;
+    const int r = (int)(m / bs);
+    const long long rem = m - (long long)r * bs;
+    const int b = (int)(rem / s), tt = (int)(rem - (long long)b * s);
+    const int t = r * s + tt;
+    const __nv_bfloat16 *base;
+    int heads_local, jj;
+    if (j < H) { base = dq; heads_local = hl; jj = j; }
+    else if (j < H + G) { base = dk; heads_local = gl; jj = j - H; }
+    else { base = dv; heads_local = gl; jj = j - H - G; }
+    const int r2 = jj / heads_local, hh = jj - r2 * heads_local;
+    const __nv_bfloat16 *src = base + ((((long long)r2 * B + b) * heads_local + hh) * n + t) * kHD;
+    const uint2 a = __ldg(reinterpret_cast<const uint2 *>(src) + l);        // elements 4l .. 4l+3
+    const uint2 c = __ldg(reinterpret_cast<const uint2 *>(src + 64) + l);   // elements 64+4l ..
+    uint2 o1 = a, o2 = c;
+    if (j < H + G) {
+      int pos = positions ? __ldg(positions + (long long)b * n + t) : t;
+      if (pos < 0 || pos >= max_pos) {
+        if (l == 0) raise_error(err, ULY_ERR_SHAPE);
+        pos = 0;
+      }
+      const float4 w0 = __ldg(rope + (long long)pos * (kHD / 4) + 2 * l);       // pairs 4l, 4l+1
+      const float4 w1 = __ldg(rope + (long long)pos * (kHD / 4) + 2 * l + 1);   // pairs 4l+2, 4l+3
+      const float2 g1a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a.x));
+      const float2 g1b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a.y));
+      const float2 g2a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&c.x));
+      const float2 g2b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&c.y));
+      o1.x = pack_bf16x2(g1a.x * w0.x + g2a.x * w0.y, g1a.y * w0.z + g2a.y * w0.w);
+      o2.x = pack_bf16x2(g2a.x * w0.x - g1a.x * w0.y, g2a.y * w0.z - g1a.y * w0.w);
+      o1.y = pack_bf16x2(g1b.x * w1.x + g2b.x * w1.y, g1b.y * w1.z + g2b.y * w1.w);
+      o2.y = pack_bf16x2(g2b.x * w1.x - g1b.x * w1.y, g2b.y * w1.z - g1b.y * w1.w);
+    }
+    __nv_bfloat16 *out = dy + R * kHD;
+    reinterpret_cast<uint2 *>(out)[l] = o1;
+    reinterpret_cast<uint2 *>(out + 64)[l] = o2;
+  }
+}
+
 uly_status launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const ProjParams &prm, int kernel_id,
                        cudaStream_t stream) {
   // the shared-memory opt-in is a per-device attribute: set it once on every
@@ -399,6 +516,99 @@ uly_status qkv_proj_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int3
   prm.err = error_word();
   prm.wait_limit = wait_limit_cycles();
   return launch_proj(ta, tb, prm, prof::K_QKV_PROJ, stream);
+}
+
+// Backward of the QKV projection: dY pre-pass into `dy` (workspace), then
+// dX = dY W and dW = dY^T X on the tensor cores.
+uly_status qkv_proj_bwd_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int32_t H, int32_t G,
+                               const void *x, const void *w, const float *rope, int32_t max_pos,
+                               const int32_t *positions, const void *dq, const void *dk, const void *dv, void *dx,
+                               float *dw, void *dy, cudaStream_t stream) {
+  const long long M = (long long)B * n;
+  const long long N = (long long)(H + 2 * G) * kHD;
+  const long long rows = M * (H + 2 * G);
+  {
+    long long blocks = (rows * 16 + 255) / 256;
+    if (blocks > 148LL * 16) blocks = 148LL * 16;
+    prof::Scope scope(prof::K_QKV_DY, stream);
+    qkv_dy_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(dq), static_cast<const __nv_bfloat16 *>(dk),
+        static_cast<const __nv_bfloat16 *>(dv), reinterpret_cast<const float4 *>(rope), max_pos, positions,
+        static_cast<__nv_bfloat16 *>(dy), B, n, n / P, H, G, H / P, G / P, rows, error_word());
+    note_launches(1);
+    if (last_launch_status() != ULY_OK) return ULY_ERR_CUDA;
+  }
+  CUtensorMap ta, tb;
+  ProjParams prm = {};
+  prm.B = B; prm.n = n; prm.s = n / P; prm.P = P;
+  prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
+  // dX[M][hidden] = dY[M][N] W[N][hidden]
+  if (!make_tmap_rows_bf16(&ta, dy, N, M, kBK, kBM) || !make_tmap_rows_bf16(&tb, w, hidden, N, 64, 64))
+    return ULY_ERR_CUDA;
+  prm.mode = MODE_DX;
+  prm.K = (int)N;
+  prm.m_tiles = (int)((M + kBM - 1) / kBM);
+  prm.n_tiles = hidden / kBN;
+  prm.a_mn = 0;
+  prm.b_mn = 1;
+  prm.ldc = hidden;
+  prm.M_rows = M;
+  prm.c16 = static_cast<__nv_bfloat16 *>(dx);
+  uly_status st = launch_proj(ta, tb, prm, prof::K_QKV_DX, stream);
+  if (st != ULY_OK) return st;
+  // dW[N][hidden] = dY^T X, summed over every token
+  if (!make_tmap_rows_bf16(&ta, dy, N, M, 64, 64) || !make_tmap_rows_bf16(&tb, x, hidden, M, 64, 64))
+    return ULY_ERR_CUDA;
+  prm.mode = MODE_DW;
+  prm.K = (int)M;
+  prm.m_tiles = (int)(N / kBM);
+  prm.n_tiles = hidden / kBN;
+  prm.a_mn = 1;
+  prm.b_mn = 1;
+  prm.ldc = hidden;
+  prm.M_rows = N;
+  prm.c16 = nullptr;
+  prm.c32 = dw;
+  return launch_proj(ta, tb, prm, prof::K_QKV_DW, stream);
+}
+
+// Backward of the output projection: dO = dY W_o stored in the head layout
+// (the first all-to-all in the epilogue), dW_o = dY^T O with O in the seq layout.
+uly_status o_proj_bwd_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int32_t H, const void *o_seq,
+                             const void *w_o, const void *dy, void *do_head, float *dw_o, cudaStream_t stream) {
+  const long long M = (long long)B * n;
+  const long long HD = (long long)H * kHD;
+  CUtensorMap ta, tb;
+  ProjParams prm = {};
+  prm.B = B; prm.n = n; prm.s = n / P; prm.P = P;
+  prm.H = H; prm.G = 0; prm.hl = H / P; prm.gl = 1;
+  prm.M = M;
+  prm.err = error_word();
+  prm.wait_limit = wait_limit_cycles();
+  if (!make_tmap_rows_bf16(&ta, dy, hidden, M, kBK, kBM) || !make_tmap_rows_bf16(&tb, w_o, HD, hidden, 64, 64))
+    return ULY_ERR_CUDA;
+  prm.mode = MODE_DO;
+  prm.K = hidden;
+  prm.m_tiles = (int)((M + kBM - 1) / kBM);
+  prm.n_tiles = (int)(HD / kBN);
+  prm.a_mn = 0;
+  prm.b_mn = 1;
+  prm.q = static_cast<__nv_bfloat16 *>(do_head);
+  uly_status st = launch_proj(ta, tb, prm, prof::K_O_PROJ_DO, stream);
+  if (st != ULY_OK) return st;
+  if (!make_tmap_rows_bf16(&ta, dy, hidden, M, 64, 64) || !make_tmap_rows_bf16(&tb, o_seq, HD, M, 64, 64))
+    return ULY_ERR_CUDA;
+  prm.mode = MODE_DWO;
+  prm.K = (int)M;
+  prm.m_tiles = hidden / kBM;
+  prm.n_tiles = (int)(HD / kBN);
+  prm.a_mn = 1;
+  prm.b_mn = 1;
+  prm.ldc = HD;
+  prm.M_rows = hidden;
+  prm.c32 = dw_o;
+  return launch_proj(ta, tb, prm, prof::K_O_PROJ_DWO, stream);
 }
 
 uly_status o_proj_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, int32_t H, const void *o,

@@ -26,7 +26,8 @@ STATUS = {0: "ULY_OK", 1: "ULY_ERR_NULL", 2: "ULY_ERR_SHAPE", 3: "ULY_ERR_DTYPE"
 EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_seq_to_head_batch", "ulysses_head_to_seq_batch",
            "ulysses_kv_seq_to_head_replicated",
            "ulysses_kv_head_to_seq_reduce", "ulysses_shift_labels", "ulysses_rope_table",
-           "ulysses_qkv_proj_rope", "ulysses_o_proj", "ulysses_attn_fwd",
+           "ulysses_qkv_proj_rope", "ulysses_o_proj", "ulysses_qkv_proj_rope_bwd_workspace_size",
+           "ulysses_qkv_proj_rope_bwd", "ulysses_o_proj_bwd", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
            "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
            "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info", "ulysses_error_word",
@@ -82,6 +83,13 @@ def lib() -> ctypes.CDLL:
             L.ulysses_qkv_proj_rope.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32, vp,
                                                 vp, vp, vp, vp]
             L.ulysses_o_proj.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+            L.ulysses_qkv_proj_rope_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(sz)]
+            L.ulysses_qkv_proj_rope_bwd.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, vp,
+                                                    vp, vp, vp, vp, sz, vp]
+            L.ulysses_o_proj_bwd.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+            for name in ("ulysses_qkv_proj_rope_bwd_workspace_size", "ulysses_qkv_proj_rope_bwd",
+                         "ulysses_o_proj_bwd"):
+                getattr(L, name).restype = ctypes.c_int
             for name in ("ulysses_kv_seq_to_head_replicated", "ulysses_kv_head_to_seq_reduce",
                          "ulysses_shift_labels", "ulysses_rope_table", "ulysses_qkv_proj_rope",
                          "ulysses_o_proj"):
@@ -310,6 +318,48 @@ def ulysses_o_proj(o: torch.Tensor, w_o: torch.Tensor, P: int, y=None, stream=No
     _check(lib().ulysses_o_proj(B, n, P, hidden, hl * P, d, _p(o), _p(w_o), _p(y), _stream(stream)),
            "ulysses_o_proj")
     return y
+
+
+def ulysses_qkv_proj_rope_bwd(x, w_qkv, P, H, G, rope_table, dq, dk, dv, positions=None, dx=None, dw=None,
+                              workspace=None, stream=None):
+    """Backward of ulysses_qkv_proj_rope: x seq layout [P][B][n/P][hidden] and
+    w_qkv as for the forward; dq [P][B][H/P][n][128], dk, dv [P][B][G/P][n][128]
+    (bf16 head layout) -> (dx bf16 like x, dw float32 like w_qkv)."""
+    P_, B, s, hidden = x.shape
+    n, d = P * s, 128
+    if P_ != P or tuple(w_qkv.shape) != ((H + 2 * G) * d, hidden):
+        raise UlyssesError(2, f"ulysses_qkv_proj_rope_bwd: x {tuple(x.shape)}, w {tuple(w_qkv.shape)} with P={P}")
+    if positions is not None and (positions.dtype != torch.int32 or tuple(positions.shape) != (B, n)):
+        raise UlyssesError(2, f"ulysses_qkv_proj_rope_bwd: positions {tuple(positions.shape)} {positions.dtype}")
+    dx = torch.empty_like(x) if dx is None else dx
+    dw = torch.empty(w_qkv.shape, dtype=torch.float32, device=x.device) if dw is None else dw
+    need = ctypes.c_size_t(0)
+    _check(lib().ulysses_qkv_proj_rope_bwd_workspace_size(B, n, H, G, d, ctypes.byref(need)),
+           "ulysses_qkv_proj_rope_bwd_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(need.value, 256), dtype=torch.uint8, device=x.device)
+    _check(lib().ulysses_qkv_proj_rope_bwd(B, n, P, hidden, H, G, d, _p(x), _p(w_qkv), _p(rope_table),
+                                           rope_table.shape[0], _p(positions), _p(dq), _p(dk), _p(dv), _p(dx),
+                                           _p(dw), _p(workspace), workspace.numel(), _stream(stream)),
+           "ulysses_qkv_proj_rope_bwd")
+    return dx, dw
+
+
+def ulysses_o_proj_bwd(o_seq, w_o, dy, P, do=None, dw_o=None, stream=None):
+    """Backward of ulysses_o_proj: o_seq [P][B][n/P][H][128] (the attention output
+    in the seq layout), w_o [hidden][H*128], dy seq layout [P][B][n/P][hidden]
+    -> (dO bf16 head layout [P][B][H/P][n][128], dW_o float32 like w_o)."""
+    P_, B, s, H, d = o_seq.shape
+    hidden = w_o.shape[0]
+    n = P * s
+    if P_ != P or tuple(w_o.shape) != (hidden, H * d) or tuple(dy.shape) != (P, B, s, hidden):
+        raise UlyssesError(2, f"ulysses_o_proj_bwd: o {tuple(o_seq.shape)}, w_o {tuple(w_o.shape)}, "
+                              f"dy {tuple(dy.shape)} with P={P}")
+    do = torch.empty((P, B, H // P, n, d), dtype=o_seq.dtype, device=o_seq.device) if do is None else do
+    dw_o = torch.empty(w_o.shape, dtype=torch.float32, device=o_seq.device) if dw_o is None else dw_o
+    _check(lib().ulysses_o_proj_bwd(B, n, P, hidden, H, d, _p(o_seq), _p(w_o), _p(dy), _p(do), _p(dw_o),
+                                    _stream(stream)), "ulysses_o_proj_bwd")
+    return do, dw_o
 
 
 # ----------------------------------------------------------------- attention
