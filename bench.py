@@ -392,6 +392,28 @@ def run_ours(args, rank, world, dev):
     except Exception as exc:  # noqa: BLE001 -- a side figure never breaks the bench line
         fwd_only = {"error": str(exc)[:200]}
 
+    # the deterministic (atomic-free, two-pass) backward on the same inputs, for
+    # comparison with the fused pass the step uses
+    det_bwd = None
+    try:
+        def det():
+            U.ulysses_attn_bwd(layer.qh, layer.kh, layer.vh, layer.o, layer.lse, layer.doh, mask=layer.mask,
+                               cu_seqlens=layer.cu, dq=layer.dq, dk=layer.dk, dv=layer.dv, workspace=layer.ws,
+                               out_seq_layout=True, deterministic=True)
+        det()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            det()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dms = e0.elapsed_time(e1) / args.steps
+        det_bwd = {"ms_per_call": dms,
+                   "tflops": 10.0 * inp["B"] * inp["H"] * inp["d"] * pairs / (dms / 1e3) / 1e12,
+                   "note": "statistics + dK/dV pass + dQ pass (S and dP formed twice), bitwise repeatable"}
+    except Exception as exc:  # noqa: BLE001 -- a side figure never breaks the bench line
+        det_bwd = {"error": str(exc)[:200]}
+
     # the fused loss + gradient, timed on its own (it follows the layer's loss
     # in training and is not part of the layer step)
     loss_bwd = None
@@ -478,6 +500,7 @@ def run_ours(args, rank, world, dev):
         "roofline": roof,
         "kernels": kernels,
         "forward_only": fwd_only,
+        "deterministic_backward": det_bwd,
         "loss_grad": loss_bwd,
         "side_kernels": side,
         "gpu_launches": launches,
@@ -560,16 +583,36 @@ def side_kernels(inp, dev, steps: int, peaks) -> dict:
         wo = (torch.randn((hidden, H * d), device=dev) / (H * d) ** 0.5).to(torch.bfloat16)
         yb = torch.empty((P, B, n // P, hidden), dtype=torch.bfloat16, device=dev)
         prof2 = timed(lambda: U.ulysses_o_proj(qb, wo, P, y=yb))
+        # the projections' backward (synthetic output gradients)
+        dx = torch.empty_like(x)
+        dwq = torch.empty(w.shape, dtype=torch.float32, device=dev)
+        ws = torch.empty(B * n * (H + 2 * G) * d * 2 + 256, dtype=torch.uint8, device=dev)
+        prof3 = timed(lambda: U.ulysses_qkv_proj_rope_bwd(x, w, P, H, G, tab, qb, kb, vb, dx=dx, dw=dwq, workspace=ws))
+        o_seq = torch.randn((P, B, n // P, H, d), device=dev).to(torch.bfloat16)
+        dyo = torch.randn((P, B, n // P, hidden), device=dev).to(torch.bfloat16)
+        do_h = torch.empty_like(qb)
+        dwo = torch.empty(wo.shape, dtype=torch.float32, device=dev)
+        prof4 = timed(lambda: U.ulysses_o_proj_bwd(o_seq, wo, dyo, P, do=do_h, dw_o=dwo))
+        fq, fo = 2.0 * B * n * (H + 2 * G) * d * hidden, 2.0 * B * n * hidden * H * d
         for name, pr, fl, note in (
-                ("qkv_proj_sm100", prof, 2.0 * B * n * (H + 2 * G) * d * hidden,
+                ("qkv_proj_sm100", prof, fq,
                  f"[Q K V] = X W^T, rotary positions, written in the head layout; hidden={hidden}"),
-                ("o_proj_sm100", prof2, 2.0 * B * n * hidden * H * d,
-                 f"Y = O W_o^T read from the head layout, written in the seq layout; hidden={hidden}")):
+                ("o_proj_sm100", prof2, fo,
+                 f"Y = O W_o^T read from the head layout, written in the seq layout; hidden={hidden}"),
+                ("qkv_proj_dx_sm100", prof3, fq, "dX = dY W (dY: head layout back to tokens, rotated by -pos)"),
+                ("qkv_proj_dw_sm100", prof3, fq, "dW = dY^T X over all tokens, fp32"),
+                ("o_proj_do_sm100", prof4, fo, "dO = dY W_o, written in the head layout"),
+                ("o_proj_dw_sm100", prof4, fo, "dW_o = dY^T O over all tokens, fp32")):
             tot, cnt = pr[name]
             tf = fl / (tot / cnt / 1e3) / 1e12
             out[name] = {"ms_per_launch": tot / cnt, "tflops": tf, "frac_bf16": tf / peaks["bf16_tflops"],
                          "flops_per_launch": fl, "note": note}
-        del x, w, tab, qb, kb, vb, wo, yb
+        tot, cnt = prof3["qkv_dy"]
+        dyb = B * n * (H + 2 * G) * d * 2.0 * 2
+        out["qkv_dy"] = {"ms_per_launch": tot / cnt, "gbs": dyb / (tot / cnt / 1e3) / 1e9,
+                         "frac_hbm": dyb / (tot / cnt / 1e3) / 1e9 / peaks["hbm_gbs"],
+                         "note": "dQ, dK, dV read from the head layout, dY written in token order (rotated)"}
+        del x, w, tab, qb, kb, vb, wo, yb, dx, dwq, ws, o_seq, dyo, do_h, dwo
     ids = torch.randint(0, 151936, (B, n), dtype=torch.int32, device=dev)
     lab = torch.empty((inp["P"], B, n // inp["P"]), dtype=torch.int32, device=dev)
     cu = inp["cu_seqlens"].to(dev) if inp["cu_seqlens"] is not None else None
