@@ -780,6 +780,21 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------------- main
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_command(gpus: int, argv) -> list:
+    """The command that runs this benchmark as `gpus` ranks, one per GPU of
+    this node (torch.distributed.run on 127.0.0.1), under a hard time limit."""
+    return ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", f"--master-port={_free_port()}",
+            os.path.abspath(__file__), *argv]
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -796,6 +811,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "ours" and args.gpus != world:
+        if world == 1 and args.gpus > 1 and "LOCAL_RANK" not in os.environ:
+            # started directly with --gpus N: run the same command as N ranks
+            raise SystemExit(subprocess.call(launch_command(args.gpus, sys.argv[1:])))
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:

@@ -105,3 +105,20 @@ def test_reference_arm_runs_on_rank_zero_only():
     class A:
         workload, steps, warmup = "qwen64k", 1, 3
     assert bench.run_reference(A, rank=1, world=2) is None
+
+
+def test_bench_gpus_flag_launches_one_rank_per_gpu():
+    """`bench.py --gpus N` started directly runs the same command as N ranks
+    (torch.distributed.run on 127.0.0.1); a WORLD_SIZE that disagrees with
+    --gpus stops it with a message."""
+    import subprocess
+    sys.path.insert(0, ROOT)
+    import bench
+    cmd = bench.launch_command(4, ["--gpus", "4", "--steps", "2"])
+    assert "torch.distributed.run" in cmd and "--nproc-per-node=4" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "2"] and cmd[-5].endswith("bench.py")
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE=3" in (r.stderr + r.stdout)
