@@ -35,8 +35,6 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kLoadsInFlight = 8;
-constexpr int kRegWarps = 8;                   // register-resident rows: one 256-thread CTA per SM
-constexpr int kRegThreads = kRegWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void merge(float &m, float &s, float m2, float s2) {
@@ -248,143 +246,6 @@ __global__ void __launch_bounds__(kThreads) ce_fwd_bwd_kernel(
   }
 }
 
-// Rows of up to 32 x 16 bytes per lane (16 KB: 8192 bf16 or 4096 fp32
-// logits): the warp holds its whole row in registers.  All of the row's loads
-// are issued at once (VPL 16-byte loads in flight per lane), then the exact
-// row maximum, the sum of exp(z - max) (eight independent sums per lane) and
-// LSE = max + log(sum); GRAD also writes dL/dz = (exp(z - LSE) - [v == y]) / C
-// from the registers -- every logit is read from memory once and no online
-// rescaling is needed.  The forward entry point and the fused gradient use
-// this same kernel body, so their loss values are bitwise equal.
-template <typename T, int VPL, bool GRAD>
-__global__ void __launch_bounds__(kRegThreads, 1) ce_row_reg_kernel(
-    const T *__restrict__ logits, const int32_t *__restrict__ labels, long long per_shard, int vocab,
-    int ignore_index, const long long *__restrict__ count, T *__restrict__ dlogits,
-    double *__restrict__ part_sum, long long *__restrict__ part_cnt, int *err) {
-  constexpr int kPerVec = 16 / sizeof(T);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y, nb = gridDim.x;
-  const int vecs = vocab / kPerVec;
-  float invC = 0.f;
-  if (GRAD) {
-    const long long C = *count;
-    invC = C > 0 ? (float)(1.0 / (double)C) : 0.f;
-  }
-  double acc = 0.0;
-  long long cnt = 0;
-  for (long long tt = (long long)blockIdx.x * kRegWarps + warp; tt < per_shard; tt += (long long)nb * kRegWarps) {
-    const long long t = (long long)r * per_shard + tt;
-    const int y = __ldg(labels + t);
-    const bool counted = y != ignore_index && y >= 0 && y < vocab;
-    if (!counted) {
-      if (y != ignore_index && lane == 0) raise_error(err, ULY_ERR_LABEL);
-      if (GRAD) {
-        uint4 *drow = reinterpret_cast<uint4 *>(dlogits + t * (long long)vocab);
-        for (int v = lane; v < vecs; v += 32) __stcs(drow + v, make_uint4(0, 0, 0, 0));
-      }
-      continue;
-    }
-    const uint4 *row = reinterpret_cast<const uint4 *>(logits + t * (long long)vocab);
-    uint4 u[VPL];
-#pragma unroll
-    for (int k = 0; k < VPL; ++k) {
-      const int v = lane + 32 * k;
-      u[k] = (v < vecs) ? __ldcs(row + v) : make_uint4(0, 0, 0, 0);
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < VPL; ++k) {
-      if (lane + 32 * k < vecs) {
-        float x[8];
-        load_vals<T>(u[k], x);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, x[e]);
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const float mx2 = mx * kLog2e;
-    float sm8[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) sm8[e] = 0.f;
-#pragma unroll
-    for (int k = 0; k < VPL; ++k) {
-      if (lane + 32 * k < vecs) {
-        float x[8];
-        load_vals<T>(u[k], x);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm8[e] += exp2f(fmaf(x[e], kLog2e, -mx2));
-      }
-    }
-    float sm = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
-    const float lse = mx + logf(sm);
-    if (lane == 0) {
-      acc += (double)lse - (double)static_cast<float>(logits[t * (long long)vocab + y]);
-      cnt += 1;
-    }
-    if (GRAD) {
-      uint4 *drow = reinterpret_cast<uint4 *>(dlogits + t * (long long)vocab);
-      const float l2 = lse * kLog2e;
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) {
-        const int v = lane + 32 * k;
-        if (v < vecs) {
-          float x[8];
-          load_vals<T>(u[k], x);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float gv = exp2f(fmaf(x[e], kLog2e, -l2)) * invC;
-            if (v * kPerVec + e == y) gv -= invC;
-            x[e] = gv;
-          }
-          __stcs(drow + v, pack_vals<T>(x));
-        }
-      }
-    }
-  }
-  __shared__ double sh_sum[kRegWarps];
-  __shared__ long long sh_cnt[kRegWarps];
-  if (lane == 0) { sh_sum[warp] = acc; sh_cnt[warp] = cnt; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double a = 0.0;
-    long long c = 0;
-    for (int w = 0; w < kRegWarps; ++w) { a += sh_sum[w]; c += sh_cnt[w]; }  // fixed order
-    part_sum[(long long)r * nb + blockIdx.x] = a;
-    part_cnt[(long long)r * nb + blockIdx.x] = c;
-  }
-}
-
-// Launch the register-resident kernel when a row fits (<= 1024 vectors);
-// false otherwise (the streaming kernels are used).
-template <bool GRAD>
-bool launch_row_reg(int dtype, dim3 grid, cudaStream_t stream, const void *logits, const int32_t *labels,
-                    long long per, int vocab, int ignore_index, const long long *count, void *dlogits,
-                    double *psum, long long *pcnt, int *err) {
-  const int eb = dtype == ULY_BF16 ? 2 : 4;
-  const int vecs = (int)((long long)vocab * eb / 16);
-#define ULY_CE_REG(VPL_)                                                                                    \
-  if (vecs <= 32 * (VPL_)) {                                                                               \
-    if (dtype == ULY_BF16)                                                                                 \
-      ce_row_reg_kernel<__nv_bfloat16, VPL_, GRAD><<<grid, kRegThreads, 0, stream>>>(                       \
-          static_cast<const __nv_bfloat16 *>(logits), labels, per, vocab, ignore_index, count,             \
-          static_cast<__nv_bfloat16 *>(dlogits), psum, pcnt, err);                                         \
-    else                                                                                                   \
-      ce_row_reg_kernel<float, VPL_, GRAD><<<grid, kRegThreads, 0, stream>>>(                               \
-          static_cast<const float *>(logits), labels, per, vocab, ignore_index, count,                     \
-          static_cast<float *>(dlogits), psum, pcnt, err);                                                 \
-    return true;                                                                                           \
-  }
-  ULY_CE_REG(4)
-  ULY_CE_REG(8)
-  ULY_CE_REG(16)
-  ULY_CE_REG(32)
-#undef ULY_CE_REG
-  return false;
-}
-
 // One CTA: shard r's partials are folded by thread r in index order; then
 // thread 0 folds the shards in rank order.
 __global__ void __launch_bounds__(256) ce_finalize_kernel(
@@ -415,8 +276,7 @@ __global__ void __launch_bounds__(256) ce_finalize_kernel(
 }  // namespace
 
 int loss_blocks_per_shard(int P, long long per_shard) {
-  // about four CTAs per SM in total (the register-resident kernel runs them
-  // in waves, one per SM at a time), at most one warp per token
+  // about four CTAs per SM in total, at most one warp per token
   long long nb = (4LL * 148 + P - 1) / P;
   long long need = (per_shard + kWarps - 1) / kWarps;
   if (nb > need) nb = need;
@@ -452,9 +312,7 @@ uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, 
   long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb * P);
   dim3 grid(nb, P);
   prof::Scope s1(prof::K_LOSS_PARTIAL, stream);
-  if (launch_row_reg<false>(dtype, grid, stream, logits, labels, per, vocab, ignore_index, nullptr, nullptr, psum,
-                            pcnt, error_word())) {
-  } else if (dtype == ULY_BF16)
+  if (dtype == ULY_BF16)
     ce_partial_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(logits), labels, per, vocab, ignore_index, psum, pcnt,
         error_word());
@@ -487,9 +345,7 @@ uly_status loss_bwd_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dty
   dim3 grid(nb, P);
   prof::Scope s1(prof::K_LOSS_FWD_BWD, stream);
   ce_count_kernel<<<1, 1024, 0, stream>>>(labels, tokens, vocab, ignore_index, count);
-  if (launch_row_reg<true>(dtype, grid, stream, logits, labels, per, vocab, ignore_index, count, dlogits, psum,
-                           pcnt, error_word())) {
-  } else if (dtype == ULY_BF16)
+  if (dtype == ULY_BF16)
     ce_fwd_bwd_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(logits), labels, per, vocab, ignore_index, count,
         static_cast<__nv_bfloat16 *>(dlogits), psum, pcnt, error_word());
