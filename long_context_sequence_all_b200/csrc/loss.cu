@@ -7,24 +7,20 @@
 //   S_r = sum_{t in shard r} l_t,  C_r = #valid tokens of shard r
 //   L   = sum_r S_r / sum_r C_r
 //
-// Pass 1: one warp per token.  Rows of up to 16 KB (the workloads' 8192
-// bf16 logits) are held whole in the warp's registers: every load of the row
-// is issued at once, then the exact row maximum, the sum of exp(z - max) and
-// LSE = max + log(sum) (ce_row_reg_kernel).  Longer rows stream through with
-// eight 16-byte loads in flight per lane and a running (max, sum) per lane,
-// merged with shuffles.  Every CTA writes one (sum, count) partial for its
-// shard into the workspace.  Pass 2: one CTA folds the partials in a fixed
-// order (deterministic) into S_r, C_r and L.  HBM-bound: each logits byte is
-// read once.
+// Pass 1: one warp per token streams the token's logits row once (16-byte
+// loads, eight in flight per lane), keeping a running (max, sum) per lane;
+// lanes merge with shuffles.  Every CTA writes one (sum, count) partial for
+// its shard into the workspace.  Pass 2: one CTA per launch folds the
+// partials in a fixed order (deterministic) into S_r, C_r and L.
+// HBM-bound: each logits byte is read once.
 //
 // The gradient (the training step after the aggregation) has the global
 // count C = sum_r C_r as its only denominator:
 //   dL/dz_tv = (softmax(z_t)_v - [v == y_t]) / C   (counted tokens; else 0)
 // The fused forward+backward counts the valid labels first (one CTA, labels
-// only); then the same row kernel, after LSE, writes dL/dz from the registers
-// with 16-byte streaming stores (longer rows: the row is read again, from L2).
-// Logits read once from HBM, dlogits written once; the loss values equal the
-// forward entry point's bit for bit.
+// only), then each token's warp computes the row's logsumexp exactly as the
+// forward does, re-reads the row (now in L2) and writes dL/dz with 16-byte
+// stores: logits read once from HBM, dlogits written once.
 #include "common.cuh"
 #include "prof.cuh"
 
