@@ -780,6 +780,53 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------------- main
 
+KERNEL_ONLY = ("attn_fwd", "attn_bwd", "attn_bwd_deterministic", "seq_to_head", "head_to_seq", "loss", "loss_bwd")
+
+
+def run_kernel_only(args, dev):
+    """One entry point of the layer, alone, `steps` times on the workload's
+    operands (no other kernel of the step runs), for profiling a single kernel
+    with few launches before it; prints its CUDA-event time per call.  Not a
+    bench line."""
+    from long_context_sequence_all_b200 import build, ulysses as U
+    build.build()
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, seed=rank_seed(w, 0))
+    layer = Layer(inp, dev)
+    P, U_ = layer.P, U
+    calls = {
+        "attn_fwd": lambda: U_.ulysses_attn_fwd(layer.qh, layer.kh, layer.vh, mask=layer.mask, cu_seqlens=layer.cu,
+                                                o=layer.o, lse=layer.lse, out_seq_layout=True),
+        "attn_bwd": lambda: U_.ulysses_attn_bwd(layer.qh, layer.kh, layer.vh, layer.o, layer.lse, layer.doh,
+                                                mask=layer.mask, cu_seqlens=layer.cu, dq=layer.dq, dk=layer.dk,
+                                                dv=layer.dv, workspace=layer.ws, out_seq_layout=True),
+        "attn_bwd_deterministic": lambda: U_.ulysses_attn_bwd(
+            layer.qh, layer.kh, layer.vh, layer.o, layer.lse, layer.doh, mask=layer.mask, cu_seqlens=layer.cu,
+            dq=layer.dq, dk=layer.dk, dv=layer.dv, workspace=layer.ws, out_seq_layout=True, deterministic=True),
+        "seq_to_head": lambda: U_.ulysses_seq_to_head_batch([layer.q, layer.k, layer.v], P,
+                                                            outs=[layer.qh, layer.kh, layer.vh]),
+        "head_to_seq": lambda: U_.ulysses_head_to_seq_batch([layer.qh, layer.kh, layer.vh], P,
+                                                            outs=[layer.q, layer.k, layer.v]),
+        "loss": lambda: U_.ulysses_loss_aggregate(layer.logits, layer.labels, P, shard_sum=layer.S,
+                                                  shard_count=layer.C, loss=layer.L, workspace=layer.lws),
+        "loss_bwd": layer.loss_bwd,
+    }
+    fn = calls[args.kernel_only]
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if U.ulysses_read_error():
+        raise RuntimeError("device error word set")
+    print(json.dumps({"kernel_only": args.kernel_only, "workload": args.workload, "calls": args.steps,
+                      "ms_per_call": e0.elapsed_time(e1) / args.steps}), flush=True)
+
+
 def _free_port() -> int:
     import socket
     with socket.socket() as sk:
@@ -804,6 +851,8 @@ def main():
     ap.add_argument("--workload", default="qwen64k", choices=sorted(k for k in WORKLOADS if k != "tiny_f32"))
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", choices=KERNEL_ONLY, default=None,
+                    help="run one entry point alone (for profiling); prints its time per call, not a bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -825,6 +874,9 @@ def main():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.kernel_only:
+        run_kernel_only(args, dev)
+        return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                              device_id=dev)

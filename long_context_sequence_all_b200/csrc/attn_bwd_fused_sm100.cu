@@ -73,13 +73,19 @@ constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTX = 384;
 
 // Register split: control warpgroup, two compute warpgroups, dQ warpgroup.
 constexpr int kRegsLaunch = 128;
-constexpr int kRegsCtl = 88, kRegsCompute = 168, kRegsDq = 88;
+constexpr int kRegsCtl = 88, kRegsCompute = 144, kRegsDq = 136;
 static_assert(128 * (kRegsCtl + 2 * kRegsCompute + kRegsDq) == kThreads * kRegsLaunch,
               "register split must use exactly the launch pool");
+static_assert(kRegsCtl < kRegsLaunch && kRegsCompute > kRegsLaunch, "the control warpgroup gives, the compute ones take");
 
 constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);   // A, B K-major
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, false, true);    // B MN-major
 constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);     // A, B MN-major
+
+// Fire-and-forget fp32 add into global memory (performed in L2).
+__device__ __forceinline__ void red_add_f32(float *p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
 
 struct FusedParams {
   const float *lse2;    // [qheads][n_pad]: LSE log2(e), 0 past n
@@ -311,18 +317,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t r[64];
       tmem_ld64(tS, r);
       uint32_t pp[32];
+      // LSE log2(e) of the 64 query rows: one broadcast 16-byte shared-memory
+      // load per 4 columns
+      const float4 *l4 = reinterpret_cast<const float4 *>(lsm);
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          float pv = ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lsm[c + u]));
-          if (!full) {
-            const int i = i0 + c + u;
-            if (i < lo_j || i > hi_j) pv = 0.f;
-          }
-          r[c + u] = __float_as_uint(pv);
+      for (int c = 0; c < 64; c += 4) {
+        const float4 L = l4[c >> 2];
+        float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -L.x));
+        float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), prm.scale_log2, -L.y));
+        float p2 = ex2_approx(fmaf(__uint_as_float(r[c + 2]), prm.scale_log2, -L.z));
+        float p3 = ex2_approx(fmaf(__uint_as_float(r[c + 3]), prm.scale_log2, -L.w));
+        if (!full) {
+          const int i = i0 + c;
+          if (i < lo_j || i > hi_j) p0 = 0.f;
+          if (i + 1 < lo_j || i + 1 > hi_j) p1 = 0.f;
+          if (i + 2 < lo_j || i + 2 > hi_j) p2 = 0.f;
+          if (i + 3 < lo_j || i + 3 > hi_j) p3 = 0.f;
         }
-        pp[c >> 1] = pack_bf16x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        r[c] = __float_as_uint(p0);
+        r[c + 1] = __float_as_uint(p1);
+        r[c + 2] = __float_as_uint(p2);
+        r[c + 3] = __float_as_uint(p3);
+        pp[c >> 1] = pack_bf16x2(p0, p1);
+        pp[(c >> 1) + 1] = pack_bf16x2(p2, p3);
       }
       tmem_st32_nowait(tS, pp);
       tmem_st_wait();
@@ -336,11 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t dp[64];
       tmem_ld64(tP, dp);
       uint32_t dd[32];
+      const float4 *d4 = reinterpret_cast<const float4 *>(dsm);
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float d0 = __uint_as_float(r[c]) * (__uint_as_float(dp[c]) - dsm[c]);
-        const float d1 = __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - dsm[c + 1]);
-        dd[c >> 1] = pack_bf16x2(d0, d1);
+      for (int c = 0; c < 64; c += 4) {
+        const float4 dq4 = d4[c >> 2];
+        dd[c >> 1] = pack_bf16x2(__uint_as_float(r[c]) * (__uint_as_float(dp[c]) - dq4.x),
+                                 __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - dq4.y));
+        dd[(c >> 1) + 1] = pack_bf16x2(__uint_as_float(r[c + 2]) * (__uint_as_float(dp[c + 2]) - dq4.z),
+                                       __uint_as_float(r[c + 3]) * (__uint_as_float(dp[c + 3]) - dq4.w));
       }
       // the previous tile's dQ^T and dK MMAs have read the buffer
       if (t > 0) {
@@ -385,7 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- dQ
-    setmaxnreg_dec<kRegsDq>();
+    if constexpr (kRegsDq > kRegsLaunch) setmaxnreg_inc<kRegsDq>();
+    else if constexpr (kRegsDq < kRegsLaunch) setmaxnreg_dec<kRegsDq>();
     const int wq = warp & 3;
     const int dcol = wq * 32 + lane;               // head dimension = TMEM lane of dQ^T
     const uint32_t tX = tmem + ((uint32_t)(wq * 32) << 16) + kTX;
@@ -394,15 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *dst = prm.dq_acc + ((long long)(qh_base + e) * prm.n_pad + i0) * kHD + dcol;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQF), t & 1, abort_flag, prm.err, prm.wait_limit))) break;
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld64(tX, v);
-#pragma unroll
-      for (int q = 0; q < 64; ++q) atomicAdd(dst + q * kHD, __uint_as_float(v[q]));
-      tmem_ld64(tX + 64, v);
+      // the whole dQ^T row (128 queries) in one read, so that the columns are
+      // handed back to the next dP^T before any of the adds is issued
+      uint32_t v[128];
+      tmem_ld64x2(tX, tX + 64, v);
       tc_fence_before();
       mbar_arrive(bar(B_DQE));
 #pragma unroll
-      for (int q = 0; q < 64; ++q) atomicAdd(dst + (64 + q) * kHD, __uint_as_float(v[q]));
+      for (int q = 0; q < 128; ++q) red_add_f32(dst + q * kHD, __uint_as_float(v[q]));
     }
   }
 
