@@ -17,8 +17,8 @@
 // run, so dQ is not bitwise repeatable (dK and dV are).
 //
 // Warp roles (512 threads):
-//   warp 0       TMA: K, V once; Q tiles (+ LSE log2 e) and dO tiles (+ D),
-//                two stages each
+//   warp 0       TMA: K, V once; Q tiles (+ LSE log2 e) in three stages, dO
+//                tiles in one
 //   warp 1       TMEM allocation and the MMA-issuing thread:
 //                  S^T  = K Q^T           (SS, M=128 keys, N=128 queries)
 //                  dP^T = V dO^T          (SS)
@@ -54,15 +54,20 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kBN = 128;   // keys per CTA
 constexpr int kBQ = 128;   // query rows per tile
-constexpr int kQStages = 2, kOStages = 2;
+// Q tiles have three stages: a Q tile is read by S^T (early) and dK (late),
+// so its stage is refilled only after the tile's dK.  dO tiles have one: their
+// last reader is dV, near the start of the tile, so the stage is released
+// right after it.  D is read by the compute warps from the statistics array in
+// global memory (L1-resident broadcast loads), so they never wait on the dO
+// stage, whose barrier completes a phase every tile.
+constexpr int kQStages = 3, kOStages = 1;
 constexpr uint32_t kTile = 128 * 128 * 2;                // one 128 x 128 bf16 tile
 constexpr uint32_t kOffK = 0, kOffV = kTile;
 constexpr uint32_t kOffQ = 2 * kTile;                    // Q stage s at kOffQ + s * kTile
 constexpr uint32_t kOffO = kOffQ + kQStages * kTile;     // dO stage s
 constexpr uint32_t kOffS = kOffO + kOStages * kTile;     // dS^T [key][query], two 64-query halves
 constexpr uint32_t kOffLse = kOffS + kTile;              // per Q stage: 128 LSE log2(e)
-constexpr uint32_t kOffD = kOffLse + kQStages * kBQ * 4; // per dO stage: 128 D
-constexpr uint32_t kEnd = kOffD + kOStages * kBQ * 4;
+constexpr uint32_t kEnd = kOffLse + kQStages * kBQ * 4;
 constexpr uint32_t kBarBytes = 192;
 constexpr uint32_t kSmemBytes = 232448;                  // all an SM offers one CTA
 // The tiles need a 1024-byte-aligned base.  The barriers go in front of it
@@ -73,7 +78,7 @@ constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTX = 384;
 
 // Register split: control warpgroup, two compute warpgroups, dQ warpgroup.
 constexpr int kRegsLaunch = 128;
-constexpr int kRegsCtl = 88, kRegsCompute = 144, kRegsDq = 136;
+constexpr int kRegsCtl = 80, kRegsCompute = 144, kRegsDq = 144;
 static_assert(128 * (kRegsCtl + 2 * kRegsCompute + kRegsDq) == kThreads * kRegsLaunch,
               "register split must use exactly the launch pool");
 static_assert(kRegsCtl < kRegsLaunch && kRegsCompute > kRegsLaunch, "the control warpgroup gives, the compute ones take");
@@ -179,10 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           issued_q = t + 1;
           const int so = t % kOStages, uo = t / kOStages;
           if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
-          mbar_arrive_expect_tx(bar(B_OF + so), kTile + kBQ * 4);
+          mbar_arrive_expect_tx(bar(B_OF + so), kTile);
           for (int c = 0; c < 2; ++c)
             tma_load_3d(sb + kOffO + so * kTile + c * 16384, &tmO, bar(B_OF + so), c * 64, i0, qh_base + e);
-          bulk_load(sb + kOffD + so * kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_OF + so));
           issued_o = t + 1;
         }
         // Every copy issued lands before the CTA can exit, also when a consumer
@@ -242,8 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dOn = sdesc_sw128(sb + kOffO + so1 * kTile, 16, 1024);     // next dP^T: B = next dO
           // dV += P^T dO_t: A from TMEM (query columns [0,64) in the S^T
           // columns [0,32), [64,128) in [64,96))
-          ok = more ? mbar_wait2(bar(B_PS), t & 1, bar(B_QF + sq1), pq1, abort_flag, prm.err, prm.wait_limit)
-                    : mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err, prm.wait_limit);
+          ok = mbar_wait(bar(B_PS), t & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -252,8 +255,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ts(tmem + kTdV, tmem + kTS + acol, sdesc_add(dOm, kk * 2048), kIdescKM,
                         (t > 0 || kk > 0) ? 1u : 0u);
           }
+          // dO_t has been read by its two MMAs (dP^T earlier, dV now)
+          tc_commit(bar(B_OE + so));
           // the next tile's S^T over this tile's P^T (after the dV MMA in issue order)
-          if (more) issue_s(dQn);
+          if (more) {
+            ok = mbar_wait(bar(B_QF + sq1), pq1, abort_flag, prm.err, prm.wait_limit);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(dQn);
+          }
           // dS^T of the tile is in shared memory and the dP^T columns are read
           ok = mbar_wait(bar(B_DS), t & 1, abort_flag, prm.err, prm.wait_limit);
           if (!ok) break;
@@ -271,9 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ss(tmem + kTdK, sdesc_add(dSa, ko), sdesc_add(dQm, kk * 2048), kIdescKM,
                         (t > 0 || kk > 0) ? 1u : 0u);
           }
-          // tile t's Q and dO stages and the dS^T buffer are free once dK is done
+          // tile t's Q stage and the dS^T buffer are free once dK is done
           tc_commit(bar(B_QE + sq));
-          tc_commit(bar(B_OE + so));
           tc_commit(bar(B_DSE));
           if (more) {
             // the next dP^T reuses the dQ^T columns once the dQ warpgroup has read them
@@ -305,9 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ + 64 * w;  // this warpgroup's first query row
-      const int sq = t % kQStages, so = t % kOStages;
+      const int sq = t % kQStages;
       const float *lsm = reinterpret_cast<const float *>(smem + kOffLse + sq * kBQ * 4) + 64 * w;
-      const float *dsm = reinterpret_cast<const float *>(smem + kOffD + so * kBQ * 4) + 64 * w;
+      // D of this warpgroup's 64 query rows (the statistics kernel's padded array)
+      const float4 *d4 = reinterpret_cast<const float4 *>(prm.Dv + (long long)(qh_base + e) * prm.n_pad + i0);
       // P^T over this warpgroup's first 32 columns of S^T
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
                                        mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err, prm.wait_limit));
@@ -346,17 +356,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_PS));
       // dS^T = P^T (dP^T - D) into shared memory
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + so), (t / kOStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
-                                       mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err, prm.wait_limit));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), t & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
       tc_fence_after();
       uint32_t dp[64];
       tmem_ld64(tP, dp);
       uint32_t dd[32];
-      const float4 *d4 = reinterpret_cast<const float4 *>(dsm);
 #pragma unroll
       for (int c = 0; c < 64; c += 4) {
-        const float4 dq4 = d4[c >> 2];
+        const float4 dq4 = __ldg(d4 + (c >> 2));
         dd[c >> 1] = pack_bf16x2(__uint_as_float(r[c]) * (__uint_as_float(dp[c]) - dq4.x),
                                  __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - dq4.y));
         dd[(c >> 1) + 1] = pack_bf16x2(__uint_as_float(r[c + 2]) * (__uint_as_float(dp[c + 2]) - dq4.z),
