@@ -25,7 +25,9 @@
 // Ordering: s_full[t] is committed after S_j(t), which is issued after
 // O_t += P_{j-1} V_{j-1}; a commit tracks every earlier MMA of the thread, so
 // when softmax sees S_j it also knows the previous PV finished (O may be
-// rescaled).  p_full[t] hands P_j to the MMA warp.  S_{j+1}(t) overwrites the
+// rescaled).  p_full[t] hands P_j to the MMA warp in two halves (keys
+// [0,64) and [64,128)), so the first half of P_j V_j runs while the softmax
+// warps compute the second.  S_{j+1}(t) overwrites the
 // columns that O_t += P_j V_j reads; both are MMAs of this one issuing thread
 // and the tensor core executes them in issue order.
 // Every wait is bounded (ULY_ERR_TIMEOUT), no wait can spin forever.
@@ -75,8 +77,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   // barrier indices
+  // B_PF + 2t + h: the P of tile t for keys [64h, 64h + 64) is in TMEM
   enum { B_Q = 0, B_KVF = 1, B_KVE = 1 + kSlots, B_SF = 1 + 2 * kSlots, B_PF = B_SF + 2,
-         B_OF = B_PF + 2, B_DRAIN = B_OF + 2, B_N = B_DRAIN + 1 };
+         B_OF = B_PF + 4, B_DRAIN = B_OF + 2, B_N = B_DRAIN + 1 };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * B_N + 4);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_N; ++i) {
       uint32_t cnt = 1;
-      if (i == B_PF || i == B_PF + 1) cnt = 128;
+      if (i >= B_PF && i < B_PF + 4) cnt = 128;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -154,13 +157,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag, prm.err, prm.wait_limit);
       tc_fence_after();
       // descriptors of the fixed operands; per-k-step offsets are constants
-      const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
-      const uint64_t dq1 = sdesc_sw128(sb + kOffQ + kTileBytes, 16, 1024);
-      auto issue_pv = [&](int t, uint64_t dv, bool first) {   // dv: V tile, MN-major
+      uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
+      uint64_t dq1 = sdesc_sw128(sb + kOffQ + kTileBytes, 16, 1024);
+      // O_t += P_t V over the keys [64h, 64h + 64) (dv: V tile, MN-major)
+      auto issue_pv = [&](int t, uint64_t dv, bool first, int h) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int k4 = 0; k4 < kBN / 32; ++k4) {
+          const int kk = 4 * h + k4;
           mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, sdesc_add(dv, kk * 2048), kIdescPV,
                       (!first || kk > 0) ? 1u : 0u);
+        }
       };
       auto issue_s = [&](int t, uint64_t dk) {
         const uint64_t dq = t ? dq1 : dq0;
@@ -176,6 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int slotK = 0, slotV = kSlots - 1;
       uint32_t parK = 0, parV = 1;
       for (int it = 0; ok && it < NT; ++it) {
+        // opaque to the compiler, so the per-step descriptors are formed next
+        // to their MMAs instead of being hoisted out of the loop
+        asm volatile("" : "+l"(dq0), "+l"(dq1));
         const uint64_t dk = sdesc_sw128(sb + kOffKV + slotK * kTileBytes, 16, 1024);
         const uint64_t dv = sdesc_sw128(sb + kOffKV + slotV * kTileBytes, 16384, 1024);   // V: MN-major
         ok = (it > 0) ? mbar_wait2(bar(B_KVF + slotK), parK, bar(B_KVF + slotV), parV, abort_flag, prm.err, prm.wait_limit)
@@ -184,10 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int t = 0; t < 2 && ok; ++t) {
           if (it > 0) {
-            ok = mbar_wait(bar(B_PF + t), (it - 1) & 1, abort_flag, prm.err, prm.wait_limit);
+            // the first half of P V starts while the softmax still computes the second
+            for (int h = 0; h < 2 && ok; ++h) {
+              ok = mbar_wait(bar(B_PF + 2 * t + h), (it - 1) & 1, abort_flag, prm.err, prm.wait_limit);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, dv, it == 1, h);
+            }
             if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, dv, it == 1);
           }
           issue_s(t, dk);
           tc_commit(bar(B_SF + t));
@@ -206,10 +219,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(bar(B_KVF + slotV), parV, abort_flag, prm.err, prm.wait_limit);
         tc_fence_after();
         for (int t = 0; t < 2 && ok; ++t) {
-          ok = mbar_wait(bar(B_PF + t), (NT - 1) & 1, abort_flag, prm.err, prm.wait_limit);
+          for (int h = 0; h < 2 && ok; ++h) {
+            ok = mbar_wait(bar(B_PF + 2 * t + h), (NT - 1) & 1, abort_flag, prm.err, prm.wait_limit);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, dv, NT == 1, h);
+          }
           if (!ok) break;
-          tc_fence_after();
-          issue_pv(t, dv, NT == 1);
           tc_commit(bar(B_OF + t));
         }
         if (ok) tc_commit(bar(B_KVE + slotV));
@@ -299,11 +315,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[(x - hh * 64) >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st32_nowait(tS + hh * 32, pk);
+        // hand this half of P to the MMA thread
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(B_PF + 2 * wg + hh));
       }
       l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(B_PF + wg));
     }
     // ---------------------------------------------------------- epilogue
     if (ok && NT > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + wg), 0, abort_flag, prm.err, prm.wait_limit));
