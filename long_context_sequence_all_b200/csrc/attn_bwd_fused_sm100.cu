@@ -17,8 +17,8 @@
 // run, so dQ is not bitwise repeatable (dK and dV are).
 //
 // Warp roles (512 threads):
-//   warp 0       TMA: K, V once; Q tiles (+ LSE log2 e) in three stages, dO
-//                tiles in one
+//   warp 0       TMA: K, V once; Q tiles (+ LSE log2 e and D of their rows)
+//                in two stages, dO tiles in one
 //   warp 1       TMEM allocation and the MMA-issuing thread:
 //                  S^T  = K Q^T           (SS, M=128 keys, N=128 queries)
 //                  dP^T = V dO^T          (SS)
@@ -27,7 +27,8 @@
 //                  dK  += dS^T Q          (SS: dS^T from shared memory)
 //   warps 4-11   two compute warpgroups, one key row per thread, each half of
 //                the tile's query columns: P^T into TMEM (bf16 pairs over the
-//                S^T columns already read), dS^T (bf16) into shared memory
+//                S^T columns already read), dS^T (bf16) into one of two
+//                shared-memory buffers
 //   warps 12-15  dQ warpgroup: one head dimension per thread reads the
 //                tile's dQ^T row from TMEM and adds it into the accumulator
 //                (32 lanes = 32 consecutive floats of one query row per add)
@@ -54,20 +55,23 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kBN = 128;   // keys per CTA
 constexpr int kBQ = 128;   // query rows per tile
-// Q tiles have three stages: a Q tile is read by S^T (early) and dK (late),
-// so its stage is refilled only after the tile's dK.  dO tiles have one: their
-// last reader is dV, near the start of the tile, so the stage is released
-// right after it.  D is read by the compute warps from the statistics array in
-// global memory (L1-resident broadcast loads), so they never wait on the dO
-// stage, whose barrier completes a phase every tile.
-constexpr int kQStages = 3, kOStages = 1;
+// Q tiles have two stages: a Q tile is read by S^T (early) and dK (late), so
+// its stage is refilled only after the tile's dK.  The LSE and D of the
+// tile's rows arrive with it, so the compute warps read both from shared
+// memory behind the one barrier they already wait on.  dO tiles have one
+// stage: their last reader is dV, near the start of the tile, so the stage is
+// released right after it.  dS^T has two buffers, so that a tile's dS^T can be
+// written while the previous tile's dQ^T and dK MMAs still read theirs.
+constexpr int kQStages = 2, kOStages = 1, kSStages = 2;
+static_assert(kSStages == 2, "the dS^T buffer of tile t is t & 1");
 constexpr uint32_t kTile = 128 * 128 * 2;                // one 128 x 128 bf16 tile
 constexpr uint32_t kOffK = 0, kOffV = kTile;
 constexpr uint32_t kOffQ = 2 * kTile;                    // Q stage s at kOffQ + s * kTile
 constexpr uint32_t kOffO = kOffQ + kQStages * kTile;     // dO stage s
-constexpr uint32_t kOffS = kOffO + kOStages * kTile;     // dS^T [key][query], two 64-query halves
-constexpr uint32_t kOffLse = kOffS + kTile;              // per Q stage: 128 LSE log2(e)
-constexpr uint32_t kEnd = kOffLse + kQStages * kBQ * 4;
+constexpr uint32_t kOffS = kOffO + kOStages * kTile;     // dS^T buffer b: [key][query], two 64-query halves
+constexpr uint32_t kOffLse = kOffS + kSStages * kTile;   // per Q stage: 128 LSE log2(e)
+constexpr uint32_t kOffD = kOffLse + kQStages * kBQ * 4; // per Q stage: 128 D
+constexpr uint32_t kEnd = kOffD + kQStages * kBQ * 4;
 constexpr uint32_t kBarBytes = 192;
 constexpr uint32_t kSmemBytes = 232448;                  // all an SM offers one CTA
 // The tiles need a 1024-byte-aligned base.  The barriers go in front of it
@@ -121,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *bar_area = (gap >= kBarBytes) ? smem_raw : smem + kEnd;
   uint64_t *bars = reinterpret_cast<uint64_t *>(bar_area);
   enum { B_KV = 0, B_QF = 1, B_QE = B_QF + kQStages, B_OF = B_QE + kQStages, B_OE = B_OF + kOStages,
-         B_SF = B_OE + kOStages, B_PS, B_DPF, B_DS, B_DSE, B_DQF, B_DQE, B_DONE, B_DRAIN, B_N };
+         B_SF = B_OE + kOStages, B_PS, B_DPF, B_DS, B_DSE, B_DQF = B_DSE + kSStages, B_DQE, B_DONE, B_DRAIN, B_N };
   static_assert(8 * B_N + 8 <= kBarBytes, "barrier area");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + 8 * B_N);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + 8 * B_N + 4);
@@ -177,10 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const long long srow = (long long)(qh_base + e) * prm.n_pad + i0;
           const int sq = t % kQStages, uq = t / kQStages;
           if (uq > 0 && !mbar_wait(bar(B_QE + sq), (uq - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
-          mbar_arrive_expect_tx(bar(B_QF + sq), kTile + kBQ * 4);
+          mbar_arrive_expect_tx(bar(B_QF + sq), kTile + 2 * kBQ * 4);
           for (int c = 0; c < 2; ++c)
             tma_load_3d(sb + kOffQ + sq * kTile + c * 16384, &tmQ, bar(B_QF + sq), c * 64, i0, qh_base + e);
           bulk_load(sb + kOffLse + sq * kBQ * 4, prm.lse2 + srow, kBQ * 4, bar(B_QF + sq));
+          bulk_load(sb + kOffD + sq * kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_QF + sq));
           issued_q = t + 1;
           const int so = t % kOStages, uo = t / kOStages;
           if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
@@ -270,20 +275,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // dQ^T = K^T dS^T into the dP^T columns: M = head dims, N = queries,
           // K = the CTA's keys (16 rows of both tiles per step)
+          const uint32_t sbo = (uint32_t)(t & 1) * kTile;   // this tile's dS^T buffer
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_bf16_ss(tmem + kTX, sdesc_add(dKt, kk * 2048), sdesc_add(dSb, kk * 2048), kIdescMM, kk > 0);
+            mma_bf16_ss(tmem + kTX, sdesc_add(dKt, kk * 2048), sdesc_add(dSb, sbo + kk * 2048), kIdescMM, kk > 0);
           tc_commit(bar(B_DQF));
           // dK += dS^T Q_t: A = dS^T (K-major: the queries of a key row)
 #pragma unroll
           for (int kk = 0; kk < kBQ / 16; ++kk) {
             const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + kTdK, sdesc_add(dSa, ko), sdesc_add(dQm, kk * 2048), kIdescKM,
+            mma_bf16_ss(tmem + kTdK, sdesc_add(dSa, sbo + ko), sdesc_add(dQm, kk * 2048), kIdescKM,
                         (t > 0 || kk > 0) ? 1u : 0u);
           }
-          // tile t's Q stage and the dS^T buffer are free once dK is done
+          // tile t's Q stage and dS^T buffer are free once dK is done
           tc_commit(bar(B_QE + sq));
-          tc_commit(bar(B_DSE));
+          tc_commit(bar(B_DSE + (t & 1)));
           if (more) {
             // the next dP^T reuses the dQ^T columns once the dQ warpgroup has read them
             ok = mbar_wait2(bar(B_DQE), t & 1, bar(B_OF + so1), po1, abort_flag, prm.err, prm.wait_limit);
@@ -310,14 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + kTS + 64 * w, tP = tmem + lane_off + kTX + 64 * w;
     // this thread's row of dS^T: 128 bytes in the warpgroup's 64-query half
-    const uint32_t ds_row = sb + kOffS + w * 16384 + row * 128;
+    const uint32_t ds_row0 = sb + kOffS + w * 16384 + row * 128;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int e = t / nqt, i0 = (qt0 + t - e * nqt) * kBQ + 64 * w;  // this warpgroup's first query row
       const int sq = t % kQStages;
       const float *lsm = reinterpret_cast<const float *>(smem + kOffLse + sq * kBQ * 4) + 64 * w;
-      // D of this warpgroup's 64 query rows (the statistics kernel's padded array)
-      const float4 *d4 = reinterpret_cast<const float4 *>(prm.Dv + (long long)(qh_base + e) * prm.n_pad + i0);
+      // D of this warpgroup's 64 query rows, staged with the Q tile
+      const float4 *d4 = reinterpret_cast<const float4 *>(smem + kOffD + sq * kBQ * 4) + 16 * w;
       // P^T over this warpgroup's first 32 columns of S^T
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QF + sq), (t / kQStages) & 1, abort_flag, prm.err, prm.wait_limit) &&
                                        mbar_wait(bar(B_SF), t & 1, abort_flag, prm.err, prm.wait_limit));
@@ -364,17 +370,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t dd[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 4) {
-        const float4 dq4 = __ldg(d4 + (c >> 2));
+        const float4 dq4 = d4[c >> 2];
         dd[c >> 1] = pack_bf16x2(__uint_as_float(r[c]) * (__uint_as_float(dp[c]) - dq4.x),
                                  __uint_as_float(r[c + 1]) * (__uint_as_float(dp[c + 1]) - dq4.y));
         dd[(c >> 1) + 1] = pack_bf16x2(__uint_as_float(r[c + 2]) * (__uint_as_float(dp[c + 2]) - dq4.z),
                                        __uint_as_float(r[c + 3]) * (__uint_as_float(dp[c + 3]) - dq4.w));
       }
-      // the previous tile's dQ^T and dK MMAs have read the buffer
-      if (t > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSE), (t - 1) & 1, abort_flag, prm.err, prm.wait_limit));
+      // the dQ^T and dK MMAs of the tile two back have read this buffer
+      if (t >= kSStages) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSE + (t & 1)), ((t >> 1) - 1) & 1, abort_flag, prm.err,
+                                               prm.wait_limit));
         if (!ok) break;
       }
+      const uint32_t ds_row = ds_row0 + (uint32_t)(t & 1) * kTile;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         st_shared_v4(ds_row + ((uint32_t)(c ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2],

@@ -176,6 +176,14 @@ __device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, uint32_t sr
                "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
                : "memory");
 }
+// 3-D tiled reduce-add from shared memory into global memory (the element
+// type of the map, e.g. fp32 adds performed in L2), tracked like a store.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N of this thread's committed bulk groups still read
 // their shared-memory source (the buffers of the others may be refilled).
