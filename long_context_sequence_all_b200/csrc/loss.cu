@@ -12,7 +12,8 @@
 // lanes merge with shuffles.  Every CTA writes one (sum, count) partial for
 // its shard into the workspace.  Pass 2: one CTA per launch folds the
 // partials in a fixed order (deterministic) into S_r, C_r and L.
-// HBM-bound: each logits byte is read once.
+// HBM-bound: each logits byte is read once.  The grids are one wave of
+// resident CTAs.
 //
 // The gradient (the training step after the aggregation) has the global
 // count C = sum_r C_r as its only denominator:
@@ -32,6 +33,13 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kLoadsInFlight = 8;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (flush-to-zero; x <= 0 here).
+__device__ __forceinline__ float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ void merge(float &m, float &s, float m2, float s2) {
   // (m, s) represents sum exp(x - m) = s; combine two such pairs.
@@ -93,7 +101,7 @@ __device__ __forceinline__ float row_lse(const T *rowp, int vocab, int lane) {
         }
         const float ml = m * kLog2e;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s += exp2f(fmaf(x[e], kLog2e, -ml));
+        for (int e = 0; e < 8; ++e) s += ex2_mufu(fmaf(x[e], kLog2e, -ml));
       }
     }
   }
@@ -213,20 +221,34 @@ __global__ void __launch_bounds__(kThreads) ce_fwd_bwd_kernel(
       acc += (double)lse - (double)static_cast<float>(rowp[y]);
       cnt += 1;
     }
-    // dL/dz = (exp(z - lse) - [v == y]) / C; the row is read again from L2
+    // dL/dz = (exp(z - lse) - [v == y]) / C; the row is read again from L2,
+    // eight 16-byte loads in flight per lane
     const float lse2 = lse * kLog2e;
     const uint4 *row = reinterpret_cast<const uint4 *>(rowp);
-    for (int v = lane; v < vecs; v += 32) {
-      float x[8];
-      load_vals<T>(__ldg(row + v), x);
+    const int yv = y / kPerVec;
+    for (int v0 = lane; v0 < vecs; v0 += 32 * kLoadsInFlight) {
+      uint4 u[kLoadsInFlight];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int col = v * kPerVec + e;
-        float gv = exp2f(fmaf(x[e], kLog2e, -lse2)) * invC;
-        if (col == y) gv -= invC;
-        x[e] = gv;
+      for (int k = 0; k < kLoadsInFlight; ++k) {
+        const int v = v0 + k * 32;
+        if (v < vecs) u[k] = __ldg(row + v);
       }
-      __stcs(drow + v, pack_vals<T>(x));
+#pragma unroll
+      for (int k = 0; k < kLoadsInFlight; ++k) {
+        const int v = v0 + k * 32;
+        if (v < vecs) {
+          float x[8];
+          load_vals<T>(u[k], x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = ex2_mufu(fmaf(x[e], kLog2e, -lse2)) * invC;
+          if (v == yv) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (v * kPerVec + e == y) x[e] -= invC;
+          }
+          __stcs(drow + v, pack_vals<T>(x));
+        }
+      }
     }
   }
   __shared__ double sh_sum[kWarps];
@@ -269,15 +291,43 @@ __global__ void __launch_bounds__(256) ce_finalize_kernel(
   }
 }
 
+// CTAs of `kernel` (kThreads threads, no dynamic shared memory) resident on
+// the current device at once: its SMs times the occupancy (cached per device).
+template <typename Kernel>
+int resident_ctas(Kernel kernel) {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess || sms <= 0 ||
+      per_sm <= 0)
+    return 148;
+  const int n = sms * per_sm;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
 }  // namespace
 
 int loss_blocks_per_shard(int P, long long per_shard) {
-  // about four CTAs per SM in total, at most one warp per token
+  // the workspace bound: about four CTAs per SM in total, at most one warp per token
   long long nb = (4LL * 148 + P - 1) / P;
   long long need = (per_shard + kWarps - 1) / kWarps;
   if (nb > need) nb = need;
   if (nb < 1) nb = 1;
   return (int)nb;
+}
+
+// The CTAs of one launch: one wave of resident CTAs split over the P shards
+// (each CTA's tokens are fixed by the grid stride, so a partial second wave
+// would run on a fraction of the SMs), within the workspace bound.
+static int launch_blocks_per_shard(int P, long long per_shard, int resident) {
+  long long nb = resident / P;
+  if (nb < 1) nb = 1;
+  const int bound = loss_blocks_per_shard(P, per_shard);
+  return (int)(nb < bound ? nb : bound);
 }
 
 size_t loss_workspace_bytes(int P, long long per_shard) {
@@ -303,9 +353,11 @@ uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, 
                        const int32_t *labels, int32_t ignore_index, float *shard_sum,
                        int64_t *shard_count, float *loss, void *ws, cudaStream_t stream) {
   const long long per = tokens / P;
-  const int nb = loss_blocks_per_shard(P, per);
+  const int nb_ws = loss_blocks_per_shard(P, per);   // the workspace layout
+  const int nb = launch_blocks_per_shard(
+      P, per, dtype == ULY_BF16 ? resident_ctas(ce_partial_kernel<__nv_bfloat16>) : resident_ctas(ce_partial_kernel<float>));
   double *psum = static_cast<double *>(ws);
-  long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb * P);
+  long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb_ws * P);
   dim3 grid(nb, P);
   prof::Scope s1(prof::K_LOSS_PARTIAL, stream);
   if (dtype == ULY_BF16)
@@ -333,9 +385,11 @@ uly_status loss_bwd_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dty
                            const int32_t *labels, int32_t ignore_index, void *dlogits, float *shard_sum,
                            int64_t *shard_count, float *loss, void *ws, cudaStream_t stream) {
   const long long per = tokens / P;
-  const int nb = loss_blocks_per_shard(P, per);
+  const int nb_ws = loss_blocks_per_shard(P, per);   // the workspace layout
+  const int nb = launch_blocks_per_shard(
+      P, per, dtype == ULY_BF16 ? resident_ctas(ce_fwd_bwd_kernel<__nv_bfloat16>) : resident_ctas(ce_fwd_bwd_kernel<float>));
   double *psum = static_cast<double *>(ws);
-  long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb * P);
+  long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb_ws * P);
   long long *count = reinterpret_cast<long long *>(static_cast<char *>(ws) +
                                                    ((loss_workspace_bytes(P, per) + 15) & ~size_t(15)));
   dim3 grid(nb, P);
