@@ -332,6 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
       uint32_t r[64];
       tmem_ld64(tS, r);
+      // masked scores become -inf (exponential 0) before the exponentials, so
+      // that their loop has no branch and its MUFU latencies overlap freely
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (i0 + c < lo_j || i0 + c > hi_j) r[c] = __float_as_uint(-INFINITY);
+      }
       uint32_t pp[32];
       // LSE log2(e) of the 64 query rows: one broadcast 16-byte shared-memory
       // load per 4 columns
@@ -339,17 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 64; c += 4) {
         const float4 L = l4[c >> 2];
-        float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -L.x));
-        float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), prm.scale_log2, -L.y));
-        float p2 = ex2_approx(fmaf(__uint_as_float(r[c + 2]), prm.scale_log2, -L.z));
-        float p3 = ex2_approx(fmaf(__uint_as_float(r[c + 3]), prm.scale_log2, -L.w));
-        if (!full) {
-          const int i = i0 + c;
-          if (i < lo_j || i > hi_j) p0 = 0.f;
-          if (i + 1 < lo_j || i + 1 > hi_j) p1 = 0.f;
-          if (i + 2 < lo_j || i + 2 > hi_j) p2 = 0.f;
-          if (i + 3 < lo_j || i + 3 > hi_j) p3 = 0.f;
-        }
+        const float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -L.x));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), prm.scale_log2, -L.y));
+        const float p2 = ex2_approx(fmaf(__uint_as_float(r[c + 2]), prm.scale_log2, -L.z));
+        const float p3 = ex2_approx(fmaf(__uint_as_float(r[c + 3]), prm.scale_log2, -L.w));
         r[c] = __float_as_uint(p0);
         r[c + 1] = __float_as_uint(p1);
         r[c + 2] = __float_as_uint(p2);

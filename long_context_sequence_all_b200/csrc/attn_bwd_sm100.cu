@@ -67,7 +67,8 @@ struct BwdParams {
 };
 
 // D_i = <dO_i, O_i> and LSE_i log2(e) of every query row (two rows per warp,
-// 16-byte loads), written to the padded per-head arrays; rows n..n_pad-1 get 0.
+// 16-byte loads), written to the padded per-head arrays; rows n..n_pad-1 get 0,
+// rows that see no key an LSE of +inf.
 // dq_acc (fused backward only, else null): the row's 128 fp32 dQ accumulators
 // are zeroed here, so the fused kernel finds them cleared.
 // O is read in the head layout, or in the seq layout when g.out_seq (the
@@ -107,7 +108,10 @@ __global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const __nv_bfloat16
   for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (l == 0 && r < rows_pad) {
     Dpad[r] = acc;
-    L2pad[r] = valid ? __ldg(lse + h * n + i) * kLog2e : 0.f;
+    // a row that sees no key (forward LSE -inf) gets +inf: every exponential
+    // of the row, masked or not, is then exactly 0
+    const float lv = valid ? __ldg(lse + h * n + i) : 0.f;
+    L2pad[r] = valid ? (lv == -INFINITY ? INFINITY : lv * kLog2e) : 0.f;
   }
 }
 
@@ -349,18 +353,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (i0 >= n0 + kBN - 1) && (i0 + 63 <= hi_a) && (i0 + 64 <= g.n) && (n0 + kBN <= g.n);
       uint32_t r[64];
       tmem_ld64(tS, r);
+      // masked scores become -inf (exponential 0): the exponential loop has no branch
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (i0 + c < lo_j || i0 + c > hi_j) r[c] = __float_as_uint(-INFINITY);
+      }
       uint32_t pp[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          float pv = ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lsm[c + u]));
-          if (!full) {
-            const int i = i0 + c + u;
-            if (i < lo_j || i > hi_j) pv = 0.f;
-          }
-          r[c + u] = __float_as_uint(pv);
-        }
+        for (int u = 0; u < 2; ++u)
+          r[c + u] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[c + u]), prm.scale_log2, -lsm[c + u])));
         pp[c >> 1] = pack_bf16x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
       }
       tmem_st32_nowait(tS, pp);
@@ -624,15 +628,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_SR));                  // the MMA thread may now overwrite S
       const int n0 = (jt0 + j) * kBK + 64 * w;
       const bool full = (n0 >= lo_last) && (n0 + 63 <= hi_first) && (n0 + 64 <= g.n);
+      // masked scores become -inf (exponential 0): the exponential loop has no branch
+      if (!full) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float pv = ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lse2));
-        if (!full) {
-          const int jj = n0 + c;
-          if (jj < lo_i || jj > hi_i) pv = 0.f;
-        }
-        r[c] = __float_as_uint(pv);
+        for (int c = 0; c < 64; ++c)
+          if (n0 + c < lo_i || n0 + c > hi_i) r[c] = __float_as_uint(-INFINITY);
       }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) r[c] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[c]), prm.scale_log2, -lse2)));
       // phase b: dS over this warpgroup's first 32 columns of dP
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPF), j & 1, abort_flag, prm.err, prm.wait_limit));
       if (!ok) break;
