@@ -32,6 +32,10 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kLoadsInFlight = 8;
+// The gradient pass keeps fewer loads in flight (its row comes from L2), so
+// that the fused kernel fits three CTAs per SM like the partials kernel and
+// both entry points share one grid.
+constexpr int kGradLoads = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // 2^x on the special-function unit (flush-to-zero; x <= 0 here).
@@ -192,7 +196,7 @@ __device__ __forceinline__ uint4 pack_vals<float>(const float (&x)[8]) {
 
 // Loss partials as ce_partial_kernel, and dL/dz for every token of the shard.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) ce_fwd_bwd_kernel(
+__global__ void __launch_bounds__(kThreads, 3) ce_fwd_bwd_kernel(
     const T *__restrict__ logits, const int32_t *__restrict__ labels, long long per_shard, int vocab,
     int ignore_index, const long long *__restrict__ count, T *__restrict__ dlogits,
     double *__restrict__ part_sum, long long *__restrict__ part_cnt, int *err) {
@@ -222,19 +226,19 @@ __global__ void __launch_bounds__(kThreads) ce_fwd_bwd_kernel(
       cnt += 1;
     }
     // dL/dz = (exp(z - lse) - [v == y]) / C; the row is read again from L2,
-    // eight 16-byte loads in flight per lane
+    // four 16-byte loads in flight per lane
     const float lse2 = lse * kLog2e;
     const uint4 *row = reinterpret_cast<const uint4 *>(rowp);
     const int yv = y / kPerVec;
-    for (int v0 = lane; v0 < vecs; v0 += 32 * kLoadsInFlight) {
-      uint4 u[kLoadsInFlight];
+    for (int v0 = lane; v0 < vecs; v0 += 32 * kGradLoads) {
+      uint4 u[kGradLoads];
 #pragma unroll
-      for (int k = 0; k < kLoadsInFlight; ++k) {
+      for (int k = 0; k < kGradLoads; ++k) {
         const int v = v0 + k * 32;
         if (v < vecs) u[k] = __ldg(row + v);
       }
 #pragma unroll
-      for (int k = 0; k < kLoadsInFlight; ++k) {
+      for (int k = 0; k < kGradLoads; ++k) {
         const int v = v0 + k * 32;
         if (v < vecs) {
           float x[8];
@@ -330,6 +334,18 @@ static int launch_blocks_per_shard(int P, long long per_shard, int resident) {
   return (int)(nb < bound ? nb : bound);
 }
 
+// The grid of both loss entry points (the forward partials and the fused
+// gradient): the same CTAs over the same tokens, so that their per-CTA
+// partial sums, and so S_r, C_r and L, are equal bit for bit.  One wave of
+// whichever of the two kernels has the lower occupancy.
+static int loss_grid_blocks(int P, long long per_shard, int dtype) {
+  const int a = dtype == ULY_BF16 ? resident_ctas(ce_partial_kernel<__nv_bfloat16>)
+                                  : resident_ctas(ce_partial_kernel<float>);
+  const int b = dtype == ULY_BF16 ? resident_ctas(ce_fwd_bwd_kernel<__nv_bfloat16>)
+                                  : resident_ctas(ce_fwd_bwd_kernel<float>);
+  return launch_blocks_per_shard(P, per_shard, a < b ? a : b);
+}
+
 size_t loss_workspace_bytes(int P, long long per_shard) {
   const size_t nb = (size_t)loss_blocks_per_shard(P, per_shard);
   return nb * (size_t)P * (sizeof(double) + sizeof(long long));
@@ -354,8 +370,7 @@ uly_status loss_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dtype, 
                        int64_t *shard_count, float *loss, void *ws, cudaStream_t stream) {
   const long long per = tokens / P;
   const int nb_ws = loss_blocks_per_shard(P, per);   // the workspace layout
-  const int nb = launch_blocks_per_shard(
-      P, per, dtype == ULY_BF16 ? resident_ctas(ce_partial_kernel<__nv_bfloat16>) : resident_ctas(ce_partial_kernel<float>));
+  const int nb = loss_grid_blocks(P, per, dtype);
   double *psum = static_cast<double *>(ws);
   long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb_ws * P);
   dim3 grid(nb, P);
@@ -386,8 +401,7 @@ uly_status loss_bwd_launch(int32_t P, int64_t tokens, int32_t vocab, int32_t dty
                            int64_t *shard_count, float *loss, void *ws, cudaStream_t stream) {
   const long long per = tokens / P;
   const int nb_ws = loss_blocks_per_shard(P, per);   // the workspace layout
-  const int nb = launch_blocks_per_shard(
-      P, per, dtype == ULY_BF16 ? resident_ctas(ce_fwd_bwd_kernel<__nv_bfloat16>) : resident_ctas(ce_fwd_bwd_kernel<float>));
+  const int nb = loss_grid_blocks(P, per, dtype);
   double *psum = static_cast<double *>(ws);
   long long *pcnt = reinterpret_cast<long long *>(psum + (size_t)nb_ws * P);
   long long *count = reinterpret_cast<long long *>(static_cast<char *>(ws) +
