@@ -64,6 +64,7 @@ constexpr int kBQ = 128;   // query rows per tile
 // written while the previous tile's dQ^T and dK MMAs still read theirs.
 constexpr int kQStages = 2, kOStages = 1, kSStages = 2;
 static_assert(kSStages == 2, "the dS^T buffer of tile t is t & 1");
+constexpr int kPrefetchAhead = 2;
 constexpr uint32_t kTile = 128 * 128 * 2;                // one 128 x 128 bf16 tile
 constexpr uint32_t kOffK = 0, kOffV = kTile;
 constexpr uint32_t kOffQ = 2 * kTile;                    // Q stage s at kOffQ + s * kTile
@@ -187,6 +188,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(sb + kOffLse + sq * kBQ * 4, prm.lse2 + srow, kBQ * 4, bar(B_QF + sq));
           bulk_load(sb + kOffD + sq * kBQ * 4, prm.Dv + srow, kBQ * 4, bar(B_QF + sq));
           issued_q = t + 1;
+          // the Q and dO tiles kPrefetchAhead tiles on, into L2 (their loads
+          // otherwise wait on L2 misses behind the dQ reduce-adds)
+          if (kPrefetchAhead > 0 && t + kPrefetchAhead < T) {
+            const int tp = t + kPrefetchAhead, ep = tp / nqt, ip = (qt0 + tp - ep * nqt) * kBQ;
+            for (int c = 0; c < 2; ++c) {
+              tma_prefetch_l2_3d(&tmQ, c * 64, ip, qh_base + ep);
+              tma_prefetch_l2_3d(&tmO, c * 64, ip, qh_base + ep);
+            }
+          }
           const int so = t % kOStages, uo = t / kOStages;
           if (uo > 0 && !mbar_wait(bar(B_OE + so), (uo - 1) & 1, abort_flag, prm.err, prm.wait_limit)) break;
           mbar_arrive_expect_tx(bar(B_OF + so), kTile);

@@ -130,6 +130,14 @@ __device__ __forceinline__ bool mbar_wait2(uint32_t bar_a, uint32_t parity_a, ui
 }
 
 // ---------------------------------------------------------------------- TMA
+// Bring a 3-D tile of a tensor map into L2 ahead of its load (no shared
+// memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
