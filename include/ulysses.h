@@ -292,8 +292,9 @@ uly_status ulysses_o_proj_bwd(int32_t batch, int32_t seq_len, int32_t world, int
  * Local attention (step 4) of every logical rank, head layout in and out:
  * q, o [P][B][H/P][n][d]; k, v [P][B][G/P][n][d]; lse [P][B][H/P][n] (fp32).
  * O = softmax(scale * Q K^T + mask) V per query head, LSE its log-sum-exp.
- * bf16: tensor-core path (fp32 accumulation), needs head_dim == 128 and an
- * even number of query heads per KV head.  f32: exact-fp32 SIMT path.
+ * bf16: tensor-core path (fp32 accumulation), needs head_dim == 128; any
+ * group size H/G (an odd one, MHA included, runs one query head per CTA of the
+ * forward instead of two, at about half its rate).  f32: exact-fp32 SIMT path.
  */
 uly_status ulysses_attn_fwd(const uly_attn_desc *desc, const void *q, const void *k,
                             const void *v, void *o, float *lse, void *stream);

@@ -53,6 +53,7 @@ def _check_register_split(src: str, ptxas_log: str):
     lines = ptxas_log.splitlines()
     for kernel, want in REGISTER_SPLIT_KERNELS[src]:
         found = False
+        # every instance of the kernel (template instantiations included)
         for i, line in enumerate(lines):
             if "Compiling entry function" in line and kernel in line:
                 for nxt in lines[i + 1:i + 6]:
@@ -63,8 +64,6 @@ def _check_register_split(src: str, ptxas_log: str):
                                                f"split needs exactly {want}; refusing to build")
                         found = True
                         break
-            if found:
-                break
         if not found:
             raise RuntimeError(f"ptxas report for {kernel} not found; refusing to build")
 

@@ -108,8 +108,7 @@ uly_status check_desc(const uly_attn_desc *d, HeadGeom &g, MaskInfo &mk) {
   const long long heads_q = (long long)d->batch * d->n_q_heads;
   if (heads_q > 65535 || (d->seq_len + 63) / 64 > 65535) return ULY_ERR_SHAPE;  // grid limits
   if (d->dtype == ULY_F32 && d->head_dim != 64 && d->head_dim != 128) return ULY_ERR_UNSUPPORTED;
-  if (d->dtype == ULY_BF16 && (d->head_dim != 128 || (d->n_q_heads / d->n_kv_heads) % 2 != 0))
-    return ULY_ERR_UNSUPPORTED;
+  if (d->dtype == ULY_BF16 && d->head_dim != 128) return ULY_ERR_UNSUPPORTED;
   g.B = d->batch;
   g.n = d->seq_len;
   g.P = d->world;

@@ -6,7 +6,9 @@
 //
 // One CTA = two 128-row query tiles at the same positions m0..m0+127 of two
 // query heads of one GQA group, so both tiles read the same K/V tiles and see
-// the same mask: K/V are loaded once for 256 query rows.
+// the same mask: K/V are loaded once for 256 query rows.  When a group has an
+// odd number of query heads (MHA: one) the CTA takes one query head: the
+// second tile's MMAs and softmax warpgroup are skipped.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q tiles once, then K_j, V_j into a 5-slot ring
@@ -68,6 +70,7 @@ struct FwdParams {
   long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
 };
 
+template <int NTILE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -86,11 +89,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = g.hl >> 1;
-  const int pair = blockIdx.x;                   // (r*B + b) * (hl/2) + pp
-  const int rb = pair / half, pp = pair - rb * half;
-  const int qhead0 = rb * g.hl + 2 * pp;         // tiles: qhead0, qhead0 + 1
-  const int kvhead = rb * g.gl + (2 * pp) / g.group;
+  constexpr int ntile = NTILE;                   // query tiles (heads) per CTA: 2, or 1 for an odd group
+  const int per = g.hl / ntile;
+  const int rb = blockIdx.x / per, pp = blockIdx.x - rb * per;   // blockIdx.x = (r*B + b) * per + pp
+  const int qhead0 = rb * g.hl + ntile * pp;     // tiles: qhead0 (, qhead0 + 1)
+  const int kvhead = rb * g.gl + (ntile * pp) / g.group;
   const int mt = gridDim.y - 1 - blockIdx.y;     // heaviest (latest) query tiles first
   const int m0 = mt * kBM;
 
@@ -129,8 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0 && NT > 0) {
-      mbar_arrive_expect_tx(bar(B_Q), 2 * kTileBytes);
-      for (int t = 0; t < 2; ++t)
+      mbar_arrive_expect_tx(bar(B_Q), ntile * kTileBytes);
+      for (int t = 0; t < ntile; ++t)
         for (int c = 0; c < 2; ++c)
           tma_load_3d(sb + kOffQ + t * kTileBytes + c * 16384, &tmQ, bar(B_Q), c * 64, m0, qhead0 + t);
       int issued = 0;
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       : mbar_wait(bar(B_KVF + slotK), parK, abort_flag, prm.err, prm.wait_limit);
         if (!ok) break;
         tc_fence_after();
-        for (int t = 0; t < 2 && ok; ++t) {
+        for (int t = 0; t < ntile && ok; ++t) {
           if (it > 0) {
             // the first half of P V starts while the softmax still computes the second
             for (int h = 0; h < 2 && ok; ++h) {
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dv = sdesc_sw128(sb + kOffKV + slotV * kTileBytes, 16384, 1024);
         ok = mbar_wait(bar(B_KVF + slotV), parV, abort_flag, prm.err, prm.wait_limit);
         tc_fence_after();
-        for (int t = 0; t < 2 && ok; ++t) {
+        for (int t = 0; t < ntile && ok; ++t) {
           for (int h = 0; h < 2 && ok; ++h) {
             ok = mbar_wait(bar(B_PF + 2 * t + h), (NT - 1) & 1, abort_flag, prm.err, prm.wait_limit);
             if (!ok) break;
@@ -239,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int wg = (warp - 4) >> 2;        // query tile 0 or 1
+    if (wg < ntile) {
     const int wq = warp & 3;               // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;
     const int i = m0 + row;
@@ -354,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (valid && (ok || NT == 0))
       prm.lse[hrow] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+    }
   }
 
   tc_fence_before();
@@ -403,8 +408,11 @@ uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
       !make_tmap_heads_bf16(&tk, k, kHD, g.n, kvheads, 128) ||
       !make_tmap_heads_bf16(&tv, v, kHD, g.n, kvheads, 128))
     return ULY_ERR_CUDA;
-  static std::atomic<uint64_t> optin_devices{0};
-  if (!smem_optin(attn_fwd_sm100_kernel, kSmemBytes, optin_devices)) return ULY_ERR_CUDA;
+  static std::atomic<uint64_t> optin_devices{0}, optin_devices1{0};
+  const int ntile = (g.group & 1) ? 1 : 2;   // two query heads per CTA need an even group
+  if (ntile == 2 ? !smem_optin(attn_fwd_sm100_kernel<2>, kSmemBytes, optin_devices)
+                 : !smem_optin(attn_fwd_sm100_kernel<1>, kSmemBytes, optin_devices1))
+    return ULY_ERR_CUDA;
   FwdParams prm;
   prm.o = static_cast<__nv_bfloat16 *>(o);
   prm.lse = lse;
@@ -413,9 +421,12 @@ uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.scale_log2 = g.scale * kLog2e;
   prm.err = error_word();
   prm.wait_limit = wait_limit_cycles();
-  dim3 grid(g.P * g.B * (g.hl / 2), (g.n + kBM - 1) / kBM);
+  dim3 grid(g.P * g.B * (g.hl / ntile), (g.n + kBM - 1) / kBM);
   prof::Scope scope(prof::K_ATTN_FWD_SM100, stream);
-  attn_fwd_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);
+  if (ntile == 2)
+    attn_fwd_sm100_kernel<2><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);
+  else
+    attn_fwd_sm100_kernel<1><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);
   note_launches(1);
   return last_launch_status();
 }

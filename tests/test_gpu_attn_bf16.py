@@ -62,6 +62,10 @@ def _lse_nat(lse_head, B, H, n):
     (640, 2, 8, 2, U.MASK_CAUSAL, 3.0),            # peaked softmax: running-max rescales
     (128, 4, 16, 4, U.MASK_CAUSAL, 1.0),           # a single tile, P = 4 with 4-way GQA
     (8, 8, 16, 8, U.MASK_CAUSAL, 1.0),             # one token per rank
+    (424, 4, 4, 4, U.MASK_CAUSAL, 128 ** -0.5),    # MHA (G = H): one query head per CTA, ragged tail
+    (392, 4, 8, 8, U.MASK_NONE, 128 ** -0.5),      # MHA, non-causal
+    (1000, 4, 8, 8, U.MASK_DOC_CAUSAL, 128 ** -0.5),   # MHA, documents
+    (424, 2, 6, 2, U.MASK_CAUSAL, 1.0),            # an odd group (3 query heads per KV head)
 ])
 def test_fwd_small_elementwise(n, P, H, G, mask, std):
     q, k, v, _ = _rand_case(n, P, H, G, std=std, seed=n)
@@ -74,14 +78,6 @@ def test_fwd_small_elementwise(n, P, H, G, mask, std):
     assert_bf16_close(o.cpu(), o_ref, "O", max_abs_tol=_abs_tol(std, o_ref))
     assert max_abs(lse.cpu(), lse_ref) <= LSE_BF16_MAX_ABS
     assert U.ulysses_read_error() == 0
-
-
-def test_fwd_rejects_odd_group():
-    q, k, v, _ = _rand_case(256, 4, 4, 4)
-    qh, kh, vh = (U.ulysses_seq_to_head(x.cuda(), 4) for x in (q, k, v))
-    with pytest.raises(U.UlyssesError) as e:
-        U.ulysses_attn_fwd(qh, kh, vh)
-    assert e.value.status == 6
 
 
 def _check_sampled_fwd(inp, o_seq, lse_head, heads, rows):
@@ -142,6 +138,9 @@ def run_layer(q, k, v, do, P, mask, cu=None):
     (640, 2, 8, 2, U.MASK_CAUSAL, 1.0),
     (128, 4, 16, 4, U.MASK_CAUSAL, 1.0),
     (8, 8, 16, 8, U.MASK_CAUSAL, 1.0),
+    (424, 4, 4, 4, U.MASK_CAUSAL, 128 ** -0.5),    # MHA
+    (1000, 4, 8, 8, U.MASK_DOC_CAUSAL, 128 ** -0.5),
+    (424, 2, 6, 2, U.MASK_CAUSAL, 1.0),            # an odd group
 ])
 def test_bwd_small_elementwise(n, P, H, G, mask, std):
     q, k, v, do = _rand_case(n, P, H, G, std=std, seed=n + 1)

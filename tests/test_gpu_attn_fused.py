@@ -42,6 +42,8 @@ CASES = [
     (392, 4, 8, 4, U.MASK_NONE, None),
     (1000, 8, 16, 8, U.MASK_DOC_CAUSAL, [0, 100, 129, 400, 401, 777, 1000]),
     (8, 8, 16, 8, U.MASK_CAUSAL, None),         # one token per rank
+    (424, 4, 4, 4, U.MASK_CAUSAL, None),        # MHA (G = H)
+    (424, 2, 6, 2, U.MASK_CAUSAL, None),        # an odd group (3 query heads per KV head)
 ]
 
 
