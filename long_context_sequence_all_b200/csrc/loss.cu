@@ -75,6 +75,23 @@ __device__ __forceinline__ void load_vals<float>(const uint4 &u, float (&x)[8]) 
   x[4] = x[5] = x[6] = x[7] = -INFINITY;
 }
 
+// Largest of the values one 16-byte vector holds (bf16: packed maxima).
+template <typename T>
+__device__ __forceinline__ float vec_max(const uint4 &u);
+
+template <>
+__device__ __forceinline__ float vec_max<__nv_bfloat16>(const uint4 &u) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  const __nv_bfloat162 m = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+  const float2 f = __bfloat1622float2(m);
+  return fmaxf(f.x, f.y);
+}
+
+template <>
+__device__ __forceinline__ float vec_max<float>(const uint4 &u) {
+  return fmaxf(fmaxf(__uint_as_float(u.x), __uint_as_float(u.y)), fmaxf(__uint_as_float(u.z), __uint_as_float(u.w)));
+}
+
 // log sum_v exp(z_v) of one row, computed by the 32 lanes of a warp (every
 // lane returns it).  STREAM: evict-first loads (the row is not read again).
 template <typename T, bool STREAM>
@@ -90,24 +107,27 @@ __device__ __forceinline__ float row_lse(const T *rowp, int vocab, int lane) {
       const int v = v0 + k * 32;
       if (v < vecs) u[k] = STREAM ? __ldcs(row + v) : __ldg(row + v);
     }
+    // one maximum (and at most one rescale) per group of loaded vectors
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kLoadsInFlight; ++k)
+      if (v0 + k * 32 < vecs) mx = fmaxf(mx, vec_max<T>(u[k]));
+    if (mx > m) {
+      s = (m == -INFINITY) ? 0.f : s * exp2f((m - mx) * kLog2e);
+      m = mx;
+    }
+    const float ml = (m == -INFINITY) ? 0.f : m * kLog2e;   // all -inf so far: every term is 0
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};   // four add chains, folded in a fixed order
 #pragma unroll
     for (int k = 0; k < kLoadsInFlight; ++k) {
-      const int v = v0 + k * 32;
-      if (v < vecs) {
+      if (v0 + k * 32 < vecs) {
         float x[8];
         load_vals<T>(u[k], x);
-        float mx = x[0];
 #pragma unroll
-        for (int e = 1; e < 8; ++e) mx = fmaxf(mx, x[e]);
-        if (mx > m) {
-          s = (m == -INFINITY) ? 0.f : s * exp2f((m - mx) * kLog2e);
-          m = mx;
-        }
-        const float ml = m * kLog2e;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s += ex2_mufu(fmaf(x[e], kLog2e, -ml));
+        for (int e = 0; e < 8; ++e) s4[e & 3] += ex2_mufu(fmaf(x[e], kLog2e, -ml));
       }
     }
+    s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
