@@ -118,6 +118,8 @@ struct ProjParams {
   __nv_bfloat16 *c16;        // DX: bf16 C
   float *c32;                // DW / DWO: fp32 C
   long long M_rows;          // DX / DW / DWO: rows of C (rows past it are not stored)
+  int ksplit;                // DW / DWO: 1, or 2 = each tile's k-steps in two halves (work units),
+                             // added into a zeroed C with fp32 reduce-adds
   int *err;
   long long wait_limit;      // cycles a pipeline wait may last (wait_limit_cycles())
 };
@@ -151,6 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = prm.m_tiles * prm.n_tiles;
   const int KT = (prm.K + kBK - 1) / kBK;   // a ragged last k-step reads zeros past K
+  const int ks = prm.ksplit;                // work unit u: tile u / ks, k-steps of its part u % ks
+  const int nunits = ntiles * ks;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_ACCE || i == B_ACCE + 1) ? 128 : 1);
@@ -173,7 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       long long idx = 0;   // k-steps issued so far (ring position)
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+      for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        const int tile = u / ks, sp = u - tile * ks;
+        const int kt0 = (int)((long long)KT * sp / ks), kt1 = (int)((long long)KT * (sp + 1) / ks);
         const int mt = tile / prm.n_tiles, nt = tile - mt * prm.n_tiles;
         const int n0 = nt * kBN;
         int b = 0, t0 = 0;
@@ -181,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           b = mt / prm.tiles_per_b;
           t0 = (mt - b * prm.tiles_per_b) * kBM;
         }
-        for (int kt = 0; kt < KT; ++kt, ++idx) {
+        for (int kt = kt0; kt < kt1; ++kt, ++idx) {
           const int stage = (int)(idx % kStages);
           const long long use = idx / kStages;
           if (use > 0 && !mbar_wait(bar(B_EMPTY + stage), (uint32_t)((use - 1) & 1), abort_flag, prm.err, prm.wait_limit)) {
@@ -220,7 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long idx = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+      for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x, ++it) {
+        const int sp = u % ks;
+        const int kt0 = (int)((long long)KT * sp / ks), kt1 = (int)((long long)KT * (sp + 1) / ks);
         const int buf = it & 1;
         if (it >= 2) {
           ok = mbar_wait(bar(B_ACCE + buf), (uint32_t)(((it >> 1) - 1) & 1), abort_flag, prm.err, prm.wait_limit);
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         const uint32_t acc = tmem + buf * kBN;
-        for (int kt = 0; kt < KT; ++kt, ++idx) {
+        for (int kt = kt0; kt < kt1; ++kt, ++idx) {
           const int stage = (int)(idx % kStages);
           const uint32_t sA = sb + stage * kStageBytes, sB = sA + kABytes;
           // K-major: 16 K-elements are 32 bytes along a row; MN-major: 16 K-rows
@@ -243,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             mma_bf16_ss(acc, sdesc_add(da, kk * astep), sdesc_add(db, kk * bstep), idesc,
-                        (kt > 0 || kk > 0) ? 1u : 0u);
+                        (kt > kt0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(B_EMPTY + stage));
         }
         if (!ok) break;
@@ -259,7 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     int it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+      const int tile = u / ks;
       const int buf = it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ACCF + buf), (uint32_t)((it >> 1) & 1), abort_flag, prm.err, prm.wait_limit)))
         break;
@@ -281,12 +290,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(a[e]);
               store_row_chunk(prm.c16 + c0 + c, x);
-            } else {
+            } else if (ks == 1) {
               float4 *d4 = reinterpret_cast<float4 *>(prm.c32 + c0 + c);
 #pragma unroll
-              for (int u = 0; u < 8; ++u)
-                d4[u] = make_float4(__uint_as_float(a[4 * u]), __uint_as_float(a[4 * u + 1]),
-                                    __uint_as_float(a[4 * u + 2]), __uint_as_float(a[4 * u + 3]));
+              for (int q = 0; q < 8; ++q)
+                d4[q] = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                    __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+            } else {
+              // the tile's two halves meet in L2; with two partials added
+              // into zero, either order gives the same bits
+              float4 *d4 = reinterpret_cast<float4 *>(prm.c32 + c0 + c);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                atomicAdd(d4 + q, make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                              __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3])));
             }
           }
         }
@@ -455,8 +472,10 @@ __global__ void __launch_bounds__(256) qkv_dy_kernel(const __nv_bfloat16 *__rest
   }
 }
 
-uly_status launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const ProjParams &prm, int kernel_id,
+uly_status launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const ProjParams &prm_in, int kernel_id,
                        cudaStream_t stream) {
+  ProjParams prm = prm_in;
+  prm.ksplit = 1;
   // the shared-memory opt-in is a per-device attribute: set it once on every
   // device this process launches on
   static std::atomic<uint64_t> attr_devices{0};
@@ -471,9 +490,20 @@ uly_status launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const ProjP
       return ULY_ERR_CUDA;
     attr_devices.fetch_or(bit, std::memory_order_acq_rel);
   }
+  // The weight gradients contract over every token (long k loops) into few
+  // output tiles: when halving each tile's k-steps fills the last wave of the
+  // persistent grid better, a work unit is half a tile, added into a zeroed C.
   const int ntiles = prm.m_tiles * prm.n_tiles;
-  const int grid = ntiles < sms ? ntiles : sms;
-  prof::Scope scope(kernel_id, stream);
+  if ((prm.mode == MODE_DW || prm.mode == MODE_DWO) && (prm.K + kBK - 1) / kBK >= 64) {
+    auto fill = [&](int units) { return (double)units / ((double)((units + sms - 1) / sms) * sms); };
+    if (fill(2 * ntiles) > fill(ntiles) + 0.02) prm.ksplit = 2;
+  }
+  const int nunits = ntiles * prm.ksplit;
+  const int grid = nunits < sms ? nunits : sms;
+  prof::Scope scope(kernel_id, stream);   // the zeroing of C is part of the timed entry point
+  if (prm.ksplit == 2 &&
+      cudaMemsetAsync(prm.c32, 0, (size_t)prm.M_rows * (size_t)prm.ldc * sizeof(float), stream) != cudaSuccess)
+    return ULY_ERR_CUDA;
   proj_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, prm);
   note_launches(1);
   return last_launch_status();

@@ -130,7 +130,10 @@ def test_qkv_projection_backward_qwen8k_shapes():
     dv = (torch.randn(P, B, G // P, n, d, generator=g) * 0.05).to(torch.bfloat16)
     tab = U.ulysses_rope_table(n, d, 1.0e6)
     dx, dw = U.ulysses_qkv_proj_rope_bwd(x.cuda(), w.cuda(), P, H, G, tab, dq.cuda(), dk.cuda(), dv.cuda())
+    dx2, dw2 = U.ulysses_qkv_proj_rope_bwd(x.cuda(), w.cuda(), P, H, G, tab, dq.cuda(), dk.cuda(), dv.cuda())
     torch.cuda.synchronize()
+    # dW's 480 tiles run as two k-halves each, added into a zeroed dW: still the same bits every call
+    assert torch.equal(dw, dw2) and torch.equal(dx, dx2)
     dx_ref, dw_ref = oracle.qkv_proj_rope_bwd(f32_inputs(x), f32_inputs(w), f32_inputs(dq), f32_inputs(dk),
                                               f32_inputs(dv), P, H, G, d, 1.0e6)
     dy = np.abs(_dy_exact(dq, dk, dv, P, H, G, B, n))
@@ -139,4 +142,31 @@ def test_qkv_projection_backward_qwen8k_shapes():
     _assert_within(dx, dx_ref.reshape(M, hidden), bx, "dX 8K")
     bw = (HALF_ULP + M * U32) * (dy.T @ np.abs(x.double().numpy().reshape(M, hidden))) + 1e-6
     _assert_within(dw, dw_ref, bw, "dW 8K")
+    assert U.ulysses_read_error() == 0
+
+
+def test_output_projection_backward_qwen8k_shapes():
+    """Qwen3-4B shapes at 8K (hidden 2560, 32 query heads, P = 4): 320 output
+    tiles of dW_o over 128 k-steps, so each tile's contraction runs as two
+    halves added into a zeroed dW_o.  Every element of dO and dW_o against the
+    oracle, and two calls give the same bits."""
+    P, B, n, H, hidden, d = 4, 1, 8192, 32, 2560, 128
+    s = n // P
+    g = torch.Generator().manual_seed(8192 + hidden)
+    o_seq = torch.randn(P, B, s, H, d, generator=g).to(torch.bfloat16)
+    w_o = (torch.randn(hidden, H * d, generator=g) / (H * d) ** 0.5).to(torch.bfloat16)
+    dy = torch.randn(P, B, s, hidden, generator=g).to(torch.bfloat16)
+    do, dw_o = U.ulysses_o_proj_bwd(o_seq.cuda(), w_o.cuda(), dy.cuda(), P)
+    do2, dw_o2 = U.ulysses_o_proj_bwd(o_seq.cuda(), w_o.cuda(), dy.cuda(), P)
+    torch.cuda.synchronize()
+    assert torch.equal(dw_o, dw_o2) and torch.equal(do, do2)
+    o_head = oracle.seq_to_head(f32_inputs(o_seq), B, n, P, H)
+    do_ref, dwo_ref = oracle.o_proj_bwd(o_head, f32_inputs(w_o), f32_inputs(dy), P)
+    M = P * B * s
+    dya = np.abs(dy.double().numpy().reshape(M, hidden))
+    prod = (dya @ np.abs(w_o.double().numpy())).reshape(P, B, s, H, d)
+    prod_head = oracle.seq_to_head(prod, B, n, P, H)
+    _assert_within(do, do_ref, HALF_ULP * np.abs(do_ref) + hidden * U32 * prod_head + 1e-6, "dO 8K")
+    oa = np.abs(o_seq.double().numpy().reshape(M, H * d))
+    _assert_within(dw_o, dwo_ref, M * U32 * (dya.T @ oa) + 1e-6, "dW_o 8K")
     assert U.ulysses_read_error() == 0
