@@ -420,55 +420,77 @@ __global__ void rope_table_kernel(int max_pos, int half, double base, float *tab
 // j's gradient row comes from the head layout (the inverse of the folded
 // all-to-all) and, for query and key heads, is rotated back by -pos (the
 // transpose of the rotation: d1 = g1 cos + g2 sin, d2 = g2 cos - g1 sin for
-// the pair (e, e + 64)).  16 threads per row, 4 pairs each; HBM-bound.
-__global__ void __launch_bounds__(256) qkv_dy_kernel(const __nv_bfloat16 *__restrict__ dq,
-                                                     const __nv_bfloat16 *__restrict__ dk,
-                                                     const __nv_bfloat16 *__restrict__ dv,
-                                                     const float4 *__restrict__ rope, int max_pos,
-                                                     const int32_t *__restrict__ positions,
-                                                     __nv_bfloat16 *__restrict__ dy, int B, int n, int s, int H,
-                                                     int G, int hl, int gl, long long rows, int *err) {
-  const int l = threadIdx.x & 15;
+// the pair (e, e + 64)).  8 threads per row, 8 pairs each; HBM-bound.
+__global__ void __launch_bounds__(512) qkv_dy_kernel(const __nv_bfloat16 *__restrict__ dq,
+                                                      const __nv_bfloat16 *__restrict__ dk,
+                                                      const __nv_bfloat16 *__restrict__ dv,
+                                                      const float4 *__restrict__ rope, int max_pos,
+                                                      const int32_t *__restrict__ positions,
+                                                      __nv_bfloat16 *__restrict__ dy, int B, int n, int s, int H,
+                                                      int G, int hl, int gl, long long M, int *err) {
+  // eight threads per output row (one head of one token): thread l moves the
+  // elements [8l, 8l + 8) and [64 + 8l, 64 + 8l + 8) as 16-byte vectors, so it
+  // holds the rotary pairs (e, e + 64) it rotates.  Two tokens per iteration,
+  // all their loads issued before any arithmetic.
+  constexpr int kTok = 2;
+  const int l = threadIdx.x & 7, grp = threadIdx.x >> 3, ngrp = blockDim.x >> 3;
   const int J = H + 2 * G;
-  for (long long R = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4; R < rows;
-       R += ((long long)gridDim.x * blockDim.x) >> 4) {
-    const long long m = R / J;
-    const int j = (int)(R - m * J);
-    const long long bs = (long long)B * s;
-    const int r = (int)(m / bs);
-    const long long rem = m - (long long)r * bs;
-    const int b = (int)(rem / s), tt = (int)(rem - (long long)b * s);
-    const int t = r * s + tt;
-    const __nv_bfloat16 *base;
-    int heads_local, jj;
-    if (j < H) { base = dq; heads_local = hl; jj = j; }
-    else if (j < H + G) { base = dk; heads_local = gl; jj = j - H; }
-    else { base = dv; heads_local = gl; jj = j - H - G; }
-    const int r2 = jj / heads_local, hh = jj - r2 * heads_local;
-    const __nv_bfloat16 *src = base + ((((long long)r2 * B + b) * heads_local + hh) * n + t) * kHD;
-    const uint2 a = __ldg(reinterpret_cast<const uint2 *>(src) + l);        // elements 4l .. 4l+3
-    const uint2 c = __ldg(reinterpret_cast<const uint2 *>(src + 64) + l);   // elements 64+4l ..
-    uint2 o1 = a, o2 = c;
-    if (j < H + G) {
-      int pos = positions ? __ldg(positions + (long long)b * n + t) : t;
+  const long long bs = (long long)B * s;
+  for (long long m0 = (long long)blockIdx.x * kTok; m0 < M; m0 += (long long)gridDim.x * kTok) {
+    int b_[kTok], t_[kTok];
+    float4 w[kTok][4];   // cos / sin of this thread's eight pairs (two per float4)
+#pragma unroll
+    for (int k = 0; k < kTok; ++k) {
+      const long long m = m0 + k < M ? m0 + k : m0;   // a past-the-end token repeats m0 (not stored)
+      const int r = (int)(m / bs);
+      const long long rem = m - (long long)r * bs;
+      b_[k] = (int)(rem / s);
+      t_[k] = r * s + (int)(rem - (long long)b_[k] * s);
+      int pos = positions ? __ldg(positions + (long long)b_[k] * n + t_[k]) : t_[k];
       if (pos < 0 || pos >= max_pos) {
-        if (l == 0) raise_error(err, ULY_ERR_SHAPE);
+        if (threadIdx.x == 0) raise_error(err, ULY_ERR_SHAPE);
         pos = 0;
       }
-      const float4 w0 = __ldg(rope + (long long)pos * (kHD / 4) + 2 * l);       // pairs 4l, 4l+1
-      const float4 w1 = __ldg(rope + (long long)pos * (kHD / 4) + 2 * l + 1);   // pairs 4l+2, 4l+3
-      const float2 g1a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a.x));
-      const float2 g1b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a.y));
-      const float2 g2a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&c.x));
-      const float2 g2b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&c.y));
-      o1.x = pack_bf16x2(g1a.x * w0.x + g2a.x * w0.y, g1a.y * w0.z + g2a.y * w0.w);
-      o2.x = pack_bf16x2(g2a.x * w0.x - g1a.x * w0.y, g2a.y * w0.z - g1a.y * w0.w);
-      o1.y = pack_bf16x2(g1b.x * w1.x + g2b.x * w1.y, g1b.y * w1.z + g2b.y * w1.w);
-      o2.y = pack_bf16x2(g2b.x * w1.x - g1b.x * w1.y, g2b.y * w1.z - g1b.y * w1.w);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[k][q] = __ldg(rope + (long long)pos * (kHD / 4) + 4 * l + q);
     }
-    __nv_bfloat16 *out = dy + R * kHD;
-    reinterpret_cast<uint2 *>(out)[l] = o1;
-    reinterpret_cast<uint2 *>(out + 64)[l] = o2;
+    for (int j = grp; j < J; j += ngrp) {
+      const __nv_bfloat16 *base;
+      int heads_local, jj;
+      if (j < H) { base = dq; heads_local = hl; jj = j; }
+      else if (j < H + G) { base = dk; heads_local = gl; jj = j - H; }
+      else { base = dv; heads_local = gl; jj = j - H - G; }
+      const int r2 = jj / heads_local, hh = jj - r2 * heads_local;
+      uint4 a[kTok], c[kTok];
+#pragma unroll
+      for (int k = 0; k < kTok; ++k) {
+        const __nv_bfloat16 *src = base + ((((long long)r2 * B + b_[k]) * heads_local + hh) * n + t_[k]) * kHD;
+        a[k] = __ldg(reinterpret_cast<const uint4 *>(src) + l);        // elements 8l .. 8l+7
+        c[k] = __ldg(reinterpret_cast<const uint4 *>(src + 64) + l);   // elements 64+8l ..
+      }
+#pragma unroll
+      for (int k = 0; k < kTok; ++k) {
+        if (m0 + k >= M) break;
+        uint4 o1 = a[k], o2 = c[k];
+        if (j < H + G) {
+          const uint32_t av[4] = {a[k].x, a[k].y, a[k].z, a[k].w}, cv[4] = {c[k].x, c[k].y, c[k].z, c[k].w};
+          uint32_t p1[4], p2[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {   // elements 8l + 2q, 8l + 2q + 1 and their partners + 64
+            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&av[q]));
+            const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&cv[q]));
+            const float4 wq = w[k][q];
+            p1[q] = pack_bf16x2(g1.x * wq.x + g2.x * wq.y, g1.y * wq.z + g2.y * wq.w);
+            p2[q] = pack_bf16x2(g2.x * wq.x - g1.x * wq.y, g2.y * wq.z - g1.y * wq.w);
+          }
+          o1 = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+          o2 = make_uint4(p2[0], p2[1], p2[2], p2[3]);
+        }
+        __nv_bfloat16 *out = dy + ((m0 + k) * J + j) * (long long)kHD;
+        reinterpret_cast<uint4 *>(out)[l] = o1;
+        reinterpret_cast<uint4 *>(out + 64)[l] = o2;
+      }
+    }
   }
 }
 
@@ -556,15 +578,24 @@ uly_status qkv_proj_bwd_launch(int32_t B, int32_t n, int32_t P, int32_t hidden, 
                                float *dw, void *dy, cudaStream_t stream) {
   const long long M = (long long)B * n;
   const long long N = (long long)(H + 2 * G) * kHD;
-  const long long rows = M * (H + 2 * G);
   {
-    long long blocks = (rows * 16 + 255) / 256;
-    if (blocks > 148LL * 16) blocks = 148LL * 16;
+    // eight threads per head of a token: one token per CTA iteration
+    const int J = H + 2 * G;
+    int threads = ((8 * J + 31) / 32) * 32;
+    if (threads > 512) threads = 512;   // more heads: a group takes several rows of a token
+    // one wave of resident CTAs (each CTA's tokens are fixed by the grid stride)
+    int per_sm = 0, dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qkv_dy_kernel, threads, 0) != cudaSuccess || per_sm < 1)
+      return ULY_ERR_CUDA;
+    long long blocks = (long long)sms * per_sm;
+    if (blocks > (M + 1) / 2) blocks = (M + 1) / 2;
+    if (blocks < 1) blocks = 1;
     prof::Scope scope(prof::K_QKV_DY, stream);
-    qkv_dy_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+    qkv_dy_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(dq), static_cast<const __nv_bfloat16 *>(dk),
         static_cast<const __nv_bfloat16 *>(dv), reinterpret_cast<const float4 *>(rope), max_pos, positions,
-        static_cast<__nv_bfloat16 *>(dy), B, n, n / P, H, G, H / P, G / P, rows, error_word());
+        static_cast<__nv_bfloat16 *>(dy), B, n, n / P, H, G, H / P, G / P, M, error_word());
     note_launches(1);
     if (last_launch_status() != ULY_OK) return ULY_ERR_CUDA;
   }
