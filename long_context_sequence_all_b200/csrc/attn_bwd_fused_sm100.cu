@@ -18,7 +18,8 @@
 //
 // Warp roles (512 threads):
 //   warp 0       TMA: K, V once; Q tiles (+ LSE log2 e and D of their rows)
-//                in two stages, dO tiles in one
+//                in two stages, dO tiles in one; the Q and dO tiles two steps
+//                ahead prefetched into L2
 //   warp 1       TMEM allocation and the MMA-issuing thread:
 //                  S^T  = K Q^T           (SS, M=128 keys, N=128 queries)
 //                  dP^T = V dO^T          (SS)

@@ -8,8 +8,9 @@
 //   L   = sum_r S_r / sum_r C_r
 //
 // Pass 1: one warp per token streams the token's logits row once (16-byte
-// loads, eight in flight per lane), keeping a running (max, sum) per lane;
-// lanes merge with shuffles.  Every CTA writes one (sum, count) partial for
+// loads, eight in flight per lane), keeping a running (max, sum) per lane
+// (the maximum taken, and the sum rescaled, once per group of eight loaded
+// vectors); lanes merge with shuffles.  Every CTA writes one (sum, count) partial for
 // its shard into the workspace.  Pass 2: one CTA per launch folds the
 // partials in a fixed order (deterministic) into S_r, C_r and L.
 // HBM-bound: each logits byte is read once.  The grids are one wave of
