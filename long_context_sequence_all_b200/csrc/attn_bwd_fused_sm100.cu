@@ -135,10 +135,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x;                    // (r*B + b)*gl + gg
+  // Blocks start in the order of their linear index (x fastest); that order
+  // walks the key tiles of one KV head at a time (earliest, so heaviest under
+  // a causal mask, first), so the CTAs in flight read the Q/dO rows and add
+  // into the dQ rows of one GQA group's heads, which stay in L2.
+  const int nk = gridDim.y;
+  const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+  const int kvh = lin / nk;                      // (r*B + b)*gl + gg
   const int rb = kvh / g.gl, gg = kvh - rb * g.gl;
   const int qh_base = rb * g.hl + gg * g.group;  // first query head of the group
-  const int n0 = blockIdx.y * kBN;
+  const int n0 = (lin - kvh * nk) * kBN;
 
   // query rows that see any of the keys [n0, n0+127]
   int lo_a, hi_a, lo_b, hi_b;

@@ -90,11 +90,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int ntile = NTILE;                   // query tiles (heads) per CTA: 2, or 1 for an odd group
-  const int per = g.hl / ntile;
-  const int rb = blockIdx.x / per, pp = blockIdx.x - rb * per;   // blockIdx.x = (r*B + b) * per + pp
+  // Blocks start in the order of their linear index (x fastest).  That
+  // order walks the CTAs of one KV head at a time (its gpp CTAs per query
+  // tile, heaviest query tiles first), so the CTAs in flight stream the K/V
+  // of one or two KV heads, which stay in L2, rather than of every head.
+  const int gpp = g.group / ntile;               // CTAs per KV head and query tile
+  const int nq = gridDim.y;
+  const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+  const int unit = lin / (gpp * nq), rem = lin - unit * (gpp * nq);   // unit = (r*B + b) * gl + KV head
+  const int mt = nq - 1 - rem / gpp;             // heaviest (latest) query tiles first
+  const int rb = unit / g.gl;
+  const int pp = (unit - rb * g.gl) * gpp + rem % gpp;   // head pair (or head) within the rank
   const int qhead0 = rb * g.hl + ntile * pp;     // tiles: qhead0 (, qhead0 + 1)
   const int kvhead = rb * g.gl + (ntile * pp) / g.group;
-  const int mt = gridDim.y - 1 - blockIdx.y;     // heaviest (latest) query tiles first
   const int m0 = mt * kBM;
 
   // KV tiles this query tile touches, and which of them need element masks.
