@@ -110,6 +110,7 @@ struct FusedParams {
   int n_pad;
   int *err;
   long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
+  int kv_major;          // block order: one KV head at a time (attn_kv_head_major)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -135,16 +136,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Blocks start in the order of their linear index (x fastest); that order
-  // walks the key tiles of one KV head at a time (earliest, so heaviest under
-  // a causal mask, first), so the CTAs in flight read the Q/dO rows and add
-  // into the dQ rows of one GQA group's heads, which stay in L2.
-  const int nk = gridDim.y;
-  const int lin = blockIdx.y * gridDim.x + blockIdx.x;
-  const int kvh = lin / nk;                      // (r*B + b)*gl + gg
-  const int rb = kvh / g.gl, gg = kvh - rb * g.gl;
+  // Blocks start in the order of their linear index (x fastest).  With
+  // kv_major that order walks the key tiles of one KV head at a time
+  // (earliest, so heaviest under a causal mask, first), so the CTAs in flight
+  // read the Q/dO rows and add into the dQ rows of one GQA group's heads,
+  // which stay in L2; without, it takes the earliest key tiles of every KV
+  // head first.
+  int kvh, kt;
+  if (prm.kv_major) {
+    const int nk = gridDim.y;
+    const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+    kvh = lin / nk;
+    kt = lin - kvh * nk;
+  } else {
+    kvh = blockIdx.x;
+    kt = blockIdx.y;
+  }
+  const int rb = kvh / g.gl, gg = kvh - rb * g.gl;   // kvh = (r*B + b)*gl + gg
   const int qh_base = rb * g.hl + gg * g.group;  // first query head of the group
-  const int n0 = (lin - kvh * nk) * kBN;
+  const int n0 = kt * kBN;
 
   // query rows that see any of the keys [n0, n0+127]
   int lo_a, hi_a, lo_b, hi_b;
@@ -517,6 +527,7 @@ uly_status attn_bf16_bwd_fused_launch(const HeadGeom &g, const MaskInfo &mk, con
   prm.n_pad = n_pad;
   prm.err = error_word();
   prm.wait_limit = wait_limit_cycles();
+  prm.kv_major = attn_kv_head_major(mk.mask, (g.n + kBN - 1) / kBN) ? 1 : 0;
   {
     prof::Scope scope(prof::K_ATTN_BWD_SM100, stream);
     attn_bwd_sm100_kernel<<<dim3(kvheads, (g.n + kBN - 1) / kBN), kThreads, kSmemBytes, stream>>>(mK, mV, mQ, mO,

@@ -68,6 +68,7 @@ struct FwdParams {
   float scale_log2;  // softmax scale * log2(e)
   int *err;          // device error word
   long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
+  int kv_major;          // block order: one KV head at a time (attn_kv_head_major)
 };
 
 template <int NTILE>
@@ -90,17 +91,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int ntile = NTILE;                   // query tiles (heads) per CTA: 2, or 1 for an odd group
-  // Blocks start in the order of their linear index (x fastest).  That
-  // order walks the CTAs of one KV head at a time (its gpp CTAs per query
-  // tile, heaviest query tiles first), so the CTAs in flight stream the K/V
-  // of one or two KV heads, which stay in L2, rather than of every head.
-  const int gpp = g.group / ntile;               // CTAs per KV head and query tile
-  const int nq = gridDim.y;
-  const int lin = blockIdx.y * gridDim.x + blockIdx.x;
-  const int unit = lin / (gpp * nq), rem = lin - unit * (gpp * nq);   // unit = (r*B + b) * gl + KV head
-  const int mt = nq - 1 - rem / gpp;             // heaviest (latest) query tiles first
-  const int rb = unit / g.gl;
-  const int pp = (unit - rb * g.gl) * gpp + rem % gpp;   // head pair (or head) within the rank
+  // Blocks start in the order of their linear index (x fastest).  With
+  // kv_major that order walks the CTAs of one KV head at a time (its gpp CTAs
+  // per query tile, heaviest query tiles first), so the CTAs in flight stream
+  // the K/V of one or two KV heads, which stay in L2; without, it takes the
+  // heaviest query tiles of every head first.
+  int rb, pp, mt;
+  if (prm.kv_major) {
+    const int gpp = g.group / ntile;             // CTAs per KV head and query tile
+    const int nq = gridDim.y;
+    const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+    const int unit = lin / (gpp * nq), rem = lin - unit * (gpp * nq);   // unit = (r*B + b) * gl + KV head
+    mt = nq - 1 - rem / gpp;
+    rb = unit / g.gl;
+    pp = (unit - rb * g.gl) * gpp + rem % gpp;   // head pair (or head) within the rank
+  } else {
+    const int per = g.hl / ntile;
+    rb = blockIdx.x / per;                       // blockIdx.x = (r*B + b) * per + pp
+    pp = blockIdx.x - rb * per;
+    mt = gridDim.y - 1 - blockIdx.y;
+  }
   const int qhead0 = rb * g.hl + ntile * pp;     // tiles: qhead0 (, qhead0 + 1)
   const int kvhead = rb * g.gl + (ntile * pp) / g.group;
   const int m0 = mt * kBM;
@@ -430,6 +440,7 @@ uly_status attn_bf16_fwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.err = error_word();
   prm.wait_limit = wait_limit_cycles();
   dim3 grid(g.P * g.B * (g.hl / ntile), (g.n + kBM - 1) / kBM);
+  prm.kv_major = attn_kv_head_major(mk.mask, (long long)grid.y * (g.group / ntile)) ? 1 : 0;
   prof::Scope scope(prof::K_ATTN_FWD_SM100, stream);
   if (ntile == 2)
     attn_fwd_sm100_kernel<2><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);

@@ -53,6 +53,28 @@ inline bool smem_optin(Kernel kernel, int bytes, std::atomic<uint64_t> &done) {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Streaming multiprocessors of the current device (148, a B200's count, if
+// the query fails).
+inline int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return 148;
+  return sms;
+}
+
+// Block order of the attention kernels.  Starting the CTAs of one KV head at
+// a time keeps the K/V (forward) or Q/dO and dQ rows (backward) of one GQA
+// group in L2; starting the heaviest tiles of every head first balances the
+// SMs' load best.  Under a causal mask the heaviest CTA does twice the
+// average, so taking the heads one at a time leaves no tail only when a
+// head's CTAs along the sequence are more than twice the SMs (64K tokens on
+// a B200: yes; 8K: no).  Document masks bound each CTA's work by its
+// document and gain little from the locality; they keep the balanced order.
+inline bool attn_kv_head_major(int mask, long long ctas_per_kv_head) {
+  return mask != ULY_MASK_DOC_CAUSAL && ctas_per_kv_head > 2LL * device_sm_count();
+}
+
 inline bool overlap(const void *a, size_t na, const void *b, size_t nb) {
   uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
