@@ -64,6 +64,7 @@ struct BwdParams {
   int n_pad;          // n rounded up to a multiple of 128
   int *err;
   long long wait_limit;  // cycles a pipeline wait may last (wait_limit_cycles())
+  int kv_major;       // block order: one KV head at a time (attn_kv_head_major)
 };
 
 // D_i = <dO_i, O_i> and LSE_i log2(e) of every query row (two rows per warp,
@@ -175,10 +176,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x;                    // (r*B + b)*gl + gg
-  const int rb = kvh / g.gl, gg = kvh - rb * g.gl;
+  // Blocks start in the order of their linear index (x fastest): with
+  // kv_major the key tiles of one KV head at a time, else those of every KV
+  // head side by side; earliest keys (heaviest) first either way.
+  int kvh, kt;
+  if (prm.kv_major) {
+    const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+    kvh = lin / gridDim.y;
+    kt = lin - kvh * gridDim.y;
+  } else {
+    kvh = blockIdx.x;
+    kt = blockIdx.y;
+  }
+  const int rb = kvh / g.gl, gg = kvh - rb * g.gl;   // kvh = (r*B + b)*gl + gg
   const int qh_base = rb * g.hl + gg * g.group;  // first query head of the group
-  const int n0 = blockIdx.y * kBN;               // earliest keys (heaviest) first
+  const int n0 = kt * kBN;
 
   // query rows that see any of the keys [n0, n0+127]
   int lo_a, hi_a, lo_b, hi_b;
@@ -468,10 +480,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const HeadGeom &g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qh = blockIdx.x;                     // (r*B + b)*hl + hh
-  const int rb = qh / g.hl, hh = qh - rb * g.hl;
+  // Blocks start in the order of their linear index (x fastest): with
+  // kv_major the query tiles of one GQA group's heads at a time (the group's
+  // heads side by side per tile), else those of every head side by side;
+  // heaviest (latest) query tiles first either way.
+  int rb, hh, mt;
+  if (prm.kv_major) {
+    const int nq = gridDim.y;
+    const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+    const int unit = lin / (g.group * nq), rem = lin - unit * (g.group * nq);   // unit = (r*B + b)*gl + KV head
+    mt = nq - 1 - rem / g.group;
+    rb = unit / g.gl;
+    hh = (unit - rb * g.gl) * g.group + rem % g.group;
+  } else {
+    const int qh = blockIdx.x;                   // (r*B + b)*hl + hh
+    rb = qh / g.hl;
+    hh = qh - rb * g.hl;
+    mt = gridDim.y - 1 - blockIdx.y;
+  }
+  const int qh = rb * g.hl + hh;
   const int kvhead = rb * g.gl + hh / g.group;
-  const int mt = gridDim.y - 1 - blockIdx.y;     // heaviest (latest) query tiles first
   const int m0 = mt * kBM;
 
   int lo_first, hi_first, lo_last, hi_last;
@@ -759,6 +787,7 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.out0 = static_cast<__nv_bfloat16 *>(dv);
   prm.out1 = static_cast<__nv_bfloat16 *>(dk);
   dim3 gkv(kvheads, (g.n + kv::kBN - 1) / kv::kBN);
+  prm.kv_major = attn_kv_head_major(mk.mask, gkv.y) ? 1 : 0;
   {
     prof::Scope scope(prof::K_ATTN_DKDV_SM100, stream);
     attn_dkdv_sm100_kernel<<<gkv, kThreads, kv::kSmemBytes, stream>>>(mK128, mV128, mQ128, mO128, prm);
@@ -766,6 +795,7 @@ uly_status attn_bf16_bwd_launch(const uly_attn_desc *d, const HeadGeom &g, const
   prm.out0 = static_cast<__nv_bfloat16 *>(dq);
   prm.out1 = nullptr;
   dim3 gq(qheads, (g.n + qk::kBM - 1) / qk::kBM);
+  prm.kv_major = attn_kv_head_major(mk.mask, (long long)gq.y * g.group) ? 1 : 0;
   {
     prof::Scope scope(prof::K_ATTN_DQ_SM100, stream);
     attn_dq_sm100_kernel<<<gq, kThreads, qk::kSmemBytes, stream>>>(mK128, mV128, prm);
