@@ -425,6 +425,24 @@ uly_status ulysses_read_error_info(int32_t *info, int32_t n);
  */
 uly_status ulysses_set_wait_limit(int64_t cycles);
 
+/*
+ * Block order of the attention kernels launched from now on (no counterpart
+ * on the pages; a scheduling choice that leaves every result unchanged).
+ * ULY_BLOCK_ORDER_AUTO (the default): the CTAs of one KV head start together
+ * (heaviest tiles first) when a KV head has more than twice as many CTAs along
+ * the sequence as the device has SMs and the mask is not a document mask, so
+ * that the CTAs in flight share one GQA group's K/V (forward) or Q/dO and dQ
+ * rows (backward) in L2; otherwise the heaviest tiles of every head start
+ * first, which balances few waves best.  ULY_BLOCK_ORDER_KV_HEAD_MAJOR and
+ * ULY_BLOCK_ORDER_HEAVIEST_FIRST fix one of the two, for tests that compare
+ * them.  O, LSE, dK, dV and the deterministic backward's dQ are bitwise the
+ * same under both; the fused backward's dQ varies at the fp32 rounding level
+ * from run to run under either.  Process-wide, host only.  Returns
+ * ULY_ERR_SHAPE for any other value.
+ */
+enum { ULY_BLOCK_ORDER_AUTO = 0, ULY_BLOCK_ORDER_KV_HEAD_MAJOR = 1, ULY_BLOCK_ORDER_HEAVIEST_FIRST = 2 };
+uly_status ulysses_set_attn_block_order(int32_t order);
+
 /* Human-readable name of a status. */
 const char *ulysses_status_string(uly_status status);
 

@@ -28,6 +28,12 @@ std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
 
+namespace {
+std::atomic<int> g_attn_block_order{ULY_BLOCK_ORDER_AUTO};
+}  // namespace
+
+int attn_block_order() { return g_attn_block_order.load(std::memory_order_relaxed); }
+
 int *error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
@@ -537,6 +543,14 @@ uly_status ulysses_set_wait_limit(int64_t cycles) {
   if (cycles < 0) return ULY_ERR_SHAPE;
   g_wait_limit.store(cycles == 0 || cycles > kDefaultWaitLimit ? kDefaultWaitLimit : cycles,
                      std::memory_order_relaxed);
+  return ULY_OK;
+}
+
+uly_status ulysses_set_attn_block_order(int32_t order) {
+  if (order != ULY_BLOCK_ORDER_AUTO && order != ULY_BLOCK_ORDER_KV_HEAD_MAJOR &&
+      order != ULY_BLOCK_ORDER_HEAVIEST_FIRST)
+    return ULY_ERR_SHAPE;
+  g_attn_block_order.store(order, std::memory_order_relaxed);
   return ULY_OK;
 }
 

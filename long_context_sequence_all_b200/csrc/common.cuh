@@ -30,6 +30,9 @@ void note_launches(int n);
 // ULY_ERR_TIMEOUT: the built-in limit, or a shorter one a test set with
 // ulysses_set_wait_limit (read by the launchers into the kernel parameters).
 long long wait_limit_cycles();
+// The attention kernels' block order set with ulysses_set_attn_block_order
+// (ULY_BLOCK_ORDER_*; read by the launchers).
+int attn_block_order();
 
 inline uly_status last_launch_status() {
   cudaError_t e = cudaGetLastError();
@@ -71,7 +74,13 @@ inline int device_sm_count() {
 // head's CTAs along the sequence are more than twice the SMs (64K tokens on
 // a B200: yes; 8K: no).  Document masks bound each CTA's work by its
 // document and gain little from the locality; they keep the balanced order.
+// ulysses_set_attn_block_order can fix either order (for tests that compare
+// them); the results do not depend on it (dQ of the fused backward aside,
+// whose fp32 adds meet in L2 in run-dependent order either way).
 inline bool attn_kv_head_major(int mask, long long ctas_per_kv_head) {
+  const int order = attn_block_order();
+  if (order == ULY_BLOCK_ORDER_KV_HEAD_MAJOR) return true;
+  if (order == ULY_BLOCK_ORDER_HEAVIEST_FIRST) return false;
   return mask != ULY_MASK_DOC_CAUSAL && ctas_per_kv_head > 2LL * device_sm_count();
 }
 

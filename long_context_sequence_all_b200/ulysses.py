@@ -31,7 +31,7 @@ EXPORTS = ["ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_seq_to_head_ba
            "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd", "ulysses_loss_workspace_size",
            "ulysses_loss_aggregate", "ulysses_loss_aggregate_noalloc", "ulysses_loss_bwd_workspace_size",
            "ulysses_loss_aggregate_bwd", "ulysses_read_error", "ulysses_read_error_info", "ulysses_error_word",
-           "ulysses_set_wait_limit",
+           "ulysses_set_wait_limit", "ulysses_set_attn_block_order",
            "ulysses_status_string", "ulysses_profile_enable", "ulysses_profile_read",
            "ulysses_kernel_count", "ulysses_kernel_name",
            "ulysses_launch_count"]
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
             L.ulysses_read_error_info.argtypes = [ctypes.POINTER(i32), i32]
             L.ulysses_set_wait_limit.argtypes = [i64]
             L.ulysses_set_wait_limit.restype = ctypes.c_int
+            L.ulysses_set_attn_block_order.argtypes = [ctypes.c_int32]
+            L.ulysses_set_attn_block_order.restype = ctypes.c_int
             L.ulysses_status_string.argtypes = [ctypes.c_int]
             L.ulysses_status_string.restype = ctypes.c_char_p
             L.ulysses_launch_count.restype = ctypes.c_uint64
@@ -520,6 +522,15 @@ def ulysses_set_wait_limit(cycles: int = 0):
     """Cycles a pipeline wait of the tcgen05 kernels may last before it reports
     ULY_ERR_TIMEOUT (0: the built-in limit).  For tests of the timeout path."""
     _check(lib().ulysses_set_wait_limit(int(cycles)), "ulysses_set_wait_limit")
+
+
+BLOCK_ORDER_AUTO, BLOCK_ORDER_KV_HEAD_MAJOR, BLOCK_ORDER_HEAVIEST_FIRST = 0, 1, 2
+
+
+def ulysses_set_attn_block_order(order: int = BLOCK_ORDER_AUTO):
+    """Block order of the attention kernels (BLOCK_ORDER_*; the default picks
+    per launch).  The results do not depend on it; for tests that compare."""
+    _check(lib().ulysses_set_attn_block_order(int(order)), "ulysses_set_attn_block_order")
 
 
 def ulysses_status_string(status: int) -> str:

@@ -232,3 +232,15 @@ def test_loss_gradient_validation(L):
 
 def test_error_word_null_argument(L):
     assert L.ulysses_error_word(None) == 1
+
+
+def test_attn_block_order_setter_validates(L):
+    """ulysses_set_attn_block_order takes the three ULY_BLOCK_ORDER_* values
+    and rejects anything else with ULY_ERR_SHAPE (no device work)."""
+    try:
+        for order in (1, 2, 0):
+            assert L.ulysses_set_attn_block_order(order) == 0
+        for bad in (-1, 3, 100):
+            assert L.ulysses_set_attn_block_order(bad) == 2
+    finally:
+        L.ulysses_set_attn_block_order(0)

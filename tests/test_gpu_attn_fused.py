@@ -142,3 +142,38 @@ def test_malformed_cu_seqlens_sets_shape_error():
     good = torch.tensor([0, 100, 256], dtype=torch.int32, device="cuda")
     U.ulysses_attn_fwd(qh, kh, vh, mask=U.MASK_DOC_CAUSAL, cu_seqlens=good)
     assert U.ulysses_read_error() == 0
+
+
+@pytest.mark.parametrize("n,P,H,G,mask,cu", [
+    (4096, 4, 32, 8, U.MASK_CAUSAL, None),      # 32 query tiles, 8 KV heads: several waves either way
+    (1000, 8, 16, 8, U.MASK_DOC_CAUSAL, [0, 100, 129, 400, 401, 777, 1000]),
+    (392, 4, 8, 4, U.MASK_NONE, None),
+    (424, 2, 6, 2, U.MASK_CAUSAL, None),        # an odd group: one query head per forward CTA
+])
+def test_block_orders_give_the_same_results(n, P, H, G, mask, cu):
+    """The attention kernels start their CTAs one KV head at a time (long
+    sequences) or with the heaviest tiles of every head first (short ones,
+    document masks); the order is scheduling only.  With each order forced:
+    O, LSE, dK, dV and the deterministic dQ are bitwise equal, the fused dQ
+    (fp32 adds meeting in L2 in run-dependent order) to one bf16 rounding."""
+    q, k, v, do = _case(n, P, H, G, seed=n + 17)
+    cud = None if cu is None else torch.tensor(cu, dtype=torch.int32).cuda()
+    qh, kh, vh, doh = _heads(q, k, v, do, P)
+    res = {}
+    try:
+        for order in (U.BLOCK_ORDER_KV_HEAD_MAJOR, U.BLOCK_ORDER_HEAVIEST_FIRST):
+            U.ulysses_set_attn_block_order(order)
+            oh, lse = U.ulysses_attn_fwd(qh, kh, vh, mask=mask, cu_seqlens=cud)
+            fused = U.ulysses_attn_bwd(qh, kh, vh, oh, lse, doh, mask=mask, cu_seqlens=cud)
+            det = U.ulysses_attn_bwd(qh, kh, vh, oh, lse, doh, mask=mask, cu_seqlens=cud, deterministic=True)
+            torch.cuda.synchronize()
+            res[order] = (oh, lse, fused, det)
+    finally:
+        U.ulysses_set_attn_block_order(U.BLOCK_ORDER_AUTO)
+    (o1, l1, f1, d1), (o2, l2, f2, d2) = res[U.BLOCK_ORDER_KV_HEAD_MAJOR], res[U.BLOCK_ORDER_HEAVIEST_FIRST]
+    assert torch.equal(o1, o2) and torch.equal(l1, l2), "forward differs between the block orders"
+    assert all(torch.equal(a, b) for a, b in zip(d1, d2)), "deterministic backward differs"
+    assert torch.equal(f1[1], f2[1]) and torch.equal(f1[2], f2[2]), "fused dK / dV differ"
+    a, b = f1[0].float().cpu(), f2[0].float().cpu()
+    assert float(((a - b).abs() / (2.0 ** -7 * torch.maximum(a.abs(), b.abs()) + 1e-6)).max()) <= 1.0
+    assert U.ulysses_read_error() == 0
